@@ -1,0 +1,355 @@
+/*
+ * rb_oracle.c -- plain, slow, obviously-correct CPU oracle for the residual
+ * dual-scale binarized linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the test-suite, the smoke check and the CPU-baseline
+ * leg of the benchmark use it.  It shares no code, header, table or constant
+ * with the CUDA library.
+ *
+ * Method (RaBiT: Residual-Aware Binarization Training, "Residual binarization"
+ * and "Core method" sections; Algorithm 2, forward pass):
+ *   W ~= sum_{i=1..k} diag(g_i) B_i diag(h_i),  B_i in {-1,+1}^{N x K}
+ *   R_0 = W;  B_i = sign(R_{i-1}) with sign(0) = +1;
+ *   R_i = R_{i-1} - (g_i h_i^T) .* B_i
+ *   Y = sum_i g_i .* (B_i (h_i .* X))      ("matmul-free" evaluation)
+ *
+ * Readings taken where the pages leave a step open (each is listed in the
+ * design notes):
+ *   - the residual update runs in IEEE fp32: t = fl(g_i[r]*h_i[c]) (one
+ *     rounding), then R = fl(R - t) if B = +1 else fl(R + t); no fused
+ *     multiply-add.  The fp32 scales given by the caller are used, not their
+ *     fp16 copies.
+ *   - sign(0) = +1 includes -0.0 (the test is R >= 0); this is the tie rule of
+ *     the binary-codebook page (BTC-LLM, binary k-means M-step: a zero
+ *     centroid entry becomes +1).
+ *   - bit = 1 <=> B = +1; 32 consecutive input columns per uint32 word with
+ *     column c at bit c % 32 ("32 columns packed into one uint32_t", RaBiT,
+ *     technical novelty paragraph).
+ *   - word order (the storage layout):  plane i is cut into S = ceil(K/256)
+ *     column slices; rows are grouped in quads (Nq = ceil(N/4));
+ *        word(i, s, r, w) = (((i*S + s)*Nq + r/4)*8 + w)*4 + r%4
+ *     holds columns 256*s + 32*w .. +31 of row r.  Bits of columns >= K and
+ *     words of rows >= N are zero.
+ *   - stored scales are fp16, rounded to nearest-even from the fp32 inputs.
+ *   - the greedy SVID initialiser (Greedy SVID, named in the technical
+ *     novelty paragraph) takes, per plane, the rank-1 approximation of
+ *     |R_{i-1}| by power iteration in float64: v0 = 1/sqrt(K), then `iters`
+ *     rounds of u = A v / |A v|, v = A^T u / |A^T u|; sigma = u^T A v;
+ *     g_i = fp32(sqrt(sigma) u), h_i = fp32(sqrt(sigma) v).
+ *
+ * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC (no fast-math);
+ * on x86-64 float arithmetic is SSE single precision, so every fp32 step
+ * above rounds exactly once.
+ */
+#include <math.h>
+#include <omp.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ */
+/* Number formats (IEEE 754 binary16, bfloat16), round-to-nearest-even */
+/* ------------------------------------------------------------------ */
+
+/* Round a double to a binary format with p significand bits (implicit bit
+ * included), minimum normal exponent emin and maximum exponent emax.
+ * Subnormals keep the fixed quantum 2^(emin-p+1); results that round to
+ * 2^(emax+1) or above overflow to infinity. */
+static double round_to_format(double v, int p, int emin, int emax)
+{
+    if (v != v || isinf(v) || v == 0.0) return v;
+    double a = fabs(v);
+    int e;
+    frexp(a, &e);           /* a = f * 2^e, f in [0.5, 1): floor(log2 a) = e-1 */
+    int E = e - 1;
+    if (E < emin) E = emin;
+    double q = ldexp(1.0, E - p + 1);
+    double r = rint(a / q) * q;          /* a/q is exact; rint rounds half to even */
+    if (r >= ldexp(1.0, emax + 1)) r = INFINITY;
+    return copysign(r, v);
+}
+
+static uint16_t encode_binary16(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    if (v != v) return 0x7e00u;
+    double r = round_to_format(v, 11, -14, 15);
+    double a = fabs(r);
+    if (isinf(a)) return sign | 0x7c00u;
+    if (a == 0.0) return sign;
+    if (a < ldexp(1.0, -14))                       /* subnormal: m * 2^-24 */
+        return sign | (uint16_t)(a / ldexp(1.0, -24));
+    int e;
+    frexp(a, &e);
+    int E = e - 1;
+    uint32_t mant = (uint32_t)(a / ldexp(1.0, E - 10)) - 1024u;
+    return sign | (uint16_t)(((uint32_t)(E + 15) << 10) | mant);
+}
+
+static double decode_binary16(uint16_t b)
+{
+    int sign = (b >> 15) & 1, ex = (b >> 10) & 31, m = b & 1023;
+    double v;
+    if (ex == 31) v = m ? NAN : INFINITY;
+    else if (ex == 0) v = ldexp((double)m, -24);
+    else v = ldexp((double)(1024 + m), ex - 25);
+    return sign ? -v : v;
+}
+
+static uint16_t encode_bfloat16(double v)
+{
+    if (v != v) return 0x7fc0u;
+    double r = round_to_format(v, 8, -126, 127);
+    float f = (float)r;                 /* exact: every bfloat16 value is a float */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(u >> 16);
+}
+
+static double decode_bfloat16(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+uint16_t oracle_f64_to_f16(double v) { return encode_binary16(v); }
+double oracle_f16_to_f64(uint16_t b) { return decode_binary16(b); }
+uint16_t oracle_f64_to_bf16(double v) { return encode_bfloat16(v); }
+double oracle_bf16_to_f64(uint16_t b) { return decode_bfloat16(b); }
+
+/* ------------------------------------------------------------------ */
+/* Storage layout                                                       */
+/* ------------------------------------------------------------------ */
+
+int64_t oracle_plane_words(int64_t N, int64_t K, int k)
+{
+    int64_t S = (K + 255) / 256, Nq = (N + 3) / 4;
+    return (int64_t)k * S * Nq * 32;
+}
+
+static int64_t word_index(int64_t N, int64_t K, int i, int64_t r, int64_t c)
+{
+    int64_t S = (K + 255) / 256, Nq = (N + 3) / 4;
+    int64_t s = c / 256, w = (c % 256) / 32;
+    return ((((int64_t)i * S + s) * Nq + r / 4) * 8 + w) * 4 + r % 4;
+}
+
+/* ------------------------------------------------------------------ */
+/* Derivation + packing (Algorithm 2 forward, fp32 recurrence)          */
+/* ------------------------------------------------------------------ */
+
+/* Return codes: 0 ok, -1 bad argument, 1 non-finite W/g/h, 2 a scale
+ * overflows fp16. Outputs are written in all non-negative-error cases. */
+static int check_args(int64_t N, int64_t K, int k)
+{
+    if (N < 1 || K < 32 || K % 32 != 0 || k < 1 || k > 8) return -1;
+    return 0;
+}
+
+/* Derive and pack one row r (row-local residual, length K). bits_out gets
+ * the k*K bits of the row in [i][c] order (1 = +1). */
+static void derive_row(const float *Wr, const float *g, const float *h,
+                       int64_t N, int64_t K, int k, int64_t r,
+                       float *R, unsigned char *bits_out)
+{
+    for (int64_t c = 0; c < K; ++c) R[c] = Wr[c];
+    for (int i = 0; i < k; ++i) {
+        float gi = g[(int64_t)i * N + r];
+        for (int64_t c = 0; c < K; ++c) {
+            int b = (R[c] >= 0.0f);             /* sign(0) = +1, -0.0 included */
+            float t = gi * h[(int64_t)i * K + c];   /* one fp32 rounding */
+            R[c] = b ? (R[c] - t) : (R[c] + t);     /* a second, separate rounding */
+            bits_out[(int64_t)i * K + c] = (unsigned char)b;
+        }
+    }
+}
+
+static int scan_inputs(const float *W, const float *g, const float *h,
+                       int64_t N, int64_t K, int k, uint16_t *g16, uint16_t *h16)
+{
+    int st = 0;
+    for (int64_t x = 0; x < N * K; ++x)
+        if (!isfinite(W[x])) st = 1;
+    for (int64_t x = 0; x < (int64_t)k * N; ++x) {
+        if (!isfinite(g[x])) st = 1;
+        uint16_t e = encode_binary16((double)g[x]);
+        if (isfinite(g[x]) && (e & 0x7c00u) == 0x7c00u && st == 0) st = 2;
+        if (g16) g16[x] = e;
+    }
+    for (int64_t x = 0; x < (int64_t)k * K; ++x) {
+        if (!isfinite(h[x])) st = 1;
+        uint16_t e = encode_binary16((double)h[x]);
+        if (isfinite(h[x]) && (e & 0x7c00u) == 0x7c00u && st == 0) st = 2;
+        if (h16) h16[x] = e;
+    }
+    return st;
+}
+
+/* Full pack. planes has oracle_plane_words(N,K,k) words. R_out (nullable,
+ * [N][K]) receives the final residual R_k. */
+int oracle_pack(const float *W, const float *g, const float *h,
+                int64_t N, int64_t K, int k,
+                uint32_t *planes, uint16_t *g16, uint16_t *h16, float *R_out)
+{
+    if (check_args(N, K, k)) return -1;
+    int st = scan_inputs(W, g, h, N, K, k, g16, h16);
+    memset(planes, 0, sizeof(uint32_t) * (size_t)oracle_plane_words(N, K, k));
+    #pragma omp parallel
+    {
+        float *R = (float *)malloc(sizeof(float) * (size_t)K);
+        unsigned char *bits = (unsigned char *)malloc((size_t)k * (size_t)K);
+        #pragma omp for schedule(static)
+        for (int64_t r = 0; r < N; ++r) {
+            derive_row(W + r * K, g, h, N, K, k, r, R, bits);
+            for (int i = 0; i < k; ++i)
+                for (int64_t c = 0; c < K; ++c)
+                    if (bits[(int64_t)i * K + c])
+                        planes[word_index(N, K, i, r, c)] |= (uint32_t)1u << (c % 32);
+            if (R_out) memcpy(R_out + r * K, R, sizeof(float) * (size_t)K);
+        }
+        free(R);
+        free(bits);
+    }
+    return st;
+}
+
+/* Pack only the listed rows (for sampled checks at full size). Output is
+ * row-local: words_out[j][i][s][w] for the j-th listed row, S = ceil(K/256). */
+int oracle_pack_rows(const float *W, const float *g, const float *h,
+                     int64_t N, int64_t K, int k,
+                     const int64_t *rows, int64_t nrows, uint32_t *words_out)
+{
+    if (check_args(N, K, k)) return -1;
+    int64_t S = (K + 255) / 256;
+    memset(words_out, 0, sizeof(uint32_t) * (size_t)(nrows * k * S * 8));
+    float *R = (float *)malloc(sizeof(float) * (size_t)K);
+    unsigned char *bits = (unsigned char *)malloc((size_t)k * (size_t)K);
+    for (int64_t j = 0; j < nrows; ++j) {
+        int64_t r = rows[j];
+        derive_row(W + r * K, g, h, N, K, k, r, R, bits);
+        for (int i = 0; i < k; ++i)
+            for (int64_t c = 0; c < K; ++c)
+                if (bits[(int64_t)i * K + c])
+                    words_out[((j * k + i) * S + c / 256) * 8 + (c % 256) / 32] |=
+                        (uint32_t)1u << (c % 32);
+    }
+    free(R);
+    free(bits);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Application: dequantise the stored representation, then multiply      */
+/* ------------------------------------------------------------------ */
+
+/* Y[m][n] = sum_c X[m][c] * What[n][c] in float64 with
+ * What[n][c] = sum_i f16(g16_i[n]) * (bit ? +1 : -1) * f16(h16_i[c]).
+ * rows / toks (nullable) select the outputs; Y is [ntoks][nrows]. */
+void oracle_apply(const uint32_t *planes, const uint16_t *g16, const uint16_t *h16,
+                  int64_t N, int64_t K, int k,
+                  const uint16_t *X, int64_t M,
+                  const int64_t *rows, int64_t nrows,
+                  const int64_t *toks, int64_t ntoks, double *Y)
+{
+    if (!rows) nrows = N;
+    if (!toks) ntoks = M;
+    double *hd = (double *)malloc(sizeof(double) * (size_t)(k * K));
+    for (int64_t x = 0; x < (int64_t)k * K; ++x) hd[x] = decode_binary16(h16[x]);
+    #pragma omp parallel
+    {
+        double *What = (double *)malloc(sizeof(double) * (size_t)K);
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t j = 0; j < nrows; ++j) {
+            int64_t n = rows ? rows[j] : j;
+            for (int64_t c = 0; c < K; ++c) What[c] = 0.0;
+            for (int i = 0; i < k; ++i) {
+                double gi = decode_binary16(g16[(int64_t)i * N + n]);
+                for (int64_t c = 0; c < K; ++c) {
+                    uint32_t word = planes[word_index(N, K, i, n, c)];
+                    double s = ((word >> (c % 32)) & 1u) ? 1.0 : -1.0;
+                    What[c] += gi * s * hd[(int64_t)i * K + c];
+                }
+            }
+            for (int64_t t = 0; t < ntoks; ++t) {
+                int64_t m = toks ? toks[t] : t;
+                double acc = 0.0;
+                for (int64_t c = 0; c < K; ++c)
+                    acc += decode_bfloat16(X[m * K + c]) * What[c];
+                Y[t * nrows + j] = acc;
+            }
+        }
+        free(What);
+    }
+    free(hd);
+}
+
+/* ------------------------------------------------------------------ */
+/* Greedy SVID scales (rank-1 of |R_{i-1}| per plane, power iteration)   */
+/* ------------------------------------------------------------------ */
+
+int oracle_svid_greedy(const float *W, int64_t N, int64_t K, int k, int iters,
+                       float *g, float *h)
+{
+    if (check_args(N, K, k) || iters < 1) return -1;
+    float *R = (float *)malloc(sizeof(float) * (size_t)(N * K));
+    double *u = (double *)malloc(sizeof(double) * (size_t)N);
+    double *v = (double *)malloc(sizeof(double) * (size_t)K);
+    if (!R || !u || !v) { free(R); free(u); free(v); return -1; }
+    memcpy(R, W, sizeof(float) * (size_t)(N * K));
+
+    for (int i = 0; i < k; ++i) {
+        for (int64_t c = 0; c < K; ++c) v[c] = 1.0 / sqrt((double)K);
+        for (int t = 0; t < iters; ++t) {
+            double nu = 0.0, nv = 0.0;
+            #pragma omp parallel for schedule(static)
+            for (int64_t r = 0; r < N; ++r) {          /* u = A v */
+                double acc = 0.0;
+                for (int64_t c = 0; c < K; ++c) acc += fabs((double)R[r * K + c]) * v[c];
+                u[r] = acc;
+            }
+            for (int64_t r = 0; r < N; ++r) nu += u[r] * u[r];
+            nu = sqrt(nu);
+            for (int64_t r = 0; r < N; ++r) u[r] = nu > 0.0 ? u[r] / nu : 0.0;
+            #pragma omp parallel
+            {                                          /* v = A^T u, rows in order */
+                int nt = omp_get_num_threads(), tid = omp_get_thread_num();
+                int64_t c0 = K * tid / nt, c1 = K * (tid + 1) / nt;
+                for (int64_t c = c0; c < c1; ++c) v[c] = 0.0;
+                for (int64_t r = 0; r < N; ++r) {
+                    double ur = u[r];
+                    for (int64_t c = c0; c < c1; ++c) v[c] += fabs((double)R[r * K + c]) * ur;
+                }
+            }
+            for (int64_t c = 0; c < K; ++c) nv += v[c] * v[c];
+            nv = sqrt(nv);
+            for (int64_t c = 0; c < K; ++c) v[c] = nv > 0.0 ? v[c] / nv : 0.0;
+        }
+        double sigma = 0.0;                            /* sigma = u^T A v */
+        for (int64_t r = 0; r < N; ++r) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < K; ++c) acc += fabs((double)R[r * K + c]) * v[c];
+            sigma += u[r] * acc;
+        }
+        double rs = sigma > 0.0 ? sqrt(sigma) : 0.0;
+        for (int64_t r = 0; r < N; ++r) g[(int64_t)i * N + r] = (float)(rs * u[r]);
+        for (int64_t c = 0; c < K; ++c) h[(int64_t)i * K + c] = (float)(rs * v[c]);
+        /* R_i from R_{i-1}: same fp32 recurrence as the packer */
+        #pragma omp parallel for schedule(static)
+        for (int64_t r = 0; r < N; ++r) {
+            float gi = g[(int64_t)i * N + r];
+            for (int64_t c = 0; c < K; ++c) {
+                float Rv = R[r * K + c];
+                int b = (Rv >= 0.0f);
+                float tt = gi * h[(int64_t)i * K + c];
+                R[r * K + c] = b ? (Rv - tt) : (Rv + tt);
+            }
+        }
+    }
+    free(R);
+    free(u);
+    free(v);
+    return 0;
+}

@@ -1,0 +1,284 @@
+"""Pins of the CPU oracle against facts fixed outside the oracle itself.
+
+Each test names the passage or the mathematical fact it rests on:
+  * RaBiT "Residual binarization": W ~= sum_i g_i . B_i . h_i, B_i in {-1,+1}.
+  * RaBiT Algorithm 2 forward: R_0 = W, B_i = sign(R_{i-1}), R_i = R_{i-1} - W_i.
+  * BTC-LLM, binary k-means M-step: a zero entry takes the sign +1.
+  * BTC-LLM, "bit-compressed computation": the +-1 dot product equals
+    n - 2*popcount(a XOR b) on packed vectors.
+  * RaBiT, limitations paragraph: 2.02 effective bits per weight at k = 2.
+No expected value here is computed by the CUDA library.
+"""
+import fractions
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from residual_binarized_weight_b200 import synth
+from tests import layout
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16_to_f64(bits):
+    return torch.from_numpy(np.asarray(bits, np.uint16).view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
+# ---------------------------------------------------------------- number formats
+
+def test_f16_encoder_matches_numpy_float16():
+    """The fp16 scale cast is IEEE binary16 round-to-nearest-even (numpy's astype)."""
+    rng = np.random.default_rng(1)
+    vals = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.uniform(-9, 5, 20000),
+        np.array([0.0, -0.0, 65504.0, 65519.99, 65520.0, -65520.0, 1e-8, 2.0 ** -24,
+                  2.0 ** -25, 3 * 2.0 ** -26, 2.0 ** -14, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11,
+                  np.inf, -np.inf]),
+    ]).astype(np.float32)
+    want = vals.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.f64_to_f16_bits(float(v)) for v in vals], np.uint16)
+    assert np.array_equal(got, want)
+    back = np.array([oracle.f16_bits_to_f64(int(b)) for b in want[:2000]])
+    assert np.array_equal(back, want[:2000].view(np.float16).astype(np.float64))
+
+
+def test_bf16_encoder_matches_torch():
+    """bfloat16 outputs are round-to-nearest-even of the exact value (torch's cast)."""
+    rng = np.random.default_rng(2)
+    vals = (rng.standard_normal(20000) * 10.0 ** rng.uniform(-30, 30, 20000)).astype(np.float32)
+    vals = np.concatenate([vals, np.float32([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -0.0, 3e38])])
+    want = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle.f64_to_bf16_bits(float(v)) for v in vals], np.uint16)
+    assert np.array_equal(got, want)
+    assert np.array_equal(np.array([oracle.bf16_bits_to_f64(int(b)) for b in want]), bf16_to_f64(want))
+
+
+# ---------------------------------------------------------------- layout, polarity, sign(0)
+
+@pytest.mark.parametrize("N,K", [(8, 256), (6, 96), (13, 544), (4, 32)])
+def test_k1_planes_are_sign_of_w(N, K):
+    """k = 1: B_1 = sign(W) with sign(0) = +1 (zeros and -0.0 give bit 1)."""
+    rng = np.random.default_rng(N * 1000 + K)
+    W = rng.standard_normal((N, K)).astype(np.float32)
+    W[0, :5] = [0.0, -0.0, 0.0, -0.0, 0.0]
+    W[-1, -3:] = -0.0
+    g = np.ones((1, N), np.float32)
+    h = np.ones((1, K), np.float32)
+    planes, g16, h16, st, _ = oracle.pack(W, g, h, 1)
+    assert st == 0
+    want = layout.pack_bits((W >= 0)[None])           # np.packbits in the stated layout
+    assert np.array_equal(planes, want)
+    assert not layout.padding_words_and_bits(planes, N, K, 1).any()
+    assert np.all(g16 == 0x3C00) and np.all(h16 == 0x3C00)
+
+
+def test_k1_unit_scales_apply_is_sign_matvec():
+    """k = 1, g = h = 1: Y = X . sign(W)^T, a textbook matrix product (numpy)."""
+    rng = np.random.default_rng(3)
+    N, K, M = 40, 320, 3
+    W = rng.standard_normal((N, K)).astype(np.float32)
+    X = synth.activations(M, K, seed=9)
+    planes, g16, h16, st, _ = oracle.pack(W, np.ones((1, N), np.float32), np.ones((1, K), np.float32), 1)
+    Y = oracle.apply(planes, g16, h16, N, K, 1, X)
+    S = np.where(W >= 0, 1.0, -1.0)
+    want = bf16_to_f64(X) @ S.T
+    np.testing.assert_allclose(Y, want, rtol=1e-12, atol=1e-12)
+
+
+def test_popcount_identity():
+    """+-1 dot = K - 2*popcount(a XOR b) on packed words (BTC-LLM Hamming step)."""
+    rng = np.random.default_rng(4)
+    N, K = 16, 512
+    W = rng.standard_normal((N, K)).astype(np.float32)
+    xs = np.where(rng.standard_normal(K) >= 0, 1.0, -1.0).astype(np.float32)
+    X = synth.to_bf16_bits(xs[None])
+    planes, g16, h16, _, _ = oracle.pack(W, np.ones((1, N), np.float32), np.ones((1, K), np.float32), 1)
+    Y = oracle.apply(planes, g16, h16, N, K, 1, X)[0]
+    xw = np.packbits(xs >= 0, bitorder="little").view("<u4")
+    rows = layout.gather_rows(planes, N, K, 1, np.arange(N)).reshape(N, -1)
+    for r in range(N):
+        ham = sum(bin(int(a) ^ int(b)).count("1") for a, b in zip(rows[r], xw))
+        assert Y[r] == K - 2 * ham
+
+
+# ---------------------------------------------------------------- derivation
+
+def _brute_best(R, T):
+    """All B in {-1,+1}^{shape} minimising ||R - T.*B||_F (exhaustive)."""
+    n = R.size
+    best, arg = None, []
+    for bits in itertools.product([1.0, -1.0], repeat=n):
+        B = np.array(bits).reshape(R.shape)
+        e = float(np.sum((R.astype(np.float64) - T * B) ** 2))
+        if best is None or e < best - 1e-300:
+            best, arg = e, [B]
+        elif e == best:
+            arg.append(B)
+    return arg
+
+
+@pytest.mark.parametrize("shape,seed", [((2, 32), 5), ((3, 32), 6)])
+def test_plane_is_least_squares_sign_brute_force(shape, seed):
+    """sign(R) minimises ||R - (g h^T).*B|| over all B (exhaustive over a 2x4/3x4 block);
+    exact zeros are ties and take +1."""
+    rng = np.random.default_rng(seed)
+    N, K = shape
+    W = rng.standard_normal((N, K)).astype(np.float32)
+    W[0, 1] = 0.0
+    W[1, 2] = -0.0
+    g, h = synth.positive_scales(2, N, K, seed)
+    planes2, _, _, _, _ = oracle.pack(W, g, h, 2)
+    _, _, _, _, R1 = oracle.pack(W, g[:1], h[:1], 1, want_residual=True)
+    Bs = np.where(layout.unpack_bits(planes2, N, K, 2), 1.0, -1.0)
+    for i, Rprev in ((0, W), (1, R1)):
+        T = np.outer(g[i], h[i]).astype(np.float64)
+        blk = (slice(0, N), slice(0, 4))            # 2^(N*4) candidates
+        cands = _brute_best(Rprev[blk], T[blk])
+        assert any(np.array_equal(Bs[i][blk], c) for c in cands)
+        if len(cands) > 1:                           # ties only at exact zeros -> +1
+            zero = Rprev[blk] == 0
+            assert np.all(Bs[i][blk][zero] == 1.0)
+    assert Bs[0][0, 1] == 1.0 and Bs[0][1, 2] == 1.0
+
+
+def test_residual_equals_w_minus_reconstruction():
+    """R_k = W - sum_i g_i . B_i . h_i up to the fp32 roundings of the recurrence."""
+    rng = np.random.default_rng(7)
+    N, K, k = 24, 288, 3
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k)
+    planes, _, _, st, R = oracle.pack(W, g, h, k, want_residual=True)
+    assert st == 0
+    B = np.where(layout.unpack_bits(planes, N, K, k), 1.0, -1.0)
+    recon = sum(np.outer(g[i], h[i]).astype(np.float64) * B[i] for i in range(k))
+    err = np.abs(R.astype(np.float64) - (W.astype(np.float64) - recon))
+    bound = 2 * k * 2.0 ** -24 * (np.abs(W) + sum(np.outer(g[i], h[i]) for i in range(k)) * 2)
+    assert np.all(err <= bound)
+
+
+def test_no_fused_multiply_add_in_recurrence():
+    """g*h is rounded to fp32 before the subtraction (worked by hand):
+    g = h = 1 + 2^-12 -> fl(g*h) = 1 + 2^-11 (tie to even drops 2^-24);
+    W = 1 + 2^-11 + 2^-23 -> R_1 = 2^-23 exactly (a fused form would give 2^-24)."""
+    g = np.float32([[1.0 + 2.0 ** -12]])
+    h = np.full((1, 32), 1.0 + 2.0 ** -12, np.float32)
+    W = np.full((1, 32), 1.0 + 2.0 ** -11 + 2.0 ** -23, np.float32)
+    _, _, _, st, R = oracle.pack(W, g, h, 1, want_residual=True)
+    assert st == 0
+    assert np.all(R == np.float32(2.0 ** -23))
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4])
+def test_residual_norm_non_increasing(k):
+    """||R_i||_F <= ||R_{i-1}||_F for rank-1 least-squares scales: |R_i| = | |R_{i-1}| - g h^T |
+    and ||A - sigma u v^T||^2 = ||A||^2 - sigma^2 for sigma = u^T A v (any unit u, v)."""
+    wl = synth.workload(1)
+    W = synth.weights(wl.layers[0], 96, 512)
+    g, h = oracle.svid_greedy(W, k)
+    norms = [float(np.linalg.norm(W.astype(np.float64)))]
+    for i in range(1, k + 1):
+        _, _, _, _, R = oracle.pack(W, g[:i], h[:i], i, want_residual=True)
+        norms.append(float(np.linalg.norm(R.astype(np.float64))))
+    for a, b in zip(norms, norms[1:]):
+        assert b <= a * (1 + 1e-6)
+    assert norms[-1] < norms[0]
+
+
+def test_svid_plane1_is_top_singular_pair_of_abs_w():
+    """Plane-1 greedy SVID scales reproduce the top singular triple of |W| (numpy SVD)."""
+    wl = synth.workload(0)
+    W = synth.weights(wl.layers[0])
+    g, h = oracle.svid_greedy(W, 1, iters=20)
+    U, s, Vt = np.linalg.svd(np.abs(W.astype(np.float64)), full_matrices=False)
+    ref = s[0] * np.outer(U[:, 0], Vt[0])
+    ref *= np.sign(ref.sum())
+    got = np.outer(g[0], h[0]).astype(np.float64)
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 1e-4
+    assert np.all(g >= 0) and np.all(h >= 0)
+
+
+def test_zero_weight_degenerate():
+    """W = 0: every plane is all +1 (sign(0) = +1), greedy scales are 0, R stays 0."""
+    N, K = 8, 64
+    W = np.zeros((N, K), np.float32)
+    g, h = oracle.svid_greedy(W, 2)
+    assert np.all(g == 0) and np.all(h == 0)
+    planes, _, _, st, R = oracle.pack(W, g, h, 2, want_residual=True)
+    assert st == 0 and np.all(R == 0)
+    assert layout.unpack_bits(planes, N, K, 2).all()
+
+
+def test_bad_inputs_status():
+    W = np.ones((4, 64), np.float32)
+    g = np.ones((1, 4), np.float32)
+    h = np.ones((1, 64), np.float32)
+    W2 = W.copy()
+    W2[1, 3] = np.nan
+    assert oracle.pack(W2, g, h, 1)[3] == 1
+    g2 = g.copy()
+    g2[0, 0] = 70000.0
+    assert oracle.pack(W, g2, h, 1)[3] == 2
+    assert oracle.pack(np.ones((4, 48), np.float32), g, np.ones((1, 48), np.float32), 1)[3] == -1
+
+
+# ---------------------------------------------------------------- application
+
+def test_apply_equals_exact_matmul_free_form():
+    """The dequantise-then-multiply oracle equals the matmul-free form
+    Y = sum_i g_i . (B_i (h_i . x)) evaluated in exact rational arithmetic."""
+    rng = np.random.default_rng(8)
+    N, K, k, M = 5, 64, 2, 2
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    X = synth.activations(M, K, seed=11)
+    Y = oracle.apply(planes, g16, h16, N, K, k, X)
+    B = layout.unpack_bits(planes, N, K, k)
+    F = fractions.Fraction
+    gq = g16.view(np.float16).astype(np.float64)
+    hq = h16.view(np.float16).astype(np.float64)
+    xq = bf16_to_f64(X)
+    for m in range(M):
+        for n in range(N):
+            tot = F(0)
+            for i in range(k):
+                acc = F(0)
+                for c in range(K):
+                    hx = F(hq[i, c]) * F(xq[m, c])
+                    acc += hx if B[i, n, c] else -hx
+                tot += F(gq[i, n]) * acc
+            assert math.isclose(Y[m, n], float(tot), rel_tol=1e-12, abs_tol=1e-15)
+
+
+def test_apply_row_and_token_subsets():
+    rng = np.random.default_rng(10)
+    N, K, k, M = 12, 256, 2, 4
+    W = rng.standard_normal((N, K)).astype(np.float32)
+    g, h = synth.positive_scales(k, N, K, 3)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    X = synth.activations(M, K, seed=1)
+    full = oracle.apply(planes, g16, h16, N, K, k, X)
+    rows, toks = [11, 0, 5], [3, 1]
+    sub = oracle.apply(planes, g16, h16, N, K, k, X, rows=rows, toks=toks)
+    assert np.array_equal(sub, full[np.ix_(toks, rows)])
+    packed_rows = oracle.pack_rows(W, g, h, k, rows)
+    assert np.array_equal(packed_rows, layout.gather_rows(planes, N, K, k, rows))
+
+
+# ---------------------------------------------------------------- sizes
+
+def test_effective_bits_matches_page():
+    """Stored bits per weight at 4096 x 4096, k = 2 with fp16 g, h (RaBiT: 2.02)."""
+    with open(os.path.join(GOLDEN, "effective_bits.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    for N, K, k, want in rows:
+        N, K, k = int(N), int(K), int(k)
+        plane_bytes = 4 * oracle.plane_words(N, K, k)
+        scale_bytes = 2 * k * (N + K)
+        bpw = 8.0 * (plane_bytes + scale_bytes) / (N * K)
+        assert round(bpw, 2) == float(want)
