@@ -26,11 +26,14 @@
  *   - bit = 1 <=> B = +1; 32 consecutive input columns per uint32 word with
  *     column c at bit c % 32 ("32 columns packed into one uint32_t", RaBiT,
  *     technical novelty paragraph).
- *   - word order (the storage layout):  plane i is cut into S = ceil(K/256)
- *     column slices; rows are grouped in quads (Nq = ceil(N/4));
- *        word(i, s, r, w) = (((i*S + s)*Nq + r/4)*8 + w)*4 + r%4
- *     holds columns 256*s + 32*w .. +31 of row r.  Bits of columns >= K and
- *     words of rows >= N are zero.
+ *   - word order (this library's storage format; the pages fix only the
+ *     32-columns-per-word packing): plane i is cut into S = ceil(K/256)
+ *     column slices and Nt = ceil(N/32) tiles of 32 rows; each
+ *     (plane, slice, tile) block has 256 words and
+ *        word(i, s, r, w) = (((i*S + s)*Nt + r/32)*256)
+ *                           + (w ^ ((r%32)/4))*32 + r%32
+ *     holds columns 256*s + 32*w .. +31 of row r (w = 0..7).  Bits of
+ *     columns >= K and words of rows >= N are zero.
  *   - stored scales are fp16, rounded to nearest-even from the fp32 inputs.
  *   - the greedy SVID initialiser (Greedy SVID, named in the technical
  *     novelty paragraph) takes, per plane, the rank-1 approximation of
@@ -126,15 +129,16 @@ double oracle_bf16_to_f64(uint16_t b) { return decode_bfloat16(b); }
 
 int64_t oracle_plane_words(int64_t N, int64_t K, int k)
 {
-    int64_t S = (K + 255) / 256, Nq = (N + 3) / 4;
-    return (int64_t)k * S * Nq * 32;
+    int64_t S = (K + 255) / 256, Nt = (N + 31) / 32;
+    return (int64_t)k * S * Nt * 256;
 }
 
 static int64_t word_index(int64_t N, int64_t K, int i, int64_t r, int64_t c)
 {
-    int64_t S = (K + 255) / 256, Nq = (N + 3) / 4;
-    int64_t s = c / 256, w = (c % 256) / 32;
-    return ((((int64_t)i * S + s) * Nq + r / 4) * 8 + w) * 4 + r % 4;
+    int64_t S = (K + 255) / 256, Nt = (N + 31) / 32;
+    int64_t s = c / 256, w = (c % 256) / 32, rho = r % 32;
+    int64_t block = ((int64_t)i * S + s) * Nt + r / 32;
+    return block * 256 + (w ^ (rho / 4)) * 32 + rho;
 }
 
 /* ------------------------------------------------------------------ */
