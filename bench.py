@@ -1,0 +1,458 @@
+#!/usr/bin/env python3
+"""Benchmark of the residual binarized linear layer on B200.
+
+Workload: the Llama-7B q_proj shape, N = K = 4096 with k = 2 residual sign
+planes (W ~ N(0, 0.02) with 0.1% x20 outliers, greedy-SVID scales), decode
+M = 1.  One step = 32 decode tokens, one after another, each through a stack
+of 96 distinct packed layers of that shape (rb_gemv per layer, launched with
+programmatic dependent launch, captured in a CUDA graph).  The 96 layers hold
+~403 MB of sign planes, more than the 126 MB L2, so every step streams the
+planes from HBM.  Metric: packed-weight bytes read per second (GB/s).
+
+Legs (one JSON line on rank 0):
+  value       device-timed (CUDA events) throughput, inputs resident in HBM;
+  e2e         the same step with X copied host->device from pinned memory and
+              the last layer's Y copied back, inside the timed region;
+  roofline    the GEMV kernel's algorithmic bytes per launch / its average
+              duration against the measured HBM copy bandwidth;
+  cpu_baseline  the CPU oracle (float64 dequantise-then-multiply) on a bounded
+              sample of the same workload (rank 0, N = 1 only);
+  rows        the other hot-path steps measured in the same run (rb_pack,
+              rb_gemv at M = 4 and 16, rb_gemm).
+--impl reference times the CPU oracle itself on this workload.
+Multi-GPU: every rank runs its own independent layer stack (weak scaling, no
+data-path collective); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+N_OUT, K_IN, K_PLANES = 4096, 4096, 2
+WORKLOAD = "q_proj_4096x4096_k2"
+METRIC = "packed-weight HBM GB/s (% of B200 peak) for k=2 binary GEMV; GEMM TFLOP/s"
+LAYERS, TOKENS = 96, 32
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ---------------------------------------------------------------- distributed plumbing
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, backend):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, x: float, device=None) -> float:
+        if not self.pg:
+            return x
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def assemble_line(*, value, unit, n_gpus, steps, warmup, ms_per_step, extra) -> dict:
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": n_gpus, "steps": steps,
+            "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u32 sign planes x bf16 -> f32",
+            "data": "synthetic"}
+    line.update(extra)
+    return line
+
+
+def throughput(bytes_per_step_per_rank: float, world: int, steps: int, seconds_max: float) -> float:
+    """Whole-job GB/s: bytes all ranks processed / max-over-ranks time."""
+    return bytes_per_step_per_rank * world * steps / seconds_max / 1e9
+
+
+# ---------------------------------------------------------------- peaks, clocks, profiles
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    def __init__(self, gpu_id: str | None, interval_ms=20):
+        self.gpu_id, self.interval_ms = gpu_id, interval_ms
+        self.proc, self.lines = None, []
+
+    def start(self):
+        cmd = ["nvidia-smi", "--query-gpu=clocks.sm,clocks.max.sm,utilization.gpu,power.draw,clocks_event_reasons.active",
+               "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.reader.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 5:
+                continue
+            try:
+                s, m, util = float(parts[0]), float(parts[1]), float(parts[2])
+                bits = int(parts[4], 16) if parts[4].lower().startswith("0x") else int(parts[4])
+            except ValueError:
+                continue
+            mx.append(m)
+            if util >= 50:
+                sm.append(s)
+                for b, name in REASON_BITS.items():
+                    if bits & b and name != "gpu_idle":
+                        reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                    "samples_under_load": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples_under_load": len(sm)}
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("rb_gemv.cu", "rbw_internal.cuh"):
+        with open(os.path.join(ROOT, "residual_binarized_weight_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_tag: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = kernel_sources_sha()
+    for ln in open(p):
+        f = dict(kv.split("=", 1) for kv in ln.split() if "=" in kv)
+        if f.get("kernel") == kernel_tag and f.get("src_sha") == sha:
+            return float(f["dram_bytes_per_launch"])
+    return None
+
+
+# ---------------------------------------------------------------- CPU oracle legs
+def oracle_sample(seconds_budget=15.0, max_layers=64):
+    """Time the oracle's float64 apply on the workload layer (bounded sample)."""
+    import oracle
+    from residual_binarized_weight_b200 import synth
+    wl = synth.workload(WORKLOAD)
+    W = synth.weights(wl.layers[0])
+    g, h = oracle.svid_greedy(W, K_PLANES, iters=20)
+    planes, g16, h16, st, _ = oracle.pack(W, g, h, K_PLANES)
+    X = synth.activations_for(wl, TOKENS, K_IN)
+    plane_bytes = 4 * planes.size
+    t0 = time.perf_counter()
+    n = 0
+    while n < max_layers:
+        oracle.apply(planes, g16, h16, N_OUT, K_IN, K_PLANES, X[n % TOKENS:n % TOKENS + 1])
+        n += 1
+        if time.perf_counter() - t0 > seconds_budget:
+            break
+    dt = time.perf_counter() - t0
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": plane_bytes * n / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": "%d single-token (M=1) applications of one %dx%d k=%d layer, float64 dequantise-then-multiply, %.1f s"
+                      % (n, N_OUT, K_IN, K_PLANES, dt)}, dt / n
+
+
+def run_reference(args, dist: Dist):
+    if dist.rank != 0:
+        return 0
+    budget = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(seconds_budget=0.5, max_layers=1)
+    cb, sec_per_layer = oracle_sample(seconds_budget=budget * args.steps, max_layers=max(1, args.steps))
+    line = assemble_line(value=cb["value"], unit="GB/s", n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
+                         ms_per_step=sec_per_layer * LAYERS * TOKENS * 1e3,
+                         extra={"impl": "reference", "config": config_dict(),
+                                "cpu_baseline": cb,
+                                "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}})
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict():
+    return {"workload": WORKLOAD, "n_out": N_OUT, "k_in": K_IN, "k_planes": K_PLANES, "M": 1,
+            "layers_per_step": LAYERS, "tokens_per_step": TOKENS,
+            "l2": "inputs larger than L2: %d distinct packed layers = %.0f MB of planes per pass" %
+                  (LAYERS, LAYERS * 4.194304),
+            "parallelism": "independent replicas (weak scaling, no collective)"}
+
+
+# ---------------------------------------------------------------- GPU leg
+def gpu_uuid(torch):
+    try:
+        u = torch.cuda.get_device_properties(torch.cuda.current_device()).uuid
+        return "GPU-" + str(u)
+    except Exception:
+        return None
+
+
+def run_rbw(args, dist: Dist):
+    import torch
+    from residual_binarized_weight_b200 import rbw, synth
+
+    torch.cuda.set_device(dist.local_rank)
+    dist.init("nccl")
+    dev = torch.device("cuda", dist.local_rank)
+    hbm_peak, bf16_peak, bf16_sust, peak_src = measured_peaks()
+    wl = synth.workload(WORKLOAD)
+
+    # ---- deploy: derive scales + pack one seeded layer, replicate to LAYERS distinct buffers
+    W = torch.from_numpy(synth.weights(wl.layers[0])).to(dev)
+    g, h = rbw.svid_greedy(W, K_PLANES, iters=20)
+    base = rbw.pack(W, g, h, K_PLANES)
+    layers = []
+    for _ in range(LAYERS):
+        L = rbw.PackedLayer(N_OUT, K_IN, K_PLANES, dev)
+        L.planes.copy_(base.planes)
+        L.g16.copy_(base.g16)
+        L.h16.copy_(base.h16)
+        layers.append(L)
+    structs = [L.struct() for L in layers]
+    X_host = synth.activations_for(wl, TOKENS, K_IN)
+    X = torch.from_numpy(X_host.view(np.int16)).to(dev)
+    Y_last = torch.empty(TOKENS, N_OUT, dtype=torch.float32, device=dev)
+    Y_tmp = torch.empty(1, N_OUT, dtype=torch.float32, device=dev)
+    ws = rbw.workspace(rbw.gemv_workspace_bytes(N_OUT, K_IN, K_PLANES, 1), dev)
+    lib = rbw.lib()
+    import ctypes
+
+    def step(stream):
+        sp = ctypes.c_void_p(stream.cuda_stream)
+        wsp, wsb = ctypes.c_void_p(ws.data_ptr()), ws.numel()
+        for t in range(TOKENS):
+            xp = ctypes.c_void_p(X.data_ptr() + t * K_IN * 2)
+            for li in range(LAYERS):
+                yp = ctypes.c_void_p((Y_last.data_ptr() + t * N_OUT * 4) if li == LAYERS - 1 else Y_tmp.data_ptr())
+                st = lib.rb_gemv(ctypes.byref(structs[li]), xp, 1, yp, rbw.RB_F32, wsp, wsb, None,
+                                 rbw.RB_LAUNCH_PDL, sp)
+                if st != 0:
+                    raise rbw.RbError("rb_gemv", st)
+
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        step(stream)                       # eager run (also sets kernel attributes)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step(stream)
+    torch.cuda.synchronize()
+
+    launches_per_step = TOKENS * LAYERS
+    plane_bytes = layers[0].packed_bytes()
+    bytes_per_step = plane_bytes * launches_per_step
+    algo_bytes_per_launch = plane_bytes + 2 * K_PLANES * (N_OUT + K_IN) + 2 * K_IN + 4 * N_OUT
+
+    for _ in range(max(3, args.warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_uuid(torch))
+    sampler.start()
+    time.sleep(0.05)
+    dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = sampler.stop()
+    t_local = ev0.elapsed_time(ev1) / 1e3
+    t_max = dist.max(t_local, dev)
+    value = throughput(bytes_per_step, dist.world, args.steps, t_max)
+    avg_launch_s = t_local / (args.steps * launches_per_step)
+    achieved = algo_bytes_per_launch / avg_launch_s / 1e9
+
+    # ---- e2e: host X in pinned memory -> device, 96-layer chain per token, Y of the last layer -> host
+    X_pin = torch.from_numpy(X_host.view(np.int16).copy()).pin_memory()
+    Y_pin = torch.empty(TOKENS, N_OUT, dtype=torch.float32).pin_memory()
+    graph_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_e2e, stream=stream):
+        X.copy_(X_pin, non_blocking=True)
+        step(stream)
+        Y_pin.copy_(Y_last, non_blocking=True)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        graph_e2e.replay()
+        stream.synchronize()
+    e2e_steps = max(1, min(args.steps, 200))
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        graph_e2e.replay()
+        stream.synchronize()               # the host reads each step's result
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = dist.max(e0.elapsed_time(e1) / 1e3, dev)
+    e2e = {"value": throughput(bytes_per_step, dist.world, e2e_steps, t_e2e), "unit": "GB/s",
+           "h2d_bytes_per_step": X_pin.numel() * 2, "d2h_bytes_per_step": Y_pin.numel() * 4,
+           "steps": e2e_steps}
+    del graph, graph_e2e
+
+    rows = other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak) if (dist.rank == 0 and not args.quick) else {}
+    dist.barrier()
+    line = None
+    if dist.rank == 0:
+        cb = None
+        if dist.world == 1 and not args.no_cpu_baseline:
+            cb, _ = oracle_sample(seconds_budget=args.cpu_seconds)
+        line = assemble_line(
+            value=value, unit="GB/s", n_gpus=dist.world, steps=args.steps, warmup=args.warmup,
+            ms_per_step=t_max / args.steps * 1e3,
+            extra={"impl": "rbw", "config": config_dict(),
+                   "pct_of_peak": {"measured_hbm": value / dist.world / hbm_peak, "spec_8tbs": value / dist.world / 8000.0},
+                   "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                                "frac": achieved / hbm_peak, "traffic": profiled_traffic("gemv_lut_kernel<2>"),
+                                "kernel": "gemv_lut_kernel<2>", "peak_source": peak_src,
+                                "algorithmic_bytes_per_launch": algo_bytes_per_launch,
+                                "avg_launch_us": avg_launch_s * 1e6},
+                   "cpu_baseline": cb, "e2e": e2e, "gpu_launches": args.steps * launches_per_step,
+                   "clocks": clocks, "rows": rows})
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+def time_events(torch, fn, reps, stream):
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / reps
+
+
+def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
+    """Device timings of the other hot-path steps on the same layer (kernels only)."""
+    out = {}
+    stream = torch.cuda.Stream(dev)
+    # rb_pack: reads W (4NK bytes), writes planes + fp16 scales
+    Lp = rbw.PackedLayer(N_OUT, K_IN, K_PLANES, dev)
+    t = time_events(torch, lambda: rbw.pack(W, g, h, K_PLANES, out=Lp, stream=stream), 20, stream)
+    pack_bytes = 4 * N_OUT * K_IN + Lp.packed_bytes() + 2 * K_PLANES * (N_OUT + K_IN)
+    out["pack"] = {"us": t * 1e6, "GBps": pack_bytes / t / 1e9, "bytes": pack_bytes}
+    # rb_gemv at M = 4 and 16 over 96 distinct layers (L2-defeating), plain launches
+    layers = []
+    for _ in range(LAYERS):
+        L = rbw.PackedLayer(N_OUT, K_IN, K_PLANES, dev)
+        L.planes.copy_(Lp.planes)
+        L.g16.copy_(Lp.g16)
+        L.h16.copy_(Lp.h16)
+        layers.append(L)
+    for M in (4, 16):
+        X = torch.from_numpy(synth.activations(M, K_IN, seed=M).view(np.int16)).to(dev)
+        Y = torch.empty(M, N_OUT, dtype=torch.float32, device=dev)
+        ws = rbw.workspace(rbw.gemv_workspace_bytes(N_OUT, K_IN, K_PLANES, M), dev)
+        it = iter(range(10 ** 9))
+
+        def f():
+            rbw.gemv(layers[next(it) % LAYERS], X, Y=Y, ws=ws, stream=stream)
+        t = time_events(torch, f, 2 * LAYERS, stream)
+        out["gemv_M%d" % M] = {"us": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
+                               "tokens_per_s": M / t}
+    # rb_gemm at M = 2048 on the prefill shape
+    try:
+        X = torch.from_numpy(synth.activations(2048, K_IN, seed=7).view(np.int16)).to(dev)
+        Lg = rbw.PackedLayer(N_OUT, K_IN, K_PLANES, dev)
+        Lg.planes.copy_(Lp.planes)
+        Lg.g16.copy_(Lp.g16)
+        Lg.h16.copy_(Lp.h16)
+        Y = torch.empty(2048, N_OUT, dtype=torch.float32, device=dev)
+        ws = rbw.workspace(rbw.gemm_workspace_bytes(N_OUT, K_IN, K_PLANES, 2048), dev)
+        t = time_events(torch, lambda: rbw.gemm(Lg, X, Y=Y, ws=ws, stream=stream), 10, stream)
+        fl = 2.0 * 2048 * N_OUT * K_IN * K_PLANES
+        out["gemm_M2048"] = {"us": t * 1e6, "TFLOPs": fl / t / 1e12, "frac_of_bf16_peak": fl / t / 1e12 / bf16_peak,
+                             "flops": fl}
+    except rbw.RbError as e:
+        out["gemm_M2048"] = {"unavailable": str(e)}
+    return out
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["rbw", "reference"], default="rbw")
+    ap.add_argument("--quick", action="store_true", help="skip the extra per-row timings")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    dist = Dist()
+    if args.impl == "reference":
+        return run_reference(args, dist)
+    return run_rbw(args, dist)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

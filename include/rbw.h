@@ -1,0 +1,166 @@
+/*
+ * rbw.h -- C ABI of the residual dual-scale binarized linear layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (RaBiT: Residual-Aware Binarization Training for Accurate and
+ * Efficient LLMs; "Residual binarization" background section and Algorithm 2):
+ *
+ *   W ~= sum_{i=1..k} diag(g_i) B_i diag(h_i),   B_i in {-1,+1}^{N x K}
+ *   R_0 = W;  B_i = sign(R_{i-1}) (sign(0) = +1);  R_i = R_{i-1} - g_i h_i^T .* B_i
+ *   Y   = sum_i g_i .* (B_i (h_i .* X))              ("matmul-free" inference)
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller (allocated
+ *     with cudaMalloc or a framework allocator).  The library allocates no
+ *     memory and keeps no global state besides the kernel attributes it sets
+ *     once per process.
+ *   - Row-major: W is [N out][K in]; X is [M][K]; Y is [M][N].
+ *   - Calls are asynchronous on `stream`.  Argument, shape and alignment
+ *     errors are returned synchronously and launch nothing.  CUDA launch
+ *     errors return RB_ERR_CUDA.  Data-dependent errors (non-finite input,
+ *     fp16 overflow of a scale, a bounded device wait that expired) are OR-ed
+ *     as RB_DEV_* bits into *dev_status (nullable, caller-zeroed), which the
+ *     caller reads after synchronising.
+ *   - Every pointer must be 16-byte aligned (RB_ERR_ALIGN otherwise).
+ *   - K must be a positive multiple of 32 (RB_ERR_SHAPE otherwise).
+ *   - Launch flags: RB_LAUNCH_PDL launches with programmatic dependent launch
+ *     so that a kernel may start streaming its weights while the previous
+ *     kernel on the stream finishes; the kernels wait for the previous grid
+ *     before reading X or writing anything.
+ *
+ * Packed sign-plane storage layout (the "32 columns packed into one
+ * uint32_t" format of RaBiT's kernel paragraph, with a word order chosen for
+ * this library):
+ *   - bit = 1 <=> B = +1; column c of a word is bit c % 32 (LSB first).
+ *   - plane i is cut into S = ceil(K/256) column slices and ceil(N/32) row
+ *     tiles of 32 rows; each (plane, slice, row tile) block is 256 words:
+ *       word(i, s, r, w) = ((((i*S + s)*Nt + r/32) * 256)
+ *                           + ((w ^ ((r % 32) / 4)) * 32) + r % 32
+ *     holds columns 256*s + 32*w .. 256*s + 32*w + 31 of row r (w = 0..7,
+ *     Nt = ceil(N/32)).  Bits of columns >= K and words of rows >= N are 0.
+ *   - scales are IEEE fp16: g16 [k][N], h16 [k][K].
+ */
+#ifndef RBW_H_
+#define RBW_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define RB_API __attribute__((visibility("default")))
+#else
+#define RB_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RB_OK = 0,
+    RB_ERR_ARG = 1,          /* null pointer, bad count, bad enum            */
+    RB_ERR_SHAPE = 2,        /* K not a multiple of 32, sizes out of range   */
+    RB_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned             */
+    RB_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required   */
+    RB_ERR_UNSUPPORTED = 5,  /* no sm_100 device current, or k/M not served  */
+    RB_ERR_CUDA = 6          /* a CUDA runtime call failed                   */
+} rb_status;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define RB_DEV_NONFINITE 0x1  /* W, g or h held a NaN or infinity            */
+#define RB_DEV_RANGE 0x2      /* |g| or |h| rounds to infinity in fp16       */
+#define RB_DEV_TIMEOUT 0x4    /* a bounded device-side wait expired          */
+
+typedef enum { RB_F32 = 0, RB_BF16 = 1 } rb_dtype;
+
+#define RB_LAUNCH_PDL 0x1u
+
+/* A packed layer: all pointers are device pointers owned by the caller. */
+typedef struct {
+    int32_t n_out;            /* N */
+    int32_t k_in;             /* K (multiple of 32) */
+    int32_t k_planes;         /* k, 1..8 */
+    int32_t reserved;         /* must be 0 */
+    const uint32_t *planes;   /* rb_packed_words(N, K, k) words */
+    const uint16_t *g16;      /* [k][N] fp16 */
+    const uint16_t *h16;      /* [k][K] fp16 */
+} rb_layer_t;
+
+/* Library version, 10000*major + 100*minor + patch. */
+RB_API int rb_version(void);
+
+/* Human-readable name of a status code (static string). */
+RB_API const char *rb_status_string(int status);
+
+/* Number of uint32 words of the sign planes of an N x K layer with k planes
+ * (layout above): k * ceil(K/256) * ceil(N/32) * 256.  Returns 0 for invalid
+ * sizes. */
+RB_API size_t rb_packed_words(int n_out, int k_in, int k_planes);
+
+/*
+ * rb_pack -- derive and bit-pack the residual sign planes (RaBiT, Algorithm 2
+ * forward pass; deployment freezes these planes and drops W).
+ *   W        [N][K] fp32 latent weight.
+ *   g, h     [k][N], [k][K] fp32 per-plane scales (any sign; normally >= 0).
+ *   planes   out, rb_packed_words(N,K,k) uint32 words (layout above).
+ *   g16, h16 out, fp16 copies of g, h (round to nearest even).
+ * The residual runs in fp32 with the product g_i[r]*h_i[c] rounded on its own
+ * before the single add/subtract (no fused multiply-add), using the fp32
+ * scales: b = (R >= 0) (so -0.0 gives +1); R <- b ? R - t : R + t.
+ * dev_status gets RB_DEV_NONFINITE / RB_DEV_RANGE.
+ */
+RB_API rb_status rb_pack(const float *W, const float *g, const float *h,
+                  int n_out, int k_in, int k_planes,
+                  uint32_t *planes, uint16_t *g16, uint16_t *h16,
+                  int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * rb_gemv -- decode-time Y = sum_i g_i .* (B_i (h_i .* X)) for 1 <= M <= 64
+ * tokens (tuned for M = 1; RaBiT "matmul-free" evaluation, additions and
+ * element-wise scaling only).
+ *   X   [M][K] bfloat16 bit patterns.
+ *   Y   [M][N] fp32 or bfloat16 (y_dtype), written, never read.
+ *   workspace: rb_gemv_workspace_bytes(N, K, k, M) bytes of device memory,
+ *   zero-filled by the caller before its first use; every call leaves it
+ *   zero-filled again.  Calls that share a workspace must not overlap on the
+ *   GPU (same stream, or PDL, is fine).
+ * h_i .* x is formed exactly in fp32 and every sum is accumulated in fp32.
+ */
+RB_API size_t rb_gemv_workspace_bytes(int n_out, int k_in, int k_planes, int M);
+RB_API rb_status rb_gemv(const rb_layer_t *layer, const uint16_t *X, int M,
+                  void *Y, rb_dtype y_dtype, void *workspace, size_t workspace_bytes,
+                  int32_t *dev_status, unsigned flags, cudaStream_t stream);
+
+/*
+ * rb_gemm -- batched (prefill) Y = X . What^T for any M >= 1 (tuned for
+ * M >= 64) on the tcgen05 tensor cores: sign tiles are expanded to +-h_i
+ * (fp16, exact) and multiplied with X converted to fp16 (exact in the normal
+ * range), fp32 accumulation in tensor memory, one accumulator per plane,
+ * epilogue Y = sum_i g_i . acc_i.
+ *   workspace: rb_gemm_workspace_bytes(N, K, k, M) bytes (holds X in fp16).
+ */
+RB_API size_t rb_gemm_workspace_bytes(int n_out, int k_in, int k_planes, int M);
+RB_API rb_status rb_gemm(const rb_layer_t *layer, const uint16_t *X, int M,
+                  void *Y, rb_dtype y_dtype, void *workspace, size_t workspace_bytes,
+                  int32_t *dev_status, unsigned flags, cudaStream_t stream);
+
+/*
+ * rb_svid_greedy -- greedy SVID scales for each plane (RaBiT names Greedy
+ * SVID as the traditional initialiser): for i = 1..k, (g_i, h_i) is the
+ * rank-1 approximation of |R_{i-1}| by `iters` rounds of power iteration in
+ * float64 (v0 = 1/sqrt(K); u = A v/|A v|; v = A^T u/|A^T u|; sigma = u^T A v;
+ * g_i = fp32(sqrt(sigma) u), h_i = fp32(sqrt(sigma) v)), with R_{i-1} from
+ * the same fp32 recurrence as rb_pack.
+ *   g, h out [k][N], [k][K] fp32.
+ *   workspace: rb_svid_workspace_bytes(N, K) bytes.
+ */
+RB_API size_t rb_svid_workspace_bytes(int n_out, int k_in);
+RB_API rb_status rb_svid_greedy(const float *W, int n_out, int k_in, int k_planes, int iters,
+                         float *g, float *h, void *workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RBW_H_ */

@@ -1,0 +1,154 @@
+// rb_pack.cu -- derive the residual sign planes and bit-pack them in one pass
+// over W (RaBiT, Algorithm 2 forward pass: R_0 = W, B_i = sign(R_{i-1}),
+// R_i = R_{i-1} - g_i h_i^T .* B_i; deployment keeps the planes and drops W).
+//
+// One warp owns a 32-row x 32-column item (one sign word per row and plane).
+// Lane l holds column c = 256 s + 32 w + l and walks the 32 rows of the tile:
+// each W row segment is one coalesced 128-byte load, the residual stays in a
+// register across the k planes, and a warp ballot turns the 32 sign decisions
+// of a row into its packed word, which the lane owning that row keeps.  After
+// the tile, lane l stores its row's word to slot w ^ (l/4) of the tile block.
+//
+// The fp32 residual update is written with explicitly rounded intrinsics
+// (__fmul_rn, __fadd_rn, __fsub_rn), so no fused multiply-add can be formed:
+// t = fl(g*h), then R = fl(R -/+ t).  This makes the planes bit-exact with
+// any IEEE fp32 evaluation of the same recurrence.
+#include <float.h>
+
+#include "rbw_internal.cuh"
+
+namespace rbw {
+namespace {
+
+constexpr int kPackThreads = 256;
+
+template <int KP>
+__global__ void __launch_bounds__(kPackThreads, 2)
+pack_kernel(const float* __restrict__ W, const float* __restrict__ g,
+            const float* __restrict__ h, int N, int K,
+            uint32_t* __restrict__ planes, int32_t* dev_status)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t S = num_slices(K), Nt = num_row_tiles(N);
+    const int64_t items = Nt * S * 8;
+    const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    int bad = 0;
+
+    for (int64_t it = gwarp; it < items; it += nwarps) {
+        const int w = (int)(it & 7);              // logical word within the slice
+        const int64_t s = (it >> 3) % S;
+        const int64_t t = (it >> 3) / S;
+        const int64_t col0 = s * 256 + (int64_t)w * 32;
+        const int64_t c = col0 + lane;
+        uint32_t mine[KP];
+#pragma unroll
+        for (int i = 0; i < KP; ++i) mine[i] = 0u;
+
+        if (col0 < K) {                           // K % 32 == 0: whole word valid
+            float hv[KP], gv[KP];
+            const int64_t my_row = t * 32 + lane;
+#pragma unroll
+            for (int i = 0; i < KP; ++i) {
+                hv[i] = h[(int64_t)i * K + c];
+                gv[i] = my_row < N ? g[(int64_t)i * N + my_row] : 0.0f;
+            }
+#pragma unroll
+            for (int r0 = 0; r0 < 32; r0 += 8) {
+                float wv[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int64_t r = t * 32 + r0 + j;
+                    wv[j] = r < N ? __ldcs(W + r * K + c) : 0.0f;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const bool row_ok = (t * 32 + r0 + j) < N;
+                    float R = wv[j];
+                    bad |= !(fabsf(R) <= FLT_MAX);
+#pragma unroll
+                    for (int i = 0; i < KP; ++i) {
+                        const float gi = __shfl_sync(0xffffffffu, gv[i], r0 + j);
+                        const bool b = R >= 0.0f;               // sign(0) = +1, -0.0 too
+                        const float tt = __fmul_rn(gi, hv[i]);
+                        R = b ? __fsub_rn(R, tt) : __fadd_rn(R, tt);
+                        const uint32_t word = __ballot_sync(0xffffffffu, b);
+                        if (lane == r0 + j) mine[i] = row_ok ? word : 0u;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < KP; ++i)
+            planes[word_offset(i, s, t * 32 + lane, w, S, Nt)] = mine[i];
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_dev_status(dev_status, RB_DEV_NONFINITE);
+}
+
+// fp16 copies of the scales (round to nearest even) with range checks.
+__global__ void cast_scales_kernel(const float* __restrict__ g, const float* __restrict__ h,
+                                   int64_t ng, int64_t nh, uint16_t* __restrict__ g16,
+                                   uint16_t* __restrict__ h16, int32_t* dev_status)
+{
+    int flags = 0;
+    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < ng + nh;
+         x += (int64_t)gridDim.x * blockDim.x) {
+        const float v = x < ng ? g[x] : h[x - ng];
+        const __half q = __float2half_rn(v);
+        if (!(fabsf(v) <= FLT_MAX)) flags |= RB_DEV_NONFINITE;
+        else if (__hisinf(q)) flags |= RB_DEV_RANGE;
+        const uint16_t bits = __half_as_ushort(q);
+        if (x < ng) g16[x] = bits;
+        else h16[x - ng] = bits;
+    }
+    if (flags) set_dev_status(dev_status, flags);
+}
+
+template <int KP>
+rb_status launch_pack(const float* W, const float* g, const float* h, int N, int K,
+                      uint32_t* planes, int32_t* dev_status, cudaStream_t stream)
+{
+    const int64_t items = num_row_tiles(N) * num_slices(K) * 8;
+    const int64_t warps_per_cta = kPackThreads / 32;
+    int64_t ctas = (items + warps_per_cta - 1) / warps_per_cta;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (ctas > cap) ctas = cap;
+    return launch(pack_kernel<KP>, dim3((unsigned)ctas), dim3(kPackThreads), 0, stream, false,
+                  W, g, h, N, K, planes, dev_status);
+}
+
+}  // namespace
+}  // namespace rbw
+
+using namespace rbw;
+
+extern "C" rb_status rb_pack(const float* W, const float* g, const float* h,
+                             int n_out, int k_in, int k_planes,
+                             uint32_t* planes, uint16_t* g16, uint16_t* h16,
+                             int32_t* dev_status, cudaStream_t stream)
+{
+    if (!W || !g || !h || !planes || !g16 || !h16) return RB_ERR_ARG;
+    if (k_planes < 1 || k_planes > 8) return RB_ERR_ARG;
+    if (n_out < 1 || k_in < 32 || k_in % 32 != 0) return RB_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(g) || !aligned16(h) || !aligned16(planes) ||
+        !aligned16(g16) || !aligned16(h16) || (dev_status && !aligned16(dev_status)))
+        return RB_ERR_ALIGN;
+    if (!device_is_sm100()) return RB_ERR_UNSUPPORTED;
+
+    const int64_t ng = (int64_t)k_planes * n_out, nh = (int64_t)k_planes * k_in;
+    int64_t cast_ctas = (ng + nh + 255) / 256;
+    if (cast_ctas > 4 * num_sms()) cast_ctas = 4 * num_sms();
+    rb_status st = launch(cast_scales_kernel, dim3((unsigned)cast_ctas), dim3(256), 0, stream,
+                          false, g, h, ng, nh, g16, h16, dev_status);
+    if (st != RB_OK) return st;
+    switch (k_planes) {
+        case 1: return launch_pack<1>(W, g, h, n_out, k_in, planes, dev_status, stream);
+        case 2: return launch_pack<2>(W, g, h, n_out, k_in, planes, dev_status, stream);
+        case 3: return launch_pack<3>(W, g, h, n_out, k_in, planes, dev_status, stream);
+        case 4: return launch_pack<4>(W, g, h, n_out, k_in, planes, dev_status, stream);
+        case 5: return launch_pack<5>(W, g, h, n_out, k_in, planes, dev_status, stream);
+        case 6: return launch_pack<6>(W, g, h, n_out, k_in, planes, dev_status, stream);
+        case 7: return launch_pack<7>(W, g, h, n_out, k_in, planes, dev_status, stream);
+        default: return launch_pack<8>(W, g, h, n_out, k_in, planes, dev_status, stream);
+    }
+}

@@ -1,0 +1,167 @@
+"""Thin ctypes binding of the C ABI in ``include/rbw.h`` (librbw.so).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  Tensors must be CUDA tensors on the current device; the calls are
+issued on torch's current stream.  A missing library raises immediately
+(there is no fallback path).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librbw.so")
+
+RB_OK, RB_ERR_ARG, RB_ERR_SHAPE, RB_ERR_ALIGN, RB_ERR_WORKSPACE, RB_ERR_UNSUPPORTED, RB_ERR_CUDA = range(7)
+RB_DEV_NONFINITE, RB_DEV_RANGE, RB_DEV_TIMEOUT = 0x1, 0x2, 0x4
+RB_F32, RB_BF16 = 0, 1
+RB_LAUNCH_PDL = 0x1
+
+# name -> (restype, argtypes); the full exported surface of include/rbw.h
+_vp, _i32, _sz, _u32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint
+SIGNATURES = {
+    "rb_version": (_i32, []),
+    "rb_status_string": (ctypes.c_char_p, [_i32]),
+    "rb_packed_words": (_sz, [_i32, _i32, _i32]),
+    "rb_pack": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "rb_gemv_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
+    "rb_gemv": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _u32, _vp]),
+    "rb_gemm_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
+    "rb_gemm": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _u32, _vp]),
+    "rb_svid_workspace_bytes": (_sz, [_i32, _i32]),
+    "rb_svid_greedy": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+}
+
+
+class RbLayer(ctypes.Structure):
+    _fields_ = [("n_out", ctypes.c_int32), ("k_in", ctypes.c_int32), ("k_planes", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("planes", _vp), ("g16", _vp), ("h16", _vp)]
+
+
+_lib = None
+
+
+def lib():
+    """Load librbw.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("librbw.so not found at %s: run residual_binarized_weight_b200/build.py" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+class RbError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__("%s failed: %s" % (fn, lib().rb_status_string(status).decode()))
+
+
+def _check(fn, status):
+    if status != RB_OK:
+        raise RbError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def packed_words(n_out, k_in, k_planes):
+    return int(lib().rb_packed_words(n_out, k_in, k_planes))
+
+
+class PackedLayer:
+    """Device tensors of one packed layer (owns them) plus its rb_layer_t view."""
+
+    def __init__(self, n_out, k_in, k_planes, device="cuda"):
+        nw = packed_words(n_out, k_in, k_planes)
+        if nw == 0:
+            raise ValueError("invalid layer shape")
+        self.n_out, self.k_in, self.k_planes = n_out, k_in, k_planes
+        self.planes = torch.empty(nw, dtype=torch.int32, device=device)
+        self.g16 = torch.empty(k_planes, n_out, dtype=torch.float16, device=device)
+        self.h16 = torch.empty(k_planes, k_in, dtype=torch.float16, device=device)
+
+    def struct(self):
+        return RbLayer(self.n_out, self.k_in, self.k_planes, 0, self.planes.data_ptr(),
+                       self.g16.data_ptr(), self.h16.data_ptr())
+
+    def packed_bytes(self):
+        return self.planes.numel() * 4
+
+
+def pack(W, g, h, k_planes, out: PackedLayer | None = None, dev_status=None, stream=None):
+    """rb_pack: W fp32 [N][K], g fp32 [k][N], h fp32 [k][K] (CUDA) -> PackedLayer."""
+    N, K = W.shape
+    out = out or PackedLayer(N, K, k_planes, W.device)
+    st = lib().rb_pack(_ptr(W), _ptr(g), _ptr(h), N, K, k_planes, _ptr(out.planes), _ptr(out.g16),
+                       _ptr(out.h16), _ptr(dev_status), _stream(stream))
+    _check("rb_pack", st)
+    return out
+
+
+def gemv_workspace_bytes(n_out, k_in, k_planes, M):
+    return int(lib().rb_gemv_workspace_bytes(n_out, k_in, k_planes, M))
+
+
+def gemm_workspace_bytes(n_out, k_in, k_planes, M):
+    return int(lib().rb_gemm_workspace_bytes(n_out, k_in, k_planes, M))
+
+
+def svid_workspace_bytes(n_out, k_in):
+    return int(lib().rb_svid_workspace_bytes(n_out, k_in))
+
+
+def workspace(nbytes, device="cuda"):
+    """Zero-filled device workspace (uint8) of at least nbytes (16-byte aligned)."""
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def _apply(fn_name, layer: PackedLayer, X, Y, ws, flags, dev_status, stream):
+    M = X.shape[0]
+    ydt = RB_BF16 if Y.dtype == torch.bfloat16 else RB_F32
+    L = layer.struct()
+    wsp, wsb = (None, 0) if ws is None else (_ptr(ws), ws.numel() * ws.element_size())
+    st = getattr(lib(), fn_name)(ctypes.byref(L), _ptr(X), M, _ptr(Y), ydt, wsp, wsb,
+                                 _ptr(dev_status), flags, _stream(stream))
+    _check(fn_name, st)
+    return Y
+
+
+def gemv(layer: PackedLayer, X, Y=None, ws=None, flags=0, dev_status=None, stream=None, y_dtype=torch.float32):
+    """rb_gemv: X bf16 [M][K] (M <= 64) -> Y [M][N] (fp32 or bf16)."""
+    if Y is None:
+        Y = torch.empty(X.shape[0], layer.n_out, dtype=y_dtype, device=X.device)
+    return _apply("rb_gemv", layer, X, Y, ws, flags, dev_status, stream)
+
+
+def gemm(layer: PackedLayer, X, Y=None, ws=None, flags=0, dev_status=None, stream=None, y_dtype=torch.float32):
+    """rb_gemm: X bf16 [M][K] -> Y [M][N] (fp32 or bf16) on the tcgen05 tensor cores."""
+    if Y is None:
+        Y = torch.empty(X.shape[0], layer.n_out, dtype=y_dtype, device=X.device)
+    return _apply("rb_gemm", layer, X, Y, ws, flags, dev_status, stream)
+
+
+def svid_greedy(W, k_planes, iters=20, ws=None, stream=None):
+    """rb_svid_greedy: fp32 W [N][K] (CUDA) -> (g [k][N], h [k][K]) fp32."""
+    N, K = W.shape
+    g = torch.empty(k_planes, N, dtype=torch.float32, device=W.device)
+    h = torch.empty(k_planes, K, dtype=torch.float32, device=W.device)
+    ws = ws if ws is not None else workspace(svid_workspace_bytes(N, K), W.device)
+    st = lib().rb_svid_greedy(_ptr(W), N, K, k_planes, iters, _ptr(g), _ptr(h), _ptr(ws),
+                              ws.numel(), _stream(stream))
+    _check("rb_svid_greedy", st)
+    return g, h

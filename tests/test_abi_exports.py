@@ -1,0 +1,113 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* librbw.so loads and exports every function declared in include/rbw.h, and
+  the Python binding describes exactly that set.
+* Size helpers agree with the oracle's independent size formula.
+* Argument errors are returned before any CUDA call, and a valid call on a
+  machine without a B200 fails loudly (RB_ERR_UNSUPPORTED), never silently.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from residual_binarized_weight_b200 import build as rbw_build
+from residual_binarized_weight_b200 import rbw
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rbw.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    rbw_build.build()
+    return rbw.lib()
+
+
+def declared_functions():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return set(re.findall(r"\b(rb_[a-z0-9_]+)\s*\(", txt))
+
+
+def test_exports_match_header(L):
+    decl = declared_functions()
+    assert decl, "no declarations parsed"
+    assert decl == set(rbw.SIGNATURES), decl ^ set(rbw.SIGNATURES)
+    for name in decl:
+        assert hasattr(L, name), name
+
+
+def test_version_and_status_strings(L):
+    assert L.rb_version() >= 100
+    for code in range(7):
+        assert L.rb_status_string(code).decode().startswith("RB_")
+
+
+@pytest.mark.parametrize("N,K,k", [(256, 512, 1), (4096, 4096, 2), (33, 288, 3), (1, 32, 8), (11008, 4096, 2)])
+def test_packed_words_matches_oracle(L, N, K, k):
+    assert L.rb_packed_words(N, K, k) == oracle.plane_words(N, K, k)
+
+
+def test_size_helpers_reject_bad_shapes(L):
+    assert L.rb_packed_words(4, 48, 1) == 0
+    assert L.rb_packed_words(0, 64, 1) == 0
+    assert L.rb_packed_words(4, 64, 9) == 0
+    assert L.rb_gemv_workspace_bytes(4096, 4096, 2, 65) == 0
+    assert L.rb_gemv_workspace_bytes(4096, 4096, 2, 1) > 0
+    assert L.rb_gemv_workspace_bytes(64, 256, 2, 1) == 0     # one slice: no cross-slice sums
+    assert L.rb_svid_workspace_bytes(4096, 4096) > 0
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_pack_argument_errors_on_host(L):
+    a = _fake(0x10000)
+    assert L.rb_pack(None, a, a, 4, 64, 1, a, a, a, None, None) == rbw.RB_ERR_ARG
+    assert L.rb_pack(a, a, a, 4, 64, 0, a, a, a, None, None) == rbw.RB_ERR_ARG
+    assert L.rb_pack(a, a, a, 4, 48, 1, a, a, a, None, None) == rbw.RB_ERR_SHAPE
+    assert L.rb_pack(a, a, a, 0, 64, 1, a, a, a, None, None) == rbw.RB_ERR_SHAPE
+    assert L.rb_pack(_fake(0x10004), a, a, 4, 64, 1, a, a, a, None, None) == rbw.RB_ERR_ALIGN
+    # well-formed call without an sm_100 device: loud failure, nothing launched
+    assert L.rb_pack(a, a, a, 4, 64, 1, a, a, a, None, None) == rbw.RB_ERR_UNSUPPORTED
+
+
+def test_apply_argument_errors_on_host(L):
+    a = _fake(0x10000)
+    lay = rbw.RbLayer(64, 256, 2, 0, 0x10000, 0x10000, 0x10000)
+    for fn in (L.rb_gemv, L.rb_gemm):
+        assert fn(None, a, 1, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_ARG
+        assert fn(ctypes.byref(lay), a, 1, a, 7, None, 0, None, 0, None) == rbw.RB_ERR_ARG
+        assert fn(ctypes.byref(lay), a, 0, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_SHAPE
+        assert fn(ctypes.byref(lay), _fake(0x10002), 1, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_ALIGN
+        bad = rbw.RbLayer(64, 250, 2, 0, 0x10000, 0x10000, 0x10000)
+        assert fn(ctypes.byref(bad), a, 1, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_SHAPE
+        res = rbw.RbLayer(64, 256, 2, 1, 0x10000, 0x10000, 0x10000)
+        assert fn(ctypes.byref(res), a, 1, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_ARG
+        assert fn(ctypes.byref(lay), a, 1, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_UNSUPPORTED
+    assert L.rb_gemv(ctypes.byref(lay), a, 65, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_SHAPE
+    assert L.rb_gemv(ctypes.byref(lay), a, 1, a, 0, None, 0, None, 2, None) == rbw.RB_ERR_ARG
+
+
+def test_svid_argument_errors_on_host(L):
+    a = _fake(0x10000)
+    assert L.rb_svid_greedy(a, 4, 64, 1, 20, a, a, None, 0, None) == rbw.RB_ERR_ARG
+    assert L.rb_svid_greedy(a, 4, 64, 1, 0, a, a, a, 1 << 20, None) == rbw.RB_ERR_ARG
+    assert L.rb_svid_greedy(a, 4, 40, 1, 20, a, a, a, 1 << 20, None) == rbw.RB_ERR_SHAPE
+    assert L.rb_svid_greedy(a, 4, 64, 1, 20, a, a, a, 16, None) == rbw.RB_ERR_WORKSPACE
+    assert L.rb_svid_greedy(a, 4, 64, 1, 20, a, a, a, 1 << 20, None) == rbw.RB_ERR_UNSUPPORTED
+
+
+def test_product_does_not_import_oracle():
+    """The CUDA binding, build script and package never reference the oracle."""
+    pkg = os.path.join(ROOT, "residual_binarized_weight_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "rb_oracle" not in txt, f

@@ -1,0 +1,110 @@
+"""rb_gemv parity against the float64 oracle (dequantise, then multiply).
+
+The GPU consumes the oracle's packed planes (uploaded), so a pack error cannot
+hide a GEMV error; one end-to-end case also runs rb_pack -> rb_gemv.  Gates:
+relative Frobenius error <= 2e-3 and a per-element bound (see cases.check_y).
+Full-size workloads check every output where the oracle is fast enough and a
+fixed sample of rows (first, last, ragged tail, random) otherwise.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from residual_binarized_weight_b200 import rbw, synth
+from tests import cases
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gemv(L, X, M, ydtype, flags=0, ws=None):
+    N, K, k = L.n_out, L.k_in, L.k_planes
+    if ws is None:
+        ws = rbw.workspace(rbw.gemv_workspace_bytes(N, K, k, M))
+    Xd = cases.to_dev(X)
+    Y = rbw.gemv(L, Xd, ws=ws, flags=flags, y_dtype=ydtype)
+    torch.cuda.synchronize()
+    return Y.float().cpu().numpy().astype(np.float64), ws
+
+
+def sample_rows(N, n=384, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = set(range(min(N, 64))) | set(range(max(0, N - 64), N))
+    rows |= set(rng.choice(N, size=min(N, n), replace=False).tolist())
+    return np.array(sorted(rows), np.int64)
+
+
+CASES = [(0, 0, 1, 1), (1, 0, 2, 1), (1, 0, 2, 4), (1, 0, 2, 16), (2, 0, 2, 1), (2, 2, 2, 1),
+         (2, 0, 2, 8), (3, 0, 1, 1), (3, 0, 2, 1), (3, 0, 2, 16), (3, 0, 1, 64)]
+
+
+@pytest.mark.parametrize("wl,li,k,M", CASES)
+@pytest.mark.parametrize("ydt", [torch.float32, torch.bfloat16])
+def test_gemv_workloads(wl, li, k, M, ydt):
+    W, g, h = cases.layer_case(wl, li, k)
+    N, K = W.shape
+    planes, g16, h16 = cases.packed_case(wl, li, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    X = synth.activations_for(synth.workload(wl), M, K)
+    Yg, ws = run_gemv(L, X, M, ydt)
+    rows = None if N * K * M <= 2 ** 27 else sample_rows(N)
+    Yr = oracle.apply(planes, g16, h16, N, K, k, X, rows=rows)
+    Yg = Yg if rows is None else Yg[:, rows]
+    cases.check_y(Yg, Yr, cases.abs_bound(g16, h16, X, rows), bf16=ydt == torch.bfloat16)
+    assert not ws.any(), "workspace not left zero-filled"
+
+
+@pytest.mark.parametrize("N,K,k,M", [(33, 288, 2, 1), (100, 800, 3, 1), (1, 32, 1, 1), (1000, 544, 4, 1),
+                                     (70, 1056, 2, 2), (65, 320, 5, 3), (40, 256, 8, 17), (97, 2080, 2, 64),
+                                     (31, 4096, 1, 5), (4097, 288, 2, 1)])
+def test_gemv_ragged(N, K, k, M):
+    rng = np.random.default_rng(N + 3 * K + 7 * k + M)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=8)
+    planes, g16, h16, st, _ = oracle.pack(W, g, h, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    X = synth.activations(M, K, seed=M + K)
+    for ydt in (torch.float32, torch.bfloat16):
+        Yg, _ = run_gemv(L, X, M, ydt)
+        Yr = oracle.apply(planes, g16, h16, N, K, k, X)
+        cases.check_y(Yg, Yr, cases.abs_bound(g16, h16, X), bf16=ydt == torch.bfloat16)
+
+
+def test_gemv_deterministic_pdl_and_reused_workspace():
+    W, g, h = cases.layer_case(1, 0, 2)
+    N, K = W.shape
+    planes, g16, h16 = cases.packed_case(1, 0, 2)
+    L = cases.upload_layer(planes, g16, h16, N, K, 2)
+    X = synth.activations(1, K, seed=123)
+    ws = rbw.workspace(rbw.gemv_workspace_bytes(N, K, 2, 1))
+    outs = [run_gemv(L, X, 1, torch.float32, flags=f, ws=ws)[0] for f in (0, rbw.RB_LAUNCH_PDL, 0, rbw.RB_LAUNCH_PDL)]
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+    assert not ws.any()
+
+
+def test_gemv_end_to_end_from_gpu_pack():
+    """rb_pack -> rb_gemv on the device vs oracle.pack -> oracle.apply."""
+    W, g, h = cases.layer_case(2, 2, 2)                 # down_proj 4096 x 11008
+    N, K = W.shape
+    L = rbw.pack(cases.to_dev(W), cases.to_dev(g), cases.to_dev(h), 2)
+    X = synth.activations_for(synth.workload(2), 1, K)
+    Yg, _ = run_gemv(L, X, 1, torch.float32)
+    planes, g16, h16 = cases.packed_case(2, 2, 2)
+    Yr = oracle.apply(planes, g16, h16, N, K, 2, X)
+    cases.check_y(Yg, Yr, cases.abs_bound(g16, h16, X), bf16=False)
+
+
+def test_gemv_errors_on_device():
+    W, g, h = cases.layer_case(1, 0, 2)
+    N, K = W.shape
+    planes, g16, h16 = cases.packed_case(1, 0, 2)
+    L = cases.upload_layer(planes, g16, h16, N, K, 2)
+    X = cases.to_dev(synth.activations(1, K, seed=1))
+    small = rbw.workspace(64)
+    with pytest.raises(rbw.RbError) as e:
+        rbw.gemv(L, X, ws=small)
+    assert e.value.status == rbw.RB_ERR_WORKSPACE
+    with pytest.raises(rbw.RbError) as e:
+        rbw.gemv(L, X, ws=None)
+    assert e.value.status == rbw.RB_ERR_WORKSPACE
