@@ -274,85 +274,109 @@ def run_rbw(args, dist: Dist):
     X_host = synth.activations_for(wl, TOKENS, K_IN)
     X = torch.from_numpy(X_host.view(np.int16)).to(dev)
     Y_last = torch.empty(TOKENS, N_OUT, dtype=torch.float32, device=dev)
-    Y_tmp = torch.empty(1, N_OUT, dtype=torch.float32, device=dev)
-    ws = rbw.workspace(rbw.gemv_workspace_bytes(N_OUT, K_IN, K_PLANES, 1), dev)
     lib = rbw.lib()
     import ctypes
 
-    def step(stream):
-        sp = ctypes.c_void_p(stream.cuda_stream)
-        wsp, wsb = ctypes.c_void_p(ws.data_ptr()), ws.numel()
-        for t in range(TOKENS):
-            xp = ctypes.c_void_p(X.data_ptr() + t * K_IN * 2)
-            for li in range(LAYERS):
-                yp = ctypes.c_void_p((Y_last.data_ptr() + t * N_OUT * 4) if li == LAYERS - 1 else Y_tmp.data_ptr())
-                st = lib.rb_gemv(ctypes.byref(structs[li]), xp, 1, yp, rbw.RB_F32, wsp, wsb, None,
-                                 rbw.RB_LAUNCH_PDL, sp)
-                if st != 0:
-                    raise rbw.RbError("rb_gemv", st)
+    NS = 4                                 # independent layers go round-robin over NS streams
+    streams = [torch.cuda.Stream(dev) for _ in range(NS)]
+    wss = [rbw.workspace(rbw.gemv_workspace_bytes(N_OUT, K_IN, K_PLANES, 1), dev) for _ in range(NS)]
+    ytmp = [torch.empty(1, N_OUT, dtype=torch.float32, device=dev) for _ in range(NS)]
 
-    stream = torch.cuda.Stream(dev)
-    with torch.cuda.stream(stream):
-        step(stream)                       # eager run (also sets kernel attributes)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        step(stream)
-    torch.cuda.synchronize()
+    def launch(li, t, stream, wsi):
+        yp = (Y_last.data_ptr() + t * N_OUT * 4) if li == LAYERS - 1 else ytmp[wsi].data_ptr()
+        st = lib.rb_gemv(ctypes.byref(structs[li]), ctypes.c_void_p(X.data_ptr() + t * K_IN * 2), 1,
+                         ctypes.c_void_p(yp), rbw.RB_F32, ctypes.c_void_p(wss[wsi].data_ptr()),
+                         wss[wsi].numel(), None, rbw.RB_LAUNCH_PDL, ctypes.c_void_p(stream.cuda_stream))
+        if st != 0:
+            raise rbw.RbError("rb_gemv", st)
+
+    def step_streams():
+        """32 tokens x 96 independent layers; layer l on stream l % NS (fork/join on streams[0])."""
+        ev = torch.cuda.Event()
+        ev.record(streams[0])
+        for sx in streams[1:]:
+            sx.wait_event(ev)
+        for t in range(TOKENS):
+            for li in range(LAYERS):
+                launch(li, t, streams[li % NS], li % NS)
+        for sx in streams[1:]:
+            e = torch.cuda.Event()
+            e.record(sx)
+            streams[0].wait_event(e)
+
+    def step_chain():
+        """The same 3072 applications as one dependent chain on one stream (PDL)."""
+        for t in range(TOKENS):
+            for li in range(LAYERS):
+                launch(li, t, streams[0], 0)
+
+    def capture(fn, pre=None, post=None):
+        with torch.cuda.stream(streams[0]):
+            fn()                           # eager run (sets kernel attributes)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=streams[0]):
+            if pre:
+                pre()
+            fn()
+            if post:
+                post()
+        torch.cuda.synchronize()
+        return gr
+
+    def time_graph(gr, steps, sync_each=False):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(streams[0]):
+            for _ in range(max(3, args.warmup)):
+                gr.replay()
+            torch.cuda.synchronize()
+            dist.barrier()
+            e0.record(streams[0])
+            for _ in range(steps):
+                gr.replay()
+                if sync_each:
+                    streams[0].synchronize()       # the host reads each step's result
+            e1.record(streams[0])
+        torch.cuda.synchronize()
+        dist.barrier()
+        return e0.elapsed_time(e1) / 1e3
 
     launches_per_step = TOKENS * LAYERS
     plane_bytes = layers[0].packed_bytes()
     bytes_per_step = plane_bytes * launches_per_step
     algo_bytes_per_launch = plane_bytes + 2 * K_PLANES * (N_OUT + K_IN) + 2 * K_IN + 4 * N_OUT
 
-    for _ in range(max(3, args.warmup)):
-        graph.replay()
-    torch.cuda.synchronize()
+    graph = capture(step_streams)
     sampler = ClockSampler(gpu_uuid(torch))
     sampler.start()
     time.sleep(0.05)
-    dist.barrier()
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        graph.replay()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    dist.barrier()
+    t_local = time_graph(graph, args.steps)
     clocks = sampler.stop()
-    t_local = ev0.elapsed_time(ev1) / 1e3
     t_max = dist.max(t_local, dev)
     value = throughput(bytes_per_step, dist.world, args.steps, t_max)
     avg_launch_s = t_local / (args.steps * launches_per_step)
     achieved = algo_bytes_per_launch / avg_launch_s / 1e9
+    del graph
 
-    # ---- e2e: host X in pinned memory -> device, 96-layer chain per token, Y of the last layer -> host
+    chain_graph = capture(step_chain)
+    chain_steps = max(1, min(args.steps, 50))
+    t_chain = dist.max(time_graph(chain_graph, chain_steps), dev)
+    chain = {"GBps": throughput(bytes_per_step, dist.world, chain_steps, t_chain),
+             "us_per_layer": t_chain / (chain_steps * launches_per_step) * 1e6,
+             "what": "one stream, each rb_gemv launched with PDL after the previous one (dependent decode chain)"}
+    del chain_graph
+
+    # ---- e2e: host X in pinned memory -> device, the step, Y of the last layer -> host
     X_pin = torch.from_numpy(X_host.view(np.int16).copy()).pin_memory()
     Y_pin = torch.empty(TOKENS, N_OUT, dtype=torch.float32).pin_memory()
-    graph_e2e = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_e2e, stream=stream):
-        X.copy_(X_pin, non_blocking=True)
-        step(stream)
-        Y_pin.copy_(Y_last, non_blocking=True)
-    torch.cuda.synchronize()
-    for _ in range(3):
-        graph_e2e.replay()
-        stream.synchronize()
+    graph_e2e = capture(step_streams, pre=lambda: X.copy_(X_pin, non_blocking=True),
+                        post=lambda: Y_pin.copy_(Y_last, non_blocking=True))
     e2e_steps = max(1, min(args.steps, 200))
-    dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        graph_e2e.replay()
-        stream.synchronize()               # the host reads each step's result
-    e1.record(stream)
-    torch.cuda.synchronize()
-    t_e2e = dist.max(e0.elapsed_time(e1) / 1e3, dev)
+    t_e2e = dist.max(time_graph(graph_e2e, e2e_steps, sync_each=True), dev)
     e2e = {"value": throughput(bytes_per_step, dist.world, e2e_steps, t_e2e), "unit": "GB/s",
            "h2d_bytes_per_step": X_pin.numel() * 2, "d2h_bytes_per_step": Y_pin.numel() * 4,
            "steps": e2e_steps}
-    del graph, graph_e2e
+    del graph_e2e
 
     rows = other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak) if (dist.rank == 0 and not args.quick) else {}
     dist.barrier()
@@ -372,6 +396,7 @@ def run_rbw(args, dist: Dist):
                                 "algorithmic_bytes_per_launch": algo_bytes_per_launch,
                                 "avg_launch_us": avg_launch_s * 1e6},
                    "cpu_baseline": cb, "e2e": e2e, "gpu_launches": args.steps * launches_per_step,
+                   "decode_chain": chain,
                    "clocks": clocks, "rows": rows})
         print(json.dumps(line), flush=True)
     dist.close()
@@ -409,7 +434,7 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
         L.g16.copy_(Lp.g16)
         L.h16.copy_(Lp.h16)
         layers.append(L)
-    for M in (4, 16):
+    for M in (1, 4, 16):
         X = torch.from_numpy(synth.activations(M, K_IN, seed=M).view(np.int16)).to(dev)
         Y = torch.empty(M, N_OUT, dtype=torch.float32, device=dev)
         ws = rbw.workspace(rbw.gemv_workspace_bytes(N_OUT, K_IN, K_PLANES, M), dev)
@@ -418,7 +443,7 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
         def f():
             rbw.gemv(layers[next(it) % LAYERS], X, Y=Y, ws=ws, stream=stream)
         t = time_events(torch, f, 2 * LAYERS, stream)
-        out["gemv_M%d" % M] = {"us": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
+        out["gemv_M%d_plain_launches" % M] = {"us": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
                                "tokens_per_s": M / t}
     # rb_gemm at M = 2048 on the prefill shape
     try:
@@ -447,11 +472,57 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="skip the extra per-row timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--mode", choices=["full", "gemv-kernel", "pack-kernel", "gemm-kernel"], default="full",
+                    help="kernel-only modes run one kernel a few times (used for ncu captures)")
+    ap.add_argument("--launches", type=int, default=20)
+    ap.add_argument("--M", type=int, default=1)
     args = ap.parse_args(argv)
     dist = Dist()
     if args.impl == "reference":
         return run_reference(args, dist)
+    if args.mode != "full":
+        return run_kernel_mode(args)
     return run_rbw(args, dist)
+
+
+def run_kernel_mode(args):
+    """Launch one kernel `--launches` times on the workload layer (distinct buffers), no graph."""
+    import torch
+    from residual_binarized_weight_b200 import rbw, synth
+    dev = torch.device("cuda", 0)
+    wl = synth.workload(WORKLOAD)
+    W = torch.from_numpy(synth.weights(wl.layers[0])).to(dev)
+    g, h = rbw.svid_greedy(W, K_PLANES, iters=20)
+    base = rbw.pack(W, g, h, K_PLANES)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    if args.mode == "pack-kernel":
+        for _ in range(args.launches):
+            rbw.pack(W, g, h, K_PLANES, out=base)
+    else:
+        nl = 32
+        layers = []
+        for _ in range(nl):
+            L = rbw.PackedLayer(N_OUT, K_IN, K_PLANES, dev)
+            L.planes.copy_(base.planes)
+            L.g16.copy_(base.g16)
+            L.h16.copy_(base.h16)
+            layers.append(L)
+        M = args.M
+        X = torch.from_numpy(synth.activations(M, K_IN, seed=M).view(np.int16)).to(dev)
+        Y = torch.empty(M, N_OUT, dtype=torch.float32, device=dev)
+        if args.mode == "gemv-kernel":
+            ws = rbw.workspace(rbw.gemv_workspace_bytes(N_OUT, K_IN, K_PLANES, M), dev)
+            for j in range(args.launches):
+                rbw.gemv(layers[j % nl], X, Y=Y, ws=ws)
+        else:
+            ws = rbw.workspace(rbw.gemm_workspace_bytes(N_OUT, K_IN, K_PLANES, M), dev)
+            for j in range(args.launches):
+                rbw.gemm(layers[j % nl], X, Y=Y, ws=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"mode": args.mode, "launches": args.launches, "M": args.M,
+                      "wall_s": time.perf_counter() - t0}), flush=True)
+    return 0
 
 
 if __name__ == "__main__":

@@ -121,10 +121,12 @@ RB_API rb_status rb_pack(const float *W, const float *g, const float *h,
  * element-wise scaling only).
  *   X   [M][K] bfloat16 bit patterns.
  *   Y   [M][N] fp32 or bfloat16 (y_dtype), written, never read.
- *   workspace: rb_gemv_workspace_bytes(N, K, k, M) bytes of device memory,
- *   zero-filled by the caller before its first use; every call leaves it
- *   zero-filled again.  Calls that share a workspace must not overlap on the
- *   GPU (same stream, or PDL, is fine).
+ *   workspace: rb_gemv_workspace_bytes(N, K, k, M) bytes of device memory
+ *   (0 when the call needs none).  It holds per-slice fp32 partial sums and
+ *   per-row-tile arrival counters; it must be zero-filled before its first
+ *   use, and every call returns the counters to zero, so later calls need no
+ *   clearing.  Calls that share a workspace must not overlap on the GPU
+ *   (same stream, with or without RB_LAUNCH_PDL, is fine).
  * h_i .* x is formed exactly in fp32 and every sum is accumulated in fp32.
  */
 RB_API size_t rb_gemv_workspace_bytes(int n_out, int k_in, int k_planes, int M);

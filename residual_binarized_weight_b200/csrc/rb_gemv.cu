@@ -31,62 +31,80 @@ constexpr int kLutWarps = kLutThreads / 32;
 // entry (byte, group) of plane i at region(i/2) + byte*256 + (i%2)*128 + group*4.
 __host__ __device__ constexpr int lut_smem_bytes(int kp) { return ((kp + 1) / 2) * 65536; }
 
+// Prefetch depth of the byte-table kernel: row tiles per warp held in registers.
+constexpr int kLutPF = 2;
+
 template <int KP>
-__global__ void __launch_bounds__(kLutThreads, 1)
+__device__ __forceinline__ void lut_load_tile(uint32_t (&wd)[KP][8], const uint32_t* __restrict__ planes,
+                                              int s, int64_t t, int64_t S, int64_t Nt, int lane)
+{
+#pragma unroll
+    for (int i = 0; i < KP; ++i) {
+        const uint32_t* blk = planes + block_index(i, s, t, S, Nt) * 256 + lane;
+#pragma unroll
+        for (int sl = 0; sl < 8; ++sl) wd[i][sl] = __ldcs(blk + sl * 32);
+    }
+}
+
+template <int KP>
+__global__ void __launch_bounds__(kLutThreads, 2)
 gemv_lut_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ g16,
                 const uint16_t* __restrict__ h16, const uint16_t* __restrict__ X,
                 int N, int K, int C, float* __restrict__ partial,
                 unsigned* __restrict__ counters, void* __restrict__ Y, int ydt)
 {
     extern __shared__ __align__(1024) float lut[];
+    __shared__ int s_last;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t S = num_slices(K), Nt = num_row_tiles(N);
     const int s = blockIdx.x / C, cta = blockIdx.x % C;
     const int64_t t_begin = Nt * cta / C, t_end = Nt * (cta + 1) / C;
 
-    // Weights never depend on the previous kernel: start streaming them first.
-    uint32_t wd[KP][8];
-    int64_t t = t_begin + warp;
-    if (t < t_end) {
+    // ---- before the dependency wait: everything that does not depend on X.
+    // Weights of this warp's first kLutPF row tiles, their g values, this
+    // thread's h values for the table build.
+    uint32_t wd[kLutPF][KP][8];
+    float gv[kLutPF][KP];
 #pragma unroll
-        for (int i = 0; i < KP; ++i) {
-            const uint32_t* blk = planes + block_index(i, s, t, S, Nt) * 256 + lane;
+    for (int p = 0; p < kLutPF; ++p) {
+        const int64_t t = t_begin + warp + (int64_t)p * kLutWarps;
+        if (t < t_end) {
+            lut_load_tile<KP>(wd[p], planes, s, t, S, Nt, lane);
+            const int64_t r = t * 32 + lane;
 #pragma unroll
-            for (int sl = 0; sl < 8; ++sl) wd[i][sl] = __ldcs(blk + sl * 32);
+            for (int i = 0; i < KP; ++i)
+                gv[p][i] = r < N ? __half2float(__ushort_as_half(g16[(int64_t)i * N + r])) : 0.0f;
         }
     }
+    const int gg = threadIdx.x & 31, part = threadIdx.x >> 5;
+    const int64_t c0 = (int64_t)s * 256 + gg * 8;
+    const bool col_ok = c0 < K;
+    uint4 hr[KP];
+#pragma unroll
+    for (int i = 0; i < KP; ++i)
+        hr[i] = col_ok ? *reinterpret_cast<const uint4*>(h16 + (int64_t)i * K + c0) : make_uint4(0, 0, 0, 0);
+
     pdl_launch_dependents();
     pdl_wait();
 
     // ---- byte tables of slice s: thread (group gg, part) writes bytes 32*part .. +31
     {
-        const int gg = threadIdx.x & 31, part = threadIdx.x >> 5;
-        const int64_t c0 = (int64_t)s * 256 + gg * 8;
         float xv[8];
-        const bool ok = c0 < K;
-        if (ok) {
-            const uint4 xr = *reinterpret_cast<const uint4*>(X + c0);
-            const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+        const uint4 xr = col_ok ? *reinterpret_cast<const uint4*>(X + c0) : make_uint4(0, 0, 0, 0);
+        const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                xv[2 * q] = bf16_bits_to_f32(xw[q] & 0xffffu);
-                xv[2 * q + 1] = bf16_bits_to_f32(xw[q] >> 16);
-            }
+        for (int q = 0; q < 4; ++q) {
+            xv[2 * q] = bf16_bits_to_f32(xw[q] & 0xffffu);
+            xv[2 * q + 1] = bf16_bits_to_f32(xw[q] >> 16);
         }
 #pragma unroll
         for (int i = 0; i < KP; ++i) {
             float v[8];
-            if (ok) {
-                const uint4 hr = *reinterpret_cast<const uint4*>(h16 + (int64_t)i * K + c0);
-                const uint32_t hw[4] = {hr.x, hr.y, hr.z, hr.w};
+            const uint32_t hw[4] = {hr[i].x, hr[i].y, hr[i].z, hr[i].w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    v[2 * q] = __half2float(__ushort_as_half((unsigned short)(hw[q] & 0xffffu))) * xv[2 * q];
-                    v[2 * q + 1] = __half2float(__ushort_as_half((unsigned short)(hw[q] >> 16))) * xv[2 * q + 1];
-                }
-            } else {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) v[q] = 0.0f;
+            for (int q = 0; q < 4; ++q) {
+                v[2 * q] = __half2float(__ushort_as_half((unsigned short)(hw[q] & 0xffffu))) * xv[2 * q];
+                v[2 * q + 1] = __half2float(__ushort_as_half((unsigned short)(hw[q] >> 16))) * xv[2 * q + 1];
             }
             float L[16];                       // signed sums of columns 0..3 of the group
             L[0] = -((v[0] + v[1]) + (v[2] + v[3]));
@@ -96,7 +114,7 @@ gemv_lut_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict_
                 const int q = low == 1 ? 0 : low == 2 ? 1 : low == 4 ? 2 : 3;
                 L[n] = L[n & (n - 1)] + 2.0f * v[q];
             }
-            float Hh[2];                       // signed sums of columns 4..7 for the two high nibbles
+            float Hh[2];                       // signed sums of columns 4..7 for this part's high nibbles
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int n = 2 * part + e;
@@ -130,62 +148,65 @@ gemv_lut_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict_
         SEL[b] = (uint32_t)(4 + b) | ((uint32_t)(b ^ (lane & 3)) << 4) |
                  ((uint32_t)(12 + b) << 8) | ((uint32_t)(12 + b) << 12);
     const char* tb = reinterpret_cast<const char*>(lut);
+    const int64_t Ntp = Nt * 32;
 
-    for (; t < t_end; t += kLutWarps) {
-        uint32_t cur[KP][8];
+    for (int64_t t0 = t_begin + warp; t0 < t_end; t0 += (int64_t)kLutPF * kLutWarps) {
 #pragma unroll
-        for (int i = 0; i < KP; ++i)
-#pragma unroll
-            for (int sl = 0; sl < 8; ++sl) cur[i][sl] = wd[i][sl];
-        const int64_t tn = t + kLutWarps;
-        if (tn < t_end) {
+        for (int p = 0; p < kLutPF; ++p) {
+            const int64_t t = t0 + (int64_t)p * kLutWarps;
+            if (t >= t_end) break;
+            float acc[KP];
 #pragma unroll
             for (int i = 0; i < KP; ++i) {
-                const uint32_t* blk = planes + block_index(i, s, tn, S, Nt) * 256 + lane;
+                float a0 = 0.0f, a1 = 0.0f;
+                const char* tp = tb + (i >> 1) * 65536 + (i & 1) * 128;
 #pragma unroll
-                for (int sl = 0; sl < 8; ++sl) wd[i][sl] = __ldcs(blk + sl * 32);
-            }
-        }
-        float acc[KP];
+                for (int sl = 0; sl < 8; ++sl) {
 #pragma unroll
-        for (int i = 0; i < KP; ++i) {
-            float a0 = 0.0f, a1 = 0.0f;
-            const char* tp = tb + (i >> 1) * 65536 + (i & 1) * 128;
-#pragma unroll
-            for (int sl = 0; sl < 8; ++sl) {
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const uint32_t off = prmt(cur[i][sl], G[sl], SEL[b]);
-                    const float e = *reinterpret_cast<const float*>(tp + off);
-                    if (b & 1) a1 += e; else a0 += e;
+                    for (int b = 0; b < 4; ++b) {
+                        const uint32_t off = prmt(wd[p][i][sl], G[sl], SEL[b]);
+                        const float e = *reinterpret_cast<const float*>(tp + off);
+                        if (b & 1) a1 += e; else a0 += e;
+                    }
                 }
+                acc[i] = a0 + a1;
             }
-            acc[i] = a0 + a1;
-        }
-        const int64_t r = t * 32 + lane;
-        float p = 0.0f;
-        if (r < N) {
+            float pr = 0.0f;
 #pragma unroll
-            for (int i = 0; i < KP; ++i)
-                p += __half2float(__ushort_as_half(g16[(int64_t)i * N + r])) * acc[i];
-        }
-        if (S == 1) {
-            if (r < N) store_y(Y, ydt, r, p);
-            continue;
-        }
-        partial[(int64_t)s * Nt * 32 + t * 32 + lane] = p;
-        __threadfence();
-        unsigned prev = 0;
-        if (lane == 0) prev = atomicAdd(counters + t, 1u);
-        prev = __shfl_sync(0xffffffffu, prev, 0);
-        if (prev == (unsigned)(S - 1)) {              // last slice of this row tile
-            __threadfence();
-            float y = 0.0f;
-            for (int64_t s2 = 0; s2 < S; ++s2) y += __ldcg(partial + s2 * Nt * 32 + t * 32 + lane);
-            if (r < N) store_y(Y, ydt, r, y);
-            if (lane == 0) counters[t] = 0u;
+            for (int i = 0; i < KP; ++i) pr += gv[p][i] * acc[i];
+            const int64_t r = t * 32 + lane;
+            if (S == 1) {
+                if (r < N) store_y(Y, ydt, r, pr);
+            } else {
+                partial[(int64_t)s * Ntp + r] = pr;
+            }
+            // refill this slot with the tile kLutPF rounds ahead
+            const int64_t tn = t + (int64_t)kLutPF * kLutWarps;
+            if (tn < t_end) {
+                lut_load_tile<KP>(wd[p], planes, s, tn, S, Nt, lane);
+                const int64_t rn = tn * 32 + lane;
+#pragma unroll
+                for (int i = 0; i < KP; ++i)
+                    gv[p][i] = rn < N ? __half2float(__ushort_as_half(g16[(int64_t)i * N + rn])) : 0.0f;
+            }
         }
     }
+    if (S == 1) return;
+
+    // ---- cross-slice sum: the last of the S CTAs that own row tiles [t_begin, t_end)
+    // adds the slice partials in slice order.
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(counters + cta, 1u) == (unsigned)(S - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int64_t r = t_begin * 32 + threadIdx.x; r < t_end * 32; r += kLutThreads) {
+        float y = 0.0f;
+        for (int64_t s2 = 0; s2 < S; ++s2) y += __ldcg(partial + s2 * Ntp + r);
+        if (r < N) store_y(Y, ydt, r, y);
+    }
+    if (threadIdx.x == 0) counters[cta] = 0u;
 }
 
 // ---------------------------------------------------------------- generic kernel

@@ -53,28 +53,26 @@ pack_kernel(const float* __restrict__ W, const float* __restrict__ g,
                 hv[i] = h[(int64_t)i * K + c];
                 gv[i] = my_row < N ? g[(int64_t)i * N + my_row] : 0.0f;
             }
+            // all 32 row segments in flight at once (4 KB per warp) before any arithmetic
+            float wv[32];
 #pragma unroll
-            for (int r0 = 0; r0 < 32; r0 += 8) {
-                float wv[8];
+            for (int j = 0; j < 32; ++j) {
+                const int64_t r = t * 32 + j;
+                wv[j] = r < N ? __ldcs(W + r * K + c) : 0.0f;
+            }
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int64_t r = t * 32 + r0 + j;
-                    wv[j] = r < N ? __ldcs(W + r * K + c) : 0.0f;
-                }
+            for (int j = 0; j < 32; ++j) {
+                const bool row_ok = (t * 32 + j) < N;
+                float R = wv[j];
+                bad |= !(fabsf(R) <= FLT_MAX);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const bool row_ok = (t * 32 + r0 + j) < N;
-                    float R = wv[j];
-                    bad |= !(fabsf(R) <= FLT_MAX);
-#pragma unroll
-                    for (int i = 0; i < KP; ++i) {
-                        const float gi = __shfl_sync(0xffffffffu, gv[i], r0 + j);
-                        const bool b = R >= 0.0f;               // sign(0) = +1, -0.0 too
-                        const float tt = __fmul_rn(gi, hv[i]);
-                        R = b ? __fsub_rn(R, tt) : __fadd_rn(R, tt);
-                        const uint32_t word = __ballot_sync(0xffffffffu, b);
-                        if (lane == r0 + j) mine[i] = row_ok ? word : 0u;
-                    }
+                for (int i = 0; i < KP; ++i) {
+                    const float gi = __shfl_sync(0xffffffffu, gv[i], j);
+                    const bool b = R >= 0.0f;               // sign(0) = +1, -0.0 too
+                    const float tt = __fmul_rn(gi, hv[i]);
+                    R = b ? __fsub_rn(R, tt) : __fadd_rn(R, tt);
+                    const uint32_t word = __ballot_sync(0xffffffffu, b);
+                    if (lane == j) mine[i] = row_ok ? word : 0u;
                 }
             }
         }
