@@ -1,16 +1,471 @@
-// rb_gemm.cu -- batched application on the tcgen05 tensor cores (in progress).
+// rb_gemm.cu -- batched application Y = X . What^T on the tcgen05 tensor cores,
+// What = sum_i diag(g_i) B_i diag(h_i)  (RaBiT, "Residual binarization"; the
+// k binary paths run side by side and are summed with their row scales).
+//
+// Per plane i the contraction D_i[n][m] = sum_c (s_i[n][c] h_i[c]) * X[m][c] is
+// a dense fp16 GEMM with fp32 accumulation:
+//   A_i = +-h_i  (sign expanded in registers, 128 output rows x 64 columns per
+//                 stage, written to tensor memory with tcgen05.st: the MMA
+//                 reads A straight from TMEM, so the expansion costs no shared
+//                 memory bandwidth),
+//   B   = X in fp16 (a pre-pass converts bf16 -> fp16, exact in the normal
+//                 range, and interleaves each 32-column group so that column
+//                 pair (j, j+16) of a sign word becomes one fp16x2 TMEM cell:
+//                 one shift + one LOP3 per two weights), loaded by TMA with a
+//                 128-byte swizzle,
+//   D_i = one fp32 accumulator per plane in TMEM (128 lanes x BT columns).
+// Epilogue: Y[m][n] = sum_i g_i[n] * D_i[n][m], one output row per TMEM lane,
+// so every store instruction writes 32 consecutive outputs.
+//
+// Warp roles (192 threads): warp 0 = TMA producer + TMEM allocator, warp 1 =
+// MMA issuer (one thread), warps 2..5 = sign expansion, then epilogue (warp w
+// owns TMEM lanes 32*(w%4) .. +31).  Every mbarrier wait is bounded: on expiry
+// the kernel raises RB_DEV_TIMEOUT in dev_status, drains what it issued,
+// frees its tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "rbw_internal.cuh"
+
+namespace rbw {
+namespace {
+
+constexpr int kBR = 128;          // output rows per CTA (MMA M, TMEM lanes)
+constexpr int kBK = 64;           // K per pipeline stage (one 128-byte swizzle row of fp16)
+constexpr int kSX = 4;            // X stages
+constexpr int kThreads = 192;
+constexpr uint32_t kSpinLimit = 1u << 26;
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.b32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Bounded wait; false (and the CTA abort flag set) once the limit is reached or
+// another thread of the CTA has already given up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t limit) {
+    for (uint32_t it = 0; it < limit; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 255u && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    return false;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+                 :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+                 :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+__device__ __forceinline__ void tc_st_32x32b_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+                 "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+                 "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+                 :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                    "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
+                    "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]),
+                    "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+                    "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+                 : "memory");
+}
+__device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+                   "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
+                   "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
+                   "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                 : "r"(taddr) : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ uint32_t lop3_sign(uint32_t shifted, uint32_t hpair) {
+    // (~shifted & 0x80008000) ^ hpair : a clear sign bit flips +h to -h
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xA6;" : "=r"(d) : "r"(shifted), "r"(0x80008000u), "r"(hpair));
+    return d;
+}
+
+// UMMA shared-memory descriptor: K-major operand, 128-byte swizzle, 8-row
+// groups 1024 bytes apart (SBO), sm100 descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+           ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 D, fp16 A and B, both K-major, N = bt, M = 128.
+__host__ __device__ constexpr uint32_t idesc_f16(int bt) {
+    return (1u << 4) | ((uint32_t)(bt >> 3) << 17) | ((uint32_t)(kBR >> 4) << 24);
+}
+
+__host__ __device__ constexpr int gemm_bt(int kp) { return kp <= 2 ? 128 : 64; }
+__host__ __device__ constexpr int gemm_sa(int kp) { return kp <= 2 ? 4 : 2; }
+__host__ __device__ constexpr int gemm_tmem_cols(int kp) {
+    return (kp * gemm_bt(kp) + gemm_sa(kp) * kp * 32) <= 256 ? 256 : 512;
+}
+__host__ __device__ constexpr int gemm_smem_bytes(int kp) { return kSX * gemm_bt(kp) * 128 + 1024 + 256; }
+
+// ---------------------------------------------------------------- pre-pass
+// X16[m][32q + 2j + e] = fp16(X[m][32q + j + 16e]);  hperm[i][16q + j] = (h[32q+j], h[32q+j+16]).
+__global__ void gemm_prepass_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ h16,
+                                    int M, int K, int kp, uint16_t* __restrict__ X16,
+                                    uint32_t* __restrict__ hperm, int32_t* dev_status)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    const int64_t groups = (int64_t)K / 32;
+    const int64_t nx = (int64_t)M * groups, nh = (int64_t)kp * groups;
+    int flags = 0;
+    for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < nx + nh;
+         it += (int64_t)gridDim.x * blockDim.x) {
+        if (it < nx) {
+            const int64_t m = it / groups, q = it % groups;
+            const uint4* src = reinterpret_cast<const uint4*>(X + m * K + q * 32);
+            uint32_t in[16];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const uint4 u = src[v];
+                in[4 * v] = u.x; in[4 * v + 1] = u.y; in[4 * v + 2] = u.z; in[4 * v + 3] = u.w;
+            }
+            uint32_t out[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const uint32_t lo = (j & 1) ? (in[j >> 1] >> 16) : (in[j >> 1] & 0xffffu);
+                const uint32_t hi = (j & 1) ? (in[8 + (j >> 1)] >> 16) : (in[8 + (j >> 1)] & 0xffffu);
+                const __half a = __float2half_rn(bf16_bits_to_f32(lo));
+                const __half b = __float2half_rn(bf16_bits_to_f32(hi));
+                if (__hisinf(a) || __hisinf(b)) flags |= RB_DEV_RANGE;
+                out[j] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(X16 + m * K + q * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(out[4 * v], out[4 * v + 1], out[4 * v + 2], out[4 * v + 3]);
+        } else {
+            const int64_t x = it - nx, i = x / groups, q = x % groups;
+            const uint16_t* hs = h16 + i * K + q * 32;
+            uint32_t* hd = hperm + i * (K / 2) + q * 16;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) hd[j] = (uint32_t)hs[j] | ((uint32_t)hs[j + 16] << 16);
+        }
+    }
+    if (flags) set_dev_status(dev_status, flags);
+}
+
+// ---------------------------------------------------------------- main kernel
+template <int KP>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ planes,
+               const uint16_t* __restrict__ g16, const uint32_t* __restrict__ hperm,
+               int N, int K, int M, void* __restrict__ Y, int ydt, int32_t* dev_status, uint32_t spin_limit)
+{
+    constexpr int BT = gemm_bt(KP), SA = gemm_sa(KP), NCOLS = gemm_tmem_cols(KP);
+    constexpr uint32_t X_STAGE = BT * 128;
+    constexpr uint32_t IDESC = idesc_f16(BT);
+    static_assert(KP * BT + SA * KP * 32 <= NCOLS, "tensor memory budget");
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base for the swizzled X stages
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (sbase - smem_u32(smem_raw));
+    const uint32_t xs0 = sbase;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + kSX * X_STAGE);
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_x = [&](int s) { return bar0 + 8u * s; };
+    auto empty_x = [&](int s) { return bar0 + 8u * (kSX + s); };
+    auto full_a = [&](int s) { return bar0 + 8u * (2 * kSX + s); };
+    auto empty_a = [&](int s) { return bar0 + 8u * (2 * kSX + SA + s); };
+    const uint32_t acc_full = bar0 + 8u * (2 * kSX + 2 * SA);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kSX + 2 * SA + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * kBR, m0 = blockIdx.y * BT;
+    const int nkb = (K + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kSX; ++s) { mbar_init(full_x(s), 1); mbar_init(empty_x(s), 1); }
+        for (int s = 0; s < SA; ++s) { mbar_init(full_a(s), 128); mbar_init(empty_a(s), 1); }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" :: "l"(&tmap_x) : "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tmem_slot)), "r"((uint32_t)NCOLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_launch_dependents();
+    pdl_wait();                                   // X16 / hperm come from the pre-pass
+
+    if (warp == 0) {
+        if (lane == 0) {                          // ---------------- TMA producer
+            int issued = 0;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % kSX, j = kb / kSX;
+                if (j > 0 && !mbar_wait(empty_x(s), (j - 1) & 1, abort_flag, spin_limit)) break;
+                mbar_arrive_expect_tx(full_x(s), X_STAGE);
+                tma_load_2d(xs0 + s * X_STAGE, &tmap_x, full_x(s), kb * kBK, m0);
+                ++issued;
+            }
+            if (*abort_flag) {                    // drain the loads this thread issued
+                for (int kb = issued - kSX < 0 ? 0 : issued - kSX; kb < issued; ++kb)
+                    for (uint32_t it = 0; it < spin_limit && !mbar_try_wait(full_x(kb % kSX), (kb / kSX) & 1); ++it) {}
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {                          // ---------------- MMA issuer
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % kSX, sa = kb % SA;
+                if (!mbar_wait(full_x(s), (kb / kSX) & 1, abort_flag, spin_limit)) break;
+                if (!mbar_wait(full_a(sa), (kb / SA) & 1, abort_flag, spin_limit)) break;
+                tc_fence_after();
+                const uint32_t xaddr = xs0 + s * X_STAGE;
+#pragma unroll
+                for (int i = 0; i < KP; ++i) {
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint32_t a_t = tmem + (uint32_t)(KP * BT + (sa * KP + i) * 32 + kk * 8);
+                        const uint32_t d_t = tmem + (uint32_t)(i * BT);
+                        tc_mma_f16_ts(d_t, a_t, smem_desc_sw128(xaddr + kk * 32), IDESC,
+                                      (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                tc_commit(empty_x(s));
+                tc_commit(empty_a(sa));
+            }
+            tc_commit(acc_full);                  // arrives once every MMA issued above is done
+        }
+    } else {                                      // ---------------- expansion, then epilogue
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const int64_t n = (int64_t)n0 + r;
+        const int64_t S = num_slices(K), Nt = num_row_tiles(N);
+        const int64_t tile = n >> 5;
+        const bool tile_ok = tile < Nt;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        bool ok = true;
+        for (int kb = 0; kb < nkb && ok; ++kb) {
+            const int sa = kb % SA;
+            if (kb >= SA) {
+                if (!mbar_wait(empty_a(sa), ((kb / SA) - 1) & 1, abort_flag, spin_limit)) { ok = false; break; }
+                tc_fence_after();
+            }
+            const int64_t sl = kb / 4;
+            const int w0 = (kb & 3) * 2;
+#pragma unroll
+            for (int i = 0; i < KP; ++i) {
+                uint32_t wv[2];
+#pragma unroll
+                for (int ww = 0; ww < 2; ++ww) {
+                    const int64_t col0 = (int64_t)kb * kBK + ww * 32;
+                    wv[ww] = (tile_ok && col0 < K)
+                        ? planes[block_index(i, sl, tile, S, Nt) * 256 + (((w0 + ww) ^ (lane >> 2)) * 32) + lane]
+                        : 0u;
+                }
+                uint32_t hp[32];
+                const int64_t hbase = (int64_t)i * (K / 2) + (int64_t)kb * 32;
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const int64_t idx = hbase + 4 * v;
+                    uint4 u = make_uint4(0, 0, 0, 0);
+                    if ((int64_t)kb * 32 + 4 * v < K / 2) u = *reinterpret_cast<const uint4*>(hperm + idx);
+                    hp[4 * v] = u.x; hp[4 * v + 1] = u.y; hp[4 * v + 2] = u.z; hp[4 * v + 3] = u.w;
+                }
+                uint32_t a[32];
+#pragma unroll
+                for (int ww = 0; ww < 2; ++ww)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        a[ww * 16 + j] = lop3_sign(wv[ww] << (15 - j), hp[ww * 16 + j]);
+                tc_st_32x32b_x32(tmem + lane_base + (uint32_t)(KP * BT + (sa * KP + i) * 32), a);
+            }
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(full_a(sa));
+        }
+        // ---- epilogue
+        if (ok && mbar_wait(acc_full, 0, abort_flag, spin_limit)) {
+            tc_fence_after();
+            float gi[KP];
+#pragma unroll
+            for (int i = 0; i < KP; ++i)
+                gi[i] = n < N ? __half2float(__ushort_as_half(g16[(int64_t)i * N + n])) : 0.0f;
+#pragma unroll 1
+            for (int c = 0; c < BT / 32; ++c) {
+                float y[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) y[j] = 0.0f;
+#pragma unroll
+                for (int i = 0; i < KP; ++i) {
+                    uint32_t v[32];
+                    tc_ld_32x32b_x32(tmem + lane_base + (uint32_t)(i * BT + c * 32), v);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) y[j] = fmaf(gi[i], __uint_as_float(v[j]), y[j]);
+                }
+                if (n < N) {
+#pragma unroll 4
+                    for (int j = 0; j < 32; ++j) {
+                        const int64_t m = (int64_t)m0 + c * 32 + j;
+                        if (m < M) store_y(Y, ydt, m * N + n, y[j]);
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- teardown: every MMA has completed (acc_full) or the CTA gave up
+    if (warp == 1 && lane == 0 && *abort_flag) {
+        for (uint32_t it = 0; it < spin_limit && !mbar_try_wait(acc_full, 0); ++it) {}
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag && threadIdx.x == 0) set_dev_status(dev_status, RB_DEV_TIMEOUT);
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                     :: "r"(tmem), "r"((uint32_t)NCOLS) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+struct GemmWs {
+    uint16_t* x16;
+    uint32_t* hperm;
+    size_t bytes;
+};
+
+GemmWs gemm_ws_layout(int K, int kp, int M, void* base)
+{
+    GemmWs w;
+    const size_t xb = ((size_t)M * K * 2 + 255) / 256 * 256;
+    const size_t hb = ((size_t)kp * K * 2 + 255) / 256 * 256;
+    w.x16 = reinterpret_cast<uint16_t*>(base);
+    w.hperm = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(base) + xb);
+    w.bytes = xb + hb;
+    return w;
+}
+
+template <int KP>
+rb_status launch_gemm(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs& ws,
+                      int32_t* dev_status, bool pdl, cudaStream_t stream, uint32_t spin_limit)
+{
+    constexpr int BT = gemm_bt(KP);
+    PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
+    if (!enc) return RB_ERR_CUDA;
+    CUtensorMap map;
+    const cuuint64_t gdim[2] = {(cuuint64_t)L->k_in, (cuuint64_t)M};
+    const cuuint64_t gstride[1] = {(cuuint64_t)L->k_in * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BT};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ws.x16, gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return RB_ERR_CUDA;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int smem = gemm_smem_bytes(KP);
+    if (dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(gemm_tc_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return RB_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    dim3 grid((unsigned)((L->n_out + kBR - 1) / kBR), (unsigned)((M + BT - 1) / BT));
+    return launch(gemm_tc_kernel<KP>, grid, dim3(kThreads), (size_t)smem, stream, pdl, map, L->planes,
+                  L->g16, (const uint32_t*)ws.hperm, L->n_out, L->k_in, M, Y, ydt, dev_status, spin_limit);
+}
+
+}  // namespace
+
+// Internal entry used by the tests of the bounded-wait path: the same kernel with a
+// caller-chosen spin limit.
+rb_status gemm_with_spin_limit(const rb_layer_t* layer, const uint16_t* X, int M, void* Y, rb_dtype y_dtype,
+                               void* workspace, size_t workspace_bytes, int32_t* dev_status, unsigned flags,
+                               cudaStream_t stream, uint32_t spin_limit)
+{
+    rb_status st = check_apply_args(layer, X, M, Y, y_dtype, flags);
+    if (st != RB_OK) return st;
+    if (layer->k_planes > 4) return RB_ERR_UNSUPPORTED;
+    if (dev_status && !aligned16(dev_status)) return RB_ERR_ALIGN;
+    GemmWs ws = gemm_ws_layout(layer->k_in, layer->k_planes, M, workspace);
+    if (!workspace || workspace_bytes < ws.bytes) return RB_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return RB_ERR_ALIGN;
+    if (!device_is_sm100()) return RB_ERR_UNSUPPORTED;
+    const bool pdl = (flags & RB_LAUNCH_PDL) != 0;
+    const int64_t groups = layer->k_in / 32;
+    int64_t items = (int64_t)M * groups + (int64_t)layer->k_planes * groups;
+    int64_t ctas = (items + 255) / 256;
+    if (ctas > 8 * num_sms()) ctas = 8 * num_sms();
+    st = launch(gemm_prepass_kernel, dim3((unsigned)ctas), dim3(256), 0, stream, pdl, X, layer->h16, M,
+                layer->k_in, layer->k_planes, ws.x16, ws.hperm, dev_status);
+    if (st != RB_OK) return st;
+    switch (layer->k_planes) {
+        case 1: return launch_gemm<1>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, spin_limit);
+        case 2: return launch_gemm<2>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, spin_limit);
+        case 3: return launch_gemm<3>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, spin_limit);
+        default: return launch_gemm<4>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, spin_limit);
+    }
+}
+
+}  // namespace rbw
+
+using namespace rbw;
 
 extern "C" size_t rb_gemm_workspace_bytes(int n_out, int k_in, int k_planes, int M)
 {
-    if (n_out < 1 || k_in < 32 || k_in % 32 != 0 || k_planes < 1 || k_planes > 8 || M < 1) return 0;
-    return ((size_t)M * (size_t)k_in * 2 + 255) / 256 * 256;
+    if (n_out < 1 || k_in < 32 || k_in % 32 != 0 || k_planes < 1 || k_planes > 4 || M < 1) return 0;
+    return gemm_ws_layout(k_in, k_planes, M, nullptr).bytes;
 }
 
 extern "C" rb_status rb_gemm(const rb_layer_t* layer, const uint16_t* X, int M, void* Y, rb_dtype y_dtype,
-                             void*, size_t, int32_t*, unsigned flags, cudaStream_t)
+                             void* workspace, size_t workspace_bytes, int32_t* dev_status, unsigned flags,
+                             cudaStream_t stream)
 {
-    rb_status st = rbw::check_apply_args(layer, X, M, Y, y_dtype, flags);
-    if (st != RB_OK) return st;
-    return RB_ERR_UNSUPPORTED;
+    return gemm_with_spin_limit(layer, X, M, Y, y_dtype, workspace, workspace_bytes, dev_status, flags,
+                                stream, kSpinLimit);
 }

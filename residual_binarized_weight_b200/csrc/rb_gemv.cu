@@ -203,7 +203,13 @@ gemv_lut_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict_
     __threadfence();
     for (int64_t r = t_begin * 32 + threadIdx.x; r < t_end * 32; r += kLutThreads) {
         float y = 0.0f;
-        for (int64_t s2 = 0; s2 < S; ++s2) y += __ldcg(partial + s2 * Ntp + r);
+        for (int64_t sb = 0; sb < S; sb += 16) {        // 16 independent L2 loads in flight
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = (sb + j < S) ? __ldcg(partial + (sb + j) * Ntp + r) : 0.0f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) y += v[j];
+        }
         if (r < N) store_y(Y, ydt, r, y);
     }
     if (threadIdx.x == 0) counters[cta] = 0u;

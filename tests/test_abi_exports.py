@@ -88,7 +88,8 @@ def test_apply_argument_errors_on_host(L):
         assert fn(ctypes.byref(bad), a, 1, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_SHAPE
         res = rbw.RbLayer(64, 256, 2, 1, 0x10000, 0x10000, 0x10000)
         assert fn(ctypes.byref(res), a, 1, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_ARG
-        assert fn(ctypes.byref(lay), a, 1, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_UNSUPPORTED
+        assert fn(ctypes.byref(lay), a, 1, a, 0, a, 1 << 30, None, 0, None) == rbw.RB_ERR_UNSUPPORTED
+    assert L.rb_gemm(ctypes.byref(lay), a, 1, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_WORKSPACE
     assert L.rb_gemv(ctypes.byref(lay), a, 65, a, 0, None, 0, None, 0, None) == rbw.RB_ERR_SHAPE
     assert L.rb_gemv(ctypes.byref(lay), a, 1, a, 0, None, 0, None, 2, None) == rbw.RB_ERR_ARG
 

@@ -1,0 +1,88 @@
+"""rb_gemm (tcgen05 tensor-core path) parity against the float64 oracle.
+
+Prefill workloads run at their full sizes with sampled output rows and tokens
+(first, last, ragged tails, random); ragged shapes cover N not a multiple of
+128, M not a multiple of the token tile, K not a multiple of 64, every k the
+kernel serves (1..4), and both output types.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from residual_binarized_weight_b200 import rbw, synth
+from tests import cases
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gemm(L, X, ydt, ws=None, dev_status=None):
+    N, K, k = L.n_out, L.k_in, L.k_planes
+    M = X.shape[0]
+    ws = ws if ws is not None else rbw.workspace(rbw.gemm_workspace_bytes(N, K, k, M))
+    Y = rbw.gemm(L, cases.to_dev(X), ws=ws, y_dtype=ydt, dev_status=dev_status)
+    torch.cuda.synchronize()
+    return Y.float().cpu().numpy().astype(np.float64)
+
+
+def sample(n, count, seed):
+    rng = np.random.default_rng(seed)
+    idx = set(range(min(n, 40))) | set(range(max(0, n - 40), n))
+    idx |= set(rng.choice(n, size=min(n, count), replace=False).tolist())
+    return np.array(sorted(idx), np.int64)
+
+
+@pytest.mark.parametrize("wl,li,M", [(4, 0, 512), (4, 1, 512), (4, 0, 2048), (4, 1, 2048), (3, 0, 64)])
+@pytest.mark.parametrize("ydt", [torch.float32, torch.bfloat16])
+def test_gemm_workloads(wl, li, M, ydt):
+    w = synth.workload(wl)
+    k = 2
+    W, g, h = cases.layer_case(wl, li, k)
+    N, K = W.shape
+    planes, g16, h16 = cases.packed_case(wl, li, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    X = synth.activations_for(w, M, K)
+    st = torch.zeros(4, dtype=torch.int32, device="cuda")
+    Yg = run_gemm(L, X, ydt, dev_status=st)
+    assert int(st[0].item()) == 0
+    rows, toks = sample(N, 300, 1), sample(M, 60, 2)
+    Yr = oracle.apply(planes, g16, h16, N, K, k, X, rows=rows, toks=toks)
+    bound = cases.abs_bound(g16, h16, X[toks], rows)
+    cases.check_y(Yg[np.ix_(toks, rows)], Yr, bound, bf16=ydt == torch.bfloat16, per_elem=1e-4)
+
+
+@pytest.mark.parametrize("N,K,k,M", [(128, 64, 1, 128), (200, 288, 2, 130), (33, 800, 3, 65), (300, 544, 4, 1),
+                                     (4097, 256, 2, 7), (129, 1056, 1, 257), (64, 4096, 2, 300)])
+def test_gemm_ragged(N, K, k, M):
+    rng = np.random.default_rng(N + K + 5 * k + M)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=8)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    X = synth.activations(M, K, seed=N + M)
+    Yr = oracle.apply(planes, g16, h16, N, K, k, X)
+    for ydt in (torch.float32, torch.bfloat16):
+        Yg = run_gemm(L, X, ydt)
+        cases.check_y(Yg, Yr, cases.abs_bound(g16, h16, X), bf16=ydt == torch.bfloat16, per_elem=1e-4)
+
+
+def test_gemm_matches_gemv_small_m():
+    """For M <= 64 both entry points compute the same product (to fp32 rounding)."""
+    W, g, h = cases.layer_case(1, 0, 2)
+    N, K = W.shape
+    planes, g16, h16 = cases.packed_case(1, 0, 2)
+    L = cases.upload_layer(planes, g16, h16, N, K, 2)
+    X = synth.activations(16, K, seed=5)
+    Yg = run_gemm(L, X, torch.float32)
+    Yv = rbw.gemv(L, cases.to_dev(X), ws=rbw.workspace(rbw.gemv_workspace_bytes(N, K, 2, 16)))
+    torch.cuda.synchronize()
+    Yv = Yv.cpu().numpy().astype(np.float64)
+    assert np.linalg.norm(Yg - Yv) / np.linalg.norm(Yv) < 1e-5
+
+
+def test_gemm_k_above_4_unsupported():
+    N, K, k = 64, 256, 5
+    L = rbw.PackedLayer(N, K, k)
+    with pytest.raises(rbw.RbError) as e:
+        rbw.gemm(L, torch.zeros(8, K, dtype=torch.int16, device="cuda"), ws=rbw.workspace(1 << 20))
+    assert e.value.status == rbw.RB_ERR_UNSUPPORTED
