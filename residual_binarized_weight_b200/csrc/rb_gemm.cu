@@ -34,7 +34,7 @@ constexpr int kBR = 128;          // output rows per CTA (MMA M, TMEM lanes)
 constexpr int kBK = 64;           // K per pipeline stage (one 128-byte swizzle row of fp16)
 constexpr int kSX = 4;            // X stages
 constexpr int kThreads = 192;
-constexpr uint32_t kSpinLimit = 1u << 26;
+constexpr uint64_t kTimeoutNs = 1000000000ull;   // 1 s per wait
 
 // ---------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -54,16 +54,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
                  : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
-// Bounded wait; false (and the CTA abort flag set) once the limit is reached or
-// another thread of the CTA has already given up.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait: gives up after timeout_ns, or as soon as another thread of the
+// CTA (abort_flag) or another CTA (RB_DEV_TIMEOUT in dev_status) has given up.
+// A thread that times out raises both flags.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t limit) {
-    for (uint32_t it = 0; it < limit; ++it) {
+                                          int32_t* dev_status, uint64_t timeout_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 255u && *abort_flag) return false;
+        if ((it & 1023u) == 0u) {
+            if (*abort_flag) return false;
+            if (dev_status && (*reinterpret_cast<volatile int32_t*>(dev_status) & RB_DEV_TIMEOUT)) {
+                *abort_flag = 1;
+                return false;
+            }
+            if (globaltimer_ns() - t0 > timeout_ns) {
+                *abort_flag = 1;
+                set_dev_status(dev_status, RB_DEV_TIMEOUT);
+                return false;
+            }
+        }
     }
-    *abort_flag = 1;
-    return false;
+}
+// Warp-uniform form for code that continues with .sync.aligned instructions.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               int32_t* dev_status, uint64_t timeout_ns) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, dev_status, timeout_ns) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
     asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
@@ -182,7 +206,7 @@ template <int KP>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ planes,
                const uint16_t* __restrict__ g16, const uint32_t* __restrict__ hperm,
-               int N, int K, int M, void* __restrict__ Y, int ydt, int32_t* dev_status, uint32_t spin_limit)
+               int N, int K, int M, void* __restrict__ Y, int ydt, int32_t* dev_status, uint64_t timeout_ns)
 {
     constexpr int BT = gemm_bt(KP), SA = gemm_sa(KP), NCOLS = gemm_tmem_cols(KP);
     constexpr uint32_t X_STAGE = BT * 128;
@@ -233,22 +257,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
             int issued = 0;
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % kSX, j = kb / kSX;
-                if (j > 0 && !mbar_wait(empty_x(s), (j - 1) & 1, abort_flag, spin_limit)) break;
+                if (j > 0 && !mbar_wait(empty_x(s), (j - 1) & 1, abort_flag, dev_status, timeout_ns)) break;
                 mbar_arrive_expect_tx(full_x(s), X_STAGE);
                 tma_load_2d(xs0 + s * X_STAGE, &tmap_x, full_x(s), kb * kBK, m0);
                 ++issued;
             }
-            if (*abort_flag) {                    // drain the loads this thread issued
+            if (*abort_flag) {                    // drain the loads this thread issued (bounded)
+                const uint64_t t0 = globaltimer_ns();
                 for (int kb = issued - kSX < 0 ? 0 : issued - kSX; kb < issued; ++kb)
-                    for (uint32_t it = 0; it < spin_limit && !mbar_try_wait(full_x(kb % kSX), (kb / kSX) & 1); ++it) {}
+                    while (!mbar_try_wait(full_x(kb % kSX), (kb / kSX) & 1) && globaltimer_ns() - t0 < timeout_ns) {}
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {                          // ---------------- MMA issuer
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % kSX, sa = kb % SA;
-                if (!mbar_wait(full_x(s), (kb / kSX) & 1, abort_flag, spin_limit)) break;
-                if (!mbar_wait(full_a(sa), (kb / SA) & 1, abort_flag, spin_limit)) break;
+                if (!mbar_wait(full_x(s), (kb / kSX) & 1, abort_flag, dev_status, timeout_ns)) break;
+                if (!mbar_wait(full_a(sa), (kb / SA) & 1, abort_flag, dev_status, timeout_ns)) break;
                 tc_fence_after();
                 const uint32_t xaddr = xs0 + s * X_STAGE;
 #pragma unroll
@@ -278,7 +303,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
         for (int kb = 0; kb < nkb && ok; ++kb) {
             const int sa = kb % SA;
             if (kb >= SA) {
-                if (!mbar_wait(empty_a(sa), ((kb / SA) - 1) & 1, abort_flag, spin_limit)) { ok = false; break; }
+                if (!mbar_wait_warp(empty_a(sa), ((kb / SA) - 1) & 1, abort_flag, dev_status, timeout_ns)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
             }
             const int64_t sl = kb / 4;
@@ -315,7 +343,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
             mbar_arrive(full_a(sa));
         }
         // ---- epilogue
-        if (ok && mbar_wait(acc_full, 0, abort_flag, spin_limit)) {
+        if (ok && mbar_wait_warp(acc_full, 0, abort_flag, dev_status, timeout_ns)) {
             tc_fence_after();
             float gi[KP];
 #pragma unroll
@@ -335,7 +363,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
                     for (int j = 0; j < 32; ++j) y[j] = fmaf(gi[i], __uint_as_float(v[j]), y[j]);
                 }
                 if (n < N) {
-#pragma unroll 4
+#pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int64_t m = (int64_t)m0 + c * 32 + j;
                         if (m < M) store_y(Y, ydt, m * N + n, y[j]);
@@ -346,8 +374,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
     }
 
     // ---- teardown: every MMA has completed (acc_full) or the CTA gave up
-    if (warp == 1 && lane == 0 && *abort_flag) {
-        for (uint32_t it = 0; it < spin_limit && !mbar_try_wait(acc_full, 0); ++it) {}
+    if (warp == 1 && lane == 0 && *abort_flag) {    // no MMA may still run when TMEM is freed
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(acc_full, 0) && globaltimer_ns() - t0 < timeout_ns) {}
     }
     tc_fence_before();
     __syncthreads();
@@ -392,7 +421,7 @@ GemmWs gemm_ws_layout(int K, int kp, int M, void* base)
 
 template <int KP>
 rb_status launch_gemm(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs& ws,
-                      int32_t* dev_status, bool pdl, cudaStream_t stream, uint32_t spin_limit)
+                      int32_t* dev_status, bool pdl, cudaStream_t stream, uint64_t timeout_ns)
 {
     constexpr int BT = gemm_bt(KP);
     PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
@@ -417,16 +446,15 @@ rb_status launch_gemm(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs
     }
     dim3 grid((unsigned)((L->n_out + kBR - 1) / kBR), (unsigned)((M + BT - 1) / BT));
     return launch(gemm_tc_kernel<KP>, grid, dim3(kThreads), (size_t)smem, stream, pdl, map, L->planes,
-                  L->g16, (const uint32_t*)ws.hperm, L->n_out, L->k_in, M, Y, ydt, dev_status, spin_limit);
+                  L->g16, (const uint32_t*)ws.hperm, L->n_out, L->k_in, M, Y, ydt, dev_status, timeout_ns);
 }
 
 }  // namespace
 
-// Internal entry used by the tests of the bounded-wait path: the same kernel with a
-// caller-chosen spin limit.
-rb_status gemm_with_spin_limit(const rb_layer_t* layer, const uint16_t* X, int M, void* Y, rb_dtype y_dtype,
+// rb_gemm with a caller-chosen bound on every device-side wait.
+rb_status gemm_with_timeout(const rb_layer_t* layer, const uint16_t* X, int M, void* Y, rb_dtype y_dtype,
                                void* workspace, size_t workspace_bytes, int32_t* dev_status, unsigned flags,
-                               cudaStream_t stream, uint32_t spin_limit)
+                               cudaStream_t stream, uint64_t timeout_ns)
 {
     rb_status st = check_apply_args(layer, X, M, Y, y_dtype, flags);
     if (st != RB_OK) return st;
@@ -445,10 +473,10 @@ rb_status gemm_with_spin_limit(const rb_layer_t* layer, const uint16_t* X, int M
                 layer->k_in, layer->k_planes, ws.x16, ws.hperm, dev_status);
     if (st != RB_OK) return st;
     switch (layer->k_planes) {
-        case 1: return launch_gemm<1>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, spin_limit);
-        case 2: return launch_gemm<2>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, spin_limit);
-        case 3: return launch_gemm<3>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, spin_limit);
-        default: return launch_gemm<4>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, spin_limit);
+        case 1: return launch_gemm<1>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, timeout_ns);
+        case 2: return launch_gemm<2>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, timeout_ns);
+        case 3: return launch_gemm<3>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, timeout_ns);
+        default: return launch_gemm<4>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, timeout_ns);
     }
 }
 
@@ -466,6 +494,6 @@ extern "C" rb_status rb_gemm(const rb_layer_t* layer, const uint16_t* X, int M, 
                              void* workspace, size_t workspace_bytes, int32_t* dev_status, unsigned flags,
                              cudaStream_t stream)
 {
-    return gemm_with_spin_limit(layer, X, M, Y, y_dtype, workspace, workspace_bytes, dev_status, flags,
-                                stream, kSpinLimit);
+    return gemm_with_timeout(layer, X, M, Y, y_dtype, workspace, workspace_bytes, dev_status, flags,
+                             stream, kTimeoutNs);
 }
