@@ -32,7 +32,7 @@ namespace {
 
 constexpr int kBR = 128;          // output rows per CTA (MMA M, TMEM lanes)
 constexpr int kBK = 64;           // K per pipeline stage (one 128-byte swizzle row of fp16)
-constexpr int kSX = 4;            // X stages
+constexpr int kSX = 8;            // X stages
 constexpr int kThreads = 192;
 constexpr uint64_t kTimeoutNs = 1000000000ull;   // 1 s per wait
 
@@ -299,9 +299,42 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
         const int64_t tile = n >> 5;
         const bool tile_ok = tile < Nt;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        // sign words and +-h pairs of one k-block, fetched one k-block ahead
+        auto load_kb = [&](int kb, uint32_t (&wv)[KP][2], uint32_t (&hp)[KP][32]) {
+            const int64_t sl = kb / 4;
+            const int w0 = (kb & 3) * 2;
+#pragma unroll
+            for (int i = 0; i < KP; ++i) {
+#pragma unroll
+                for (int ww = 0; ww < 2; ++ww) {
+                    const int64_t col0 = (int64_t)kb * kBK + ww * 32;
+                    wv[i][ww] = (tile_ok && col0 < K)
+                        ? planes[block_index(i, sl, tile, S, Nt) * 256 + (((w0 + ww) ^ (lane >> 2)) * 32) + lane]
+                        : 0u;
+                }
+                const int64_t hbase = (int64_t)i * (K / 2) + (int64_t)kb * 32;
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    uint4 u = make_uint4(0, 0, 0, 0);
+                    if ((int64_t)kb * 32 + 4 * v < K / 2) u = *reinterpret_cast<const uint4*>(hperm + hbase + 4 * v);
+                    hp[i][4 * v] = u.x; hp[i][4 * v + 1] = u.y; hp[i][4 * v + 2] = u.z; hp[i][4 * v + 3] = u.w;
+                }
+            }
+        };
+        uint32_t wv[KP][2], hp[KP][32];
+        load_kb(0, wv, hp);
         bool ok = true;
         for (int kb = 0; kb < nkb && ok; ++kb) {
             const int sa = kb % SA;
+            uint32_t cw[KP][2], ch[KP][32];
+#pragma unroll
+            for (int i = 0; i < KP; ++i) {
+                cw[i][0] = wv[i][0];
+                cw[i][1] = wv[i][1];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) ch[i][j] = hp[i][j];
+            }
+            if (kb + 1 < nkb) load_kb(kb + 1, wv, hp);
             if (kb >= SA) {
                 if (!mbar_wait_warp(empty_a(sa), ((kb / SA) - 1) & 1, abort_flag, dev_status, timeout_ns)) {
                     ok = false;
@@ -309,33 +342,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
                 }
                 tc_fence_after();
             }
-            const int64_t sl = kb / 4;
-            const int w0 = (kb & 3) * 2;
 #pragma unroll
             for (int i = 0; i < KP; ++i) {
-                uint32_t wv[2];
-#pragma unroll
-                for (int ww = 0; ww < 2; ++ww) {
-                    const int64_t col0 = (int64_t)kb * kBK + ww * 32;
-                    wv[ww] = (tile_ok && col0 < K)
-                        ? planes[block_index(i, sl, tile, S, Nt) * 256 + (((w0 + ww) ^ (lane >> 2)) * 32) + lane]
-                        : 0u;
-                }
-                uint32_t hp[32];
-                const int64_t hbase = (int64_t)i * (K / 2) + (int64_t)kb * 32;
-#pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const int64_t idx = hbase + 4 * v;
-                    uint4 u = make_uint4(0, 0, 0, 0);
-                    if ((int64_t)kb * 32 + 4 * v < K / 2) u = *reinterpret_cast<const uint4*>(hperm + idx);
-                    hp[4 * v] = u.x; hp[4 * v + 1] = u.y; hp[4 * v + 2] = u.z; hp[4 * v + 3] = u.w;
-                }
                 uint32_t a[32];
 #pragma unroll
                 for (int ww = 0; ww < 2; ++ww)
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        a[ww * 16 + j] = lop3_sign(wv[ww] << (15 - j), hp[ww * 16 + j]);
+                        a[ww * 16 + j] = lop3_sign(cw[i][ww] << (15 - j), ch[i][ww * 16 + j]);
                 tc_st_32x32b_x32(tmem + lane_base + (uint32_t)(KP * BT + (sa * KP + i) * 32), a);
             }
             tc_wait_st();

@@ -2,7 +2,7 @@
 // (RaBiT, "Residual binarization": matmul-free inference with additions and
 // element-wise scaling; the k paths run side by side).
 //
-// M = 1, k <= 4: byte-table kernel.  For each 256-column slice the CTA builds,
+// M = 1, k <= 4: byte-table kernel.  For each 256-column slice a CTA builds,
 // per plane, T_i[byte][group] = sum_{q<8} (bit q of byte ? +1 : -1) * hx_i[8*group + q]
 // with hx_i = h_i .* x formed exactly in fp32 (a bf16 x fp16 product has at
 // most 19 significant bits).  One table lookup then stands for eight signed
@@ -11,10 +11,12 @@
 // lanes read 32 different groups: group (4*slot + b) ^ l lives in smem bank
 // ((4*slot + b) ^ l) and the lookups are conflict-free.  One PRMT forms the
 // byte offset (byte << 8 | group << 2), one LDS fetches the entry, one FADD
-// accumulates: three instructions per eight weights.  Row sums across the
-// slices go through a small fp32 workspace; the last warp to finish a row tile
-// (per-tile arrival counter) adds the slice partials in slice order, so the
-// result is deterministic.
+// accumulates: three instructions per eight weights.  The CTAs that share a
+// row chunk form a thread-block cluster, one CTA per group of slices; their
+// per-row sums meet over distributed shared memory after one cluster barrier
+// and are added in rank order, so the result is deterministic and no global
+// workspace is needed.  Weights and g are fetched before the
+// programmatic-dependent-launch wait; X and h are read after it.
 //
 // Any M <= 64, any k <= 8: generic CUDA-core kernel (lane = row, one signed
 // fused add per bit and token); it keeps every plane and token block in
@@ -26,17 +28,13 @@ namespace {
 
 constexpr int kLutThreads = 256;
 constexpr int kLutWarps = kLutThreads / 32;
+constexpr int kLutPF = 2;              // row tiles per warp held in registers ahead of use
 
-// smem bytes of the byte tables: planes (2p, 2p+1) share a 64 KB region with
-// entry (byte, group) of plane i at region(i/2) + byte*256 + (i%2)*128 + group*4.
-__host__ __device__ constexpr int lut_smem_bytes(int kp) { return ((kp + 1) / 2) * 65536; }
-
-// Prefetch depth of the byte-table kernel: row tiles per warp held in registers.
-constexpr int kLutPF = 2;
+__host__ __device__ constexpr int lut_table_bytes(int kp) { return ((kp + 1) / 2) * 65536; }
 
 template <int KP>
 __device__ __forceinline__ void lut_load_tile(uint32_t (&wd)[KP][8], const uint32_t* __restrict__ planes,
-                                              int s, int64_t t, int64_t S, int64_t Nt, int lane)
+                                              int64_t s, int64_t t, int64_t S, int64_t Nt, int lane)
 {
 #pragma unroll
     for (int i = 0; i < KP; ++i) {
@@ -47,91 +45,117 @@ __device__ __forceinline__ void lut_load_tile(uint32_t (&wd)[KP][8], const uint3
 }
 
 template <int KP>
+__device__ __forceinline__ void lut_load_g(float (&gv)[KP], const uint16_t* __restrict__ g16, int64_t r, int N)
+{
+#pragma unroll
+    for (int i = 0; i < KP; ++i)
+        gv[i] = r < N ? __half2float(__ushort_as_half(g16[(int64_t)i * N + r])) : 0.0f;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_saddr, uint32_t rank) {
+    uint32_t remote;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+// Byte tables of slice s for all KP planes (256 threads: thread (group gg,
+// part) writes bytes 32*part .. 32*part+31 of group gg).  Plane i's entry
+// (byte, group) sits at region(i/2) + byte*256 + (i%2)*128 + group*4.
+template <int KP>
+__device__ __forceinline__ void lut_build(float* lut, const uint16_t* __restrict__ h16,
+                                          const uint16_t* __restrict__ X, int64_t s, int K)
+{
+    const int gg = threadIdx.x & 31, part = threadIdx.x >> 5;
+    const int64_t c0 = s * 256 + gg * 8;
+    const bool col_ok = c0 < K;                   // K % 32 == 0: a group is all in or all out
+    float xv[8];
+    const uint4 xr = col_ok ? *reinterpret_cast<const uint4*>(X + c0) : make_uint4(0, 0, 0, 0);
+    const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        xv[2 * q] = bf16_bits_to_f32(xw[q] & 0xffffu);
+        xv[2 * q + 1] = bf16_bits_to_f32(xw[q] >> 16);
+    }
+#pragma unroll
+    for (int i = 0; i < KP; ++i) {
+        const uint4 hr = col_ok ? *reinterpret_cast<const uint4*>(h16 + (int64_t)i * K + c0) : make_uint4(0, 0, 0, 0);
+        const uint32_t hw[4] = {hr.x, hr.y, hr.z, hr.w};
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            v[2 * q] = __half2float(__ushort_as_half((unsigned short)(hw[q] & 0xffffu))) * xv[2 * q];
+            v[2 * q + 1] = __half2float(__ushort_as_half((unsigned short)(hw[q] >> 16))) * xv[2 * q + 1];
+        }
+        float L[16];                              // signed sums of columns 0..3 of the group
+        L[0] = -((v[0] + v[1]) + (v[2] + v[3]));
+#pragma unroll
+        for (int n = 1; n < 16; ++n) {
+            const int low = n & -n;
+            const int q = low == 1 ? 0 : low == 2 ? 1 : low == 4 ? 2 : 3;
+            L[n] = L[n & (n - 1)] + 2.0f * v[q];
+        }
+        float Hh[2];                              // signed sums of columns 4..7 for this part's high nibbles
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int n = 2 * part + e;
+            float acc = 0.0f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc += ((n >> q) & 1) ? v[4 + q] : -v[4 + q];
+            Hh[e] = acc;
+        }
+        char* base = reinterpret_cast<char*>(lut) + (i >> 1) * 65536 + (i & 1) * 128 + gg * 4;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int b = 32 * part + j;
+            *reinterpret_cast<float*>(base + b * 256) = L[b & 15] + Hh[(b >> 4) & 1];
+        }
+    }
+}
+
+// Grid: R clusters of CS CTAs.  Cluster c owns row tiles [Nt*c/R, Nt*(c+1)/R);
+// its CTA of rank j handles slices j, j+CS, j+2CS, ... < S.  Per-row slice sums
+// stay in shared memory; after one cluster barrier every CTA adds, for its
+// share of the rows, the CS partial sums read over distributed shared memory
+// (rank order) and writes Y.  With CS = 1 the CTA owns every slice.
+template <int KP>
 __global__ void __launch_bounds__(kLutThreads, 2)
 gemv_lut_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ g16,
                 const uint16_t* __restrict__ h16, const uint16_t* __restrict__ X,
-                int N, int K, int C, float* __restrict__ partial,
-                unsigned* __restrict__ counters, void* __restrict__ Y, int ydt)
+                int N, int K, int CS, int R, void* __restrict__ Y, int ydt)
 {
     extern __shared__ __align__(1024) float lut[];
-    __shared__ int s_last;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t S = num_slices(K), Nt = num_row_tiles(N);
-    const int s = blockIdx.x / C, cta = blockIdx.x % C;
-    const int64_t t_begin = Nt * cta / C, t_end = Nt * (cta + 1) / C;
+    const int rank = CS > 1 ? (int)cluster_rank() : 0;
+    const int chunk = blockIdx.x / CS;
+    const int64_t t_begin = Nt * chunk / R, t_end = Nt * (chunk + 1) / R;
+    const int64_t chunk_rows = (t_end - t_begin) * 32;
+    float* red = lut + lut_table_bytes(KP) / 4;   // per-row sums of this CTA's slices
 
-    // ---- before the dependency wait: everything that does not depend on X.
-    // Weights of this warp's first kLutPF row tiles, their g values, this
-    // thread's h values for the table build.
+    // ---- before the dependency wait: the weights of the first slice's first
+    // tiles and their g values (neither depends on the previous kernel).
     uint32_t wd[kLutPF][KP][8];
     float gv[kLutPF][KP];
+    const int64_t s_first = rank;
 #pragma unroll
     for (int p = 0; p < kLutPF; ++p) {
         const int64_t t = t_begin + warp + (int64_t)p * kLutWarps;
-        if (t < t_end) {
-            lut_load_tile<KP>(wd[p], planes, s, t, S, Nt, lane);
-            const int64_t r = t * 32 + lane;
-#pragma unroll
-            for (int i = 0; i < KP; ++i)
-                gv[p][i] = r < N ? __half2float(__ushort_as_half(g16[(int64_t)i * N + r])) : 0.0f;
+        if (t < t_end && s_first < S) {
+            lut_load_tile<KP>(wd[p], planes, s_first, t, S, Nt, lane);
+            lut_load_g<KP>(gv[p], g16, t * 32 + lane, N);
         }
     }
-    const int gg = threadIdx.x & 31, part = threadIdx.x >> 5;
-    const int64_t c0 = (int64_t)s * 256 + gg * 8;
-    const bool col_ok = c0 < K;
-    uint4 hr[KP];
-#pragma unroll
-    for (int i = 0; i < KP; ++i)
-        hr[i] = col_ok ? *reinterpret_cast<const uint4*>(h16 + (int64_t)i * K + c0) : make_uint4(0, 0, 0, 0);
-
-    pdl_launch_dependents();
-    pdl_wait();
-
-    // ---- byte tables of slice s: thread (group gg, part) writes bytes 32*part .. +31
-    {
-        float xv[8];
-        const uint4 xr = col_ok ? *reinterpret_cast<const uint4*>(X + c0) : make_uint4(0, 0, 0, 0);
-        const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            xv[2 * q] = bf16_bits_to_f32(xw[q] & 0xffffu);
-            xv[2 * q + 1] = bf16_bits_to_f32(xw[q] >> 16);
-        }
-#pragma unroll
-        for (int i = 0; i < KP; ++i) {
-            float v[8];
-            const uint32_t hw[4] = {hr[i].x, hr[i].y, hr[i].z, hr[i].w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                v[2 * q] = __half2float(__ushort_as_half((unsigned short)(hw[q] & 0xffffu))) * xv[2 * q];
-                v[2 * q + 1] = __half2float(__ushort_as_half((unsigned short)(hw[q] >> 16))) * xv[2 * q + 1];
-            }
-            float L[16];                       // signed sums of columns 0..3 of the group
-            L[0] = -((v[0] + v[1]) + (v[2] + v[3]));
-#pragma unroll
-            for (int n = 1; n < 16; ++n) {
-                const int low = n & -n;
-                const int q = low == 1 ? 0 : low == 2 ? 1 : low == 4 ? 2 : 3;
-                L[n] = L[n & (n - 1)] + 2.0f * v[q];
-            }
-            float Hh[2];                       // signed sums of columns 4..7 for this part's high nibbles
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int n = 2 * part + e;
-                float acc = 0.0f;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) acc += ((n >> q) & 1) ? v[4 + q] : -v[4 + q];
-                Hh[e] = acc;
-            }
-            char* base = reinterpret_cast<char*>(lut) + (i >> 1) * 65536 + (i & 1) * 128 + gg * 4;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int b = 32 * part + j;
-                *reinterpret_cast<float*>(base + b * 256) = L[b & 15] + Hh[(b >> 4) & 1];
-            }
-        }
-    }
-    __syncthreads();
+    for (int64_t x = threadIdx.x; x < chunk_rows; x += kLutThreads) red[x] = 0.0f;
 
     // Per-lane lookup constants: G[sl] byte b' = group offset ((4 sl + b') ^ lane) * 4;
     // SEL[b'] = PRMT selector giving (word byte (b' ^ lane%4)) << 8 | G byte b', zeros above.
@@ -148,71 +172,79 @@ gemv_lut_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict_
         SEL[b] = (uint32_t)(4 + b) | ((uint32_t)(b ^ (lane & 3)) << 4) |
                  ((uint32_t)(12 + b) << 8) | ((uint32_t)(12 + b) << 12);
     const char* tb = reinterpret_cast<const char*>(lut);
-    const int64_t Ntp = Nt * 32;
 
-    for (int64_t t0 = t_begin + warp; t0 < t_end; t0 += (int64_t)kLutPF * kLutWarps) {
+    pdl_launch_dependents();
+    pdl_wait();
+
+    for (int64_t s = s_first; s < S; s += CS) {
+        if (s != s_first) {
+            __syncthreads();                      // the previous slice's lookups are done with the tables
 #pragma unroll
-        for (int p = 0; p < kLutPF; ++p) {
-            const int64_t t = t0 + (int64_t)p * kLutWarps;
-            if (t >= t_end) break;
-            float acc[KP];
-#pragma unroll
-            for (int i = 0; i < KP; ++i) {
-                float a0 = 0.0f, a1 = 0.0f;
-                const char* tp = tb + (i >> 1) * 65536 + (i & 1) * 128;
-#pragma unroll
-                for (int sl = 0; sl < 8; ++sl) {
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        const uint32_t off = prmt(wd[p][i][sl], G[sl], SEL[b]);
-                        const float e = *reinterpret_cast<const float*>(tp + off);
-                        if (b & 1) a1 += e; else a0 += e;
-                    }
+            for (int p = 0; p < kLutPF; ++p) {
+                const int64_t t = t_begin + warp + (int64_t)p * kLutWarps;
+                if (t < t_end) {
+                    lut_load_tile<KP>(wd[p], planes, s, t, S, Nt, lane);
+                    lut_load_g<KP>(gv[p], g16, t * 32 + lane, N);
                 }
-                acc[i] = a0 + a1;
             }
-            float pr = 0.0f;
+        }
+        lut_build<KP>(lut, h16, X, s, K);
+        __syncthreads();
+
+        for (int64_t t0 = t_begin + warp; t0 < t_end; t0 += (int64_t)kLutPF * kLutWarps) {
 #pragma unroll
-            for (int i = 0; i < KP; ++i) pr += gv[p][i] * acc[i];
-            const int64_t r = t * 32 + lane;
-            if (S == 1) {
-                if (r < N) store_y(Y, ydt, r, pr);
-            } else {
-                partial[(int64_t)s * Ntp + r] = pr;
-            }
-            // refill this slot with the tile kLutPF rounds ahead
-            const int64_t tn = t + (int64_t)kLutPF * kLutWarps;
-            if (tn < t_end) {
-                lut_load_tile<KP>(wd[p], planes, s, tn, S, Nt, lane);
-                const int64_t rn = tn * 32 + lane;
+            for (int p = 0; p < kLutPF; ++p) {
+                const int64_t t = t0 + (int64_t)p * kLutWarps;
+                if (t >= t_end) break;
+                float pr = 0.0f;
 #pragma unroll
-                for (int i = 0; i < KP; ++i)
-                    gv[p][i] = rn < N ? __half2float(__ushort_as_half(g16[(int64_t)i * N + rn])) : 0.0f;
+                for (int i = 0; i < KP; ++i) {
+                    float a0 = 0.0f, a1 = 0.0f;
+                    const char* tp = tb + (i >> 1) * 65536 + (i & 1) * 128;
+#pragma unroll
+                    for (int sl = 0; sl < 8; ++sl) {
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            const uint32_t off = prmt(wd[p][i][sl], G[sl], SEL[b]);
+                            const float e = *reinterpret_cast<const float*>(tp + off);
+                            if (b & 1) a1 += e; else a0 += e;
+                        }
+                    }
+                    pr += gv[p][i] * (a0 + a1);
+                }
+                red[(t - t_begin) * 32 + lane] += pr;
+                const int64_t tn = t + (int64_t)kLutPF * kLutWarps;   // refill this slot
+                if (tn < t_end) {
+                    lut_load_tile<KP>(wd[p], planes, s, tn, S, Nt, lane);
+                    lut_load_g<KP>(gv[p], g16, tn * 32 + lane, N);
+                }
             }
         }
     }
-    if (S == 1) return;
 
-    // ---- cross-slice sum: the last of the S CTAs that own row tiles [t_begin, t_end)
-    // adds the slice partials in slice order.
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(counters + cta, 1u) == (unsigned)(S - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int64_t r = t_begin * 32 + threadIdx.x; r < t_end * 32; r += kLutThreads) {
-        float y = 0.0f;
-        for (int64_t sb = 0; sb < S; sb += 16) {        // 16 independent L2 loads in flight
-            float v[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = (sb + j < S) ? __ldcg(partial + (sb + j) * Ntp + r) : 0.0f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) y += v[j];
+    // ---- cross-slice sum (every CTA of the cluster reaches both barriers)
+    if (CS == 1) {
+        __syncthreads();
+        for (int64_t x = threadIdx.x; x < chunk_rows; x += kLutThreads) {
+            const int64_t r = t_begin * 32 + x;
+            if (r < N) store_y(Y, ydt, r, red[x]);
         }
+        return;
+    }
+    cluster_sync_all();
+    const int64_t x0 = chunk_rows * rank / CS, x1 = chunk_rows * (rank + 1) / CS;
+    const uint32_t red_s = smem_u32(red);
+    for (int64_t x = x0 + threadIdx.x; x < x1; x += kLutThreads) {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = j < CS ? ld_dsmem_f32(red_s + (uint32_t)x * 4u, (uint32_t)j) : 0.0f;
+        float y = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) y += v[j];
+        const int64_t r = t_begin * 32 + x;
         if (r < N) store_y(Y, ydt, r, y);
     }
-    if (threadIdx.x == 0) counters[cta] = 0u;
+    cluster_sync_all();                           // peers keep their shared memory until every read is done
 }
 
 // ---------------------------------------------------------------- generic kernel
@@ -282,60 +314,89 @@ gemv_generic_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restr
     }
 }
 
-// CTAs per slice for the byte-table kernel: minimise the per-SM load
-// ceil(S*C / SMs) * (table build + ceil(Nt/C) row tiles); one table build costs
-// about as many shared-memory wavefronts as 6.4 row tiles.
-int lut_ctas_per_slice(int64_t S, int64_t Nt, int sms, int kp)
-{
-    const int occ = kp <= 2 ? 3 : 1;
-    int best = 1;
-    double best_cost = 1e30;
-    for (int C = 1; C <= Nt && C <= 4 * sms; ++C) {
-        const int64_t ctas = S * C;
-        if (ctas > (int64_t)sms * occ) break;
-        const double per_sm = (double)((ctas + sms - 1) / sms);
-        const double cost = per_sm * (6.4 + (double)((Nt + C - 1) / C));
-        if (cost < best_cost - 1e-9) { best_cost = cost; best = C; }
-    }
-    return best;
-}
-
-struct GemvWs {
-    unsigned* counters;
-    float* partial;
-    size_t bytes;
+// ---------------------------------------------------------------- host side
+struct LutPlan {
+    int CS;          // CTAs per cluster (slice groups)
+    int R;           // clusters (row chunks)
+    int smem;        // dynamic shared memory bytes
 };
 
-GemvWs gemv_ws_layout(int N, int K, void* base)
+cudaLaunchConfig_t lut_config(const LutPlan& p, cudaLaunchAttribute* attr, bool pdl, cudaStream_t stream)
 {
-    const int64_t S = num_slices(K), Nt = num_row_tiles(N);
-    const size_t cnt_bytes = ((size_t)Nt * 4 + 255) / 256 * 256;
-    const size_t part_bytes = (size_t)S * Nt * 32 * 4;
-    GemvWs w;
-    w.counters = reinterpret_cast<unsigned*>(base);
-    w.partial = reinterpret_cast<float*>(reinterpret_cast<char*>(base) + cnt_bytes);
-    w.bytes = S > 1 ? cnt_bytes + part_bytes : 0;
-    return w;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.CS * p.R));
+    cfg.blockDim = dim3(kLutThreads);
+    cfg.dynamicSmemBytes = (size_t)p.smem;
+    cfg.stream = stream;
+    int na = 0;
+    if (p.CS > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)p.CS;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cfg;
 }
 
+// Slices per CTA = ceil(S/16), CS = ceil(S / that) CTAs per cluster; as many
+// clusters (row chunks) as fit one CTA per SM, capped by how many clusters of
+// that size the GPU keeps resident at once and by the number of row tiles.
 template <int KP>
-rb_status launch_lut(const rb_layer_t* L, const uint16_t* X, void* Y, int ydt,
-                     const GemvWs& ws, bool pdl, cudaStream_t stream)
+rb_status lut_plan(int N, int K, LutPlan* plan)
 {
+    const int64_t S = num_slices(K), Nt = num_row_tiles(N);
+    const int spc = (int)((S + 15) / 16);
+    const int CS = (int)((S + spc - 1) / spc);
+    const int sms = num_sms();
+    int R = CS > 1 ? sms / CS : sms;
+    if (R < 1) R = 1;
+    if (R > Nt) R = (int)Nt;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    const int smem = lut_smem_bytes(KP);
-    if (dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(gemv_lut_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (dev < 0 || dev >= 64) return RB_ERR_UNSUPPORTED;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(gemv_lut_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+            return RB_ERR_CUDA;
+        if (cudaFuncSetAttribute(gemv_lut_kernel<KP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
             return RB_ERR_CUDA;
         attr_set[dev] = true;
     }
-    const int64_t S = num_slices(L->k_in), Nt = num_row_tiles(L->n_out);
-    const int C = lut_ctas_per_slice(S, Nt, num_sms(), KP);
-    return launch(gemv_lut_kernel<KP>, dim3((unsigned)(S * C)), dim3(kLutThreads), (size_t)smem,
-                  stream, pdl, L->planes, L->g16, L->h16, X, L->n_out, L->k_in, C,
-                  ws.partial, ws.counters, Y, ydt);
+    LutPlan p{CS, R, lut_table_bytes(KP) + (int)(((Nt + R - 1) / R) * 32 * 4)};
+    if (CS > 1) {
+        cudaLaunchAttribute attr[2];
+        cudaLaunchConfig_t cfg = lut_config(p, attr, false, 0);
+        int active = 0;
+        if (cudaOccupancyMaxActiveClusters(&active, gemv_lut_kernel<KP>, &cfg) == cudaSuccess && active > 0 &&
+            active < R) {
+            p.R = active;
+            p.smem = lut_table_bytes(KP) + (int)(((Nt + p.R - 1) / p.R) * 32 * 4);
+        }
+    }
+    if (p.smem > 227 * 1024) return RB_ERR_UNSUPPORTED;
+    *plan = p;
+    return RB_OK;
+}
+
+template <int KP>
+rb_status launch_lut(const rb_layer_t* L, const uint16_t* X, void* Y, int ydt, bool pdl, cudaStream_t stream)
+{
+    LutPlan plan;
+    rb_status st = lut_plan<KP>(L->n_out, L->k_in, &plan);
+    if (st != RB_OK) return st;
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = lut_config(plan, attr, pdl, stream);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel<KP>, L->planes, L->g16, L->h16, X,
+                                             (int)L->n_out, (int)L->k_in, plan.CS, plan.R, Y, ydt);
+    return e == cudaSuccess ? RB_OK : RB_ERR_CUDA;
 }
 
 template <int KP>
@@ -357,11 +418,8 @@ using namespace rbw;
 
 extern "C" size_t rb_gemv_workspace_bytes(int n_out, int k_in, int k_planes, int M)
 {
-    if (n_out < 1 || k_in < 32 || k_in % 32 != 0 || k_planes < 1 || k_planes > 8 || M < 1 || M > 64)
-        return 0;
-    rb_layer_t L = {n_out, k_in, k_planes, 0, nullptr, nullptr, nullptr};
-    if (!use_lut(&L, M)) return 0;
-    return gemv_ws_layout(n_out, k_in, nullptr).bytes;
+    (void)n_out; (void)k_in; (void)k_planes; (void)M;
+    return 0;          // every rb_gemv path keeps its partial sums on chip
 }
 
 extern "C" rb_status rb_gemv(const rb_layer_t* layer, const uint16_t* X, int M, void* Y,
@@ -369,6 +427,8 @@ extern "C" rb_status rb_gemv(const rb_layer_t* layer, const uint16_t* X, int M, 
                              int32_t* dev_status, unsigned flags, cudaStream_t stream)
 {
     (void)dev_status;
+    (void)workspace;
+    (void)workspace_bytes;
     rb_status st = check_apply_args(layer, X, M, Y, y_dtype, flags);
     if (st != RB_OK) return st;
     if (M > 64) return RB_ERR_SHAPE;
@@ -376,14 +436,11 @@ extern "C" rb_status rb_gemv(const rb_layer_t* layer, const uint16_t* X, int M, 
     const bool pdl = (flags & RB_LAUNCH_PDL) != 0;
     const int ydt = (int)y_dtype;
     if (use_lut(layer, M)) {
-        GemvWs ws = gemv_ws_layout(layer->n_out, layer->k_in, workspace);
-        if (ws.bytes && (!workspace || workspace_bytes < ws.bytes)) return RB_ERR_WORKSPACE;
-        if (workspace && !aligned16(workspace)) return RB_ERR_ALIGN;
         switch (layer->k_planes) {
-            case 1: return launch_lut<1>(layer, X, Y, ydt, ws, pdl, stream);
-            case 2: return launch_lut<2>(layer, X, Y, ydt, ws, pdl, stream);
-            case 3: return launch_lut<3>(layer, X, Y, ydt, ws, pdl, stream);
-            default: return launch_lut<4>(layer, X, Y, ydt, ws, pdl, stream);
+            case 1: return launch_lut<1>(layer, X, Y, ydt, pdl, stream);
+            case 2: return launch_lut<2>(layer, X, Y, ydt, pdl, stream);
+            case 3: return launch_lut<3>(layer, X, Y, ydt, pdl, stream);
+            default: return launch_lut<4>(layer, X, Y, ydt, pdl, stream);
         }
     }
     switch (layer->k_planes) {
