@@ -60,20 +60,26 @@ pack_kernel(const float* __restrict__ W, const float* __restrict__ g,
                 const int64_t r = t * 32 + j;
                 wv[j] = r < N ? __ldcs(W + r * K + c) : 0.0f;
             }
+            float nonfinite = 0.0f;               // stays 0 unless some W is NaN or +-inf
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const bool row_ok = (t * 32 + j) < N;
                 float R = wv[j];
-                bad |= !(fabsf(R) <= FLT_MAX);
+                nonfinite = fmaf(R, 0.0f, nonfinite);
+                const bool mine_row = lane == j;
 #pragma unroll
                 for (int i = 0; i < KP; ++i) {
                     const float gi = __shfl_sync(0xffffffffu, gv[i], j);
-                    const bool b = R >= 0.0f;               // sign(0) = +1, -0.0 too
                     const float tt = __fmul_rn(gi, hv[i]);
-                    R = b ? __fsub_rn(R, tt) : __fadd_rn(R, tt);
+                    const bool b = R >= 0.0f;               // sign(0) = +1, -0.0 too
+                    R = __fadd_rn(R, b ? -tt : tt);         // R - t or R + t, one rounding
                     const uint32_t word = __ballot_sync(0xffffffffu, b);
-                    if (lane == j) mine[i] = row_ok ? word : 0u;
+                    if (mine_row) mine[i] = word;
                 }
+            }
+            bad |= nonfinite != 0.0f;
+            if (t * 32 + lane >= N) {
+#pragma unroll
+                for (int i = 0; i < KP; ++i) mine[i] = 0u;   // padding rows of the last tile
             }
         }
 #pragma unroll

@@ -55,9 +55,9 @@ def test_size_helpers_reject_bad_shapes(L):
     assert L.rb_packed_words(4, 48, 1) == 0
     assert L.rb_packed_words(0, 64, 1) == 0
     assert L.rb_packed_words(4, 64, 9) == 0
-    assert L.rb_gemv_workspace_bytes(4096, 4096, 2, 65) == 0
-    assert L.rb_gemv_workspace_bytes(4096, 4096, 2, 1) > 0
-    assert L.rb_gemv_workspace_bytes(64, 256, 2, 1) == 0     # one slice: no cross-slice sums
+    assert L.rb_gemv_workspace_bytes(4096, 4096, 2, 1) == 0   # partial sums stay on chip
+    assert L.rb_gemm_workspace_bytes(4096, 4096, 2, 64) >= 64 * 4096 * 2
+    assert L.rb_gemm_workspace_bytes(4096, 4096, 5, 64) == 0  # the tensor-core path serves k <= 4
     assert L.rb_svid_workspace_bytes(4096, 4096) > 0
 
 

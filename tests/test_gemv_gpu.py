@@ -51,7 +51,6 @@ def test_gemv_workloads(wl, li, k, M, ydt):
     Yr = oracle.apply(planes, g16, h16, N, K, k, X, rows=rows)
     Yg = Yg if rows is None else Yg[:, rows]
     cases.check_y(Yg, Yr, cases.abs_bound(g16, h16, X, rows), bf16=ydt == torch.bfloat16)
-    assert not ws[:4 * ((N + 31) // 32)].any(), "arrival counters not reset"
 
 
 @pytest.mark.parametrize("N,K,k,M", [(33, 288, 2, 1), (100, 800, 3, 1), (1, 32, 1, 1), (1000, 544, 4, 1),
@@ -80,7 +79,6 @@ def test_gemv_deterministic_pdl_and_reused_workspace():
     outs = [run_gemv(L, X, 1, torch.float32, flags=f, ws=ws)[0] for f in (0, rbw.RB_LAUNCH_PDL, 0, rbw.RB_LAUNCH_PDL)]
     for o in outs[1:]:
         assert np.array_equal(o, outs[0])
-    assert not ws[:4 * ((N + 31) // 32)].any()
 
 
 def test_gemv_end_to_end_from_gpu_pack():
@@ -100,11 +98,11 @@ def test_gemv_errors_on_device():
     N, K = W.shape
     planes, g16, h16 = cases.packed_case(1, 0, 2)
     L = cases.upload_layer(planes, g16, h16, N, K, 2)
-    X = cases.to_dev(synth.activations(1, K, seed=1))
-    small = rbw.workspace(64)
+    X = cases.to_dev(synth.activations(65, K, seed=1))
     with pytest.raises(rbw.RbError) as e:
-        rbw.gemv(L, X, ws=small)
-    assert e.value.status == rbw.RB_ERR_WORKSPACE
+        rbw.gemv(L, X)                                  # M > 64
+    assert e.value.status == rbw.RB_ERR_SHAPE
+    Xbad = torch.zeros(2 * K + 8, dtype=torch.int16, device="cuda")[1:1 + K].view(1, K)   # 2-byte offset
     with pytest.raises(rbw.RbError) as e:
-        rbw.gemv(L, X, ws=None)
-    assert e.value.status == rbw.RB_ERR_WORKSPACE
+        rbw.gemv(L, Xbad)
+    assert e.value.status == rbw.RB_ERR_ALIGN
