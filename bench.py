@@ -3,11 +3,14 @@
 
 Workload: the Llama-7B q_proj shape, N = K = 4096 with k = 2 residual sign
 planes (W ~ N(0, 0.02) with 0.1% x20 outliers, greedy-SVID scales), decode
-M = 1.  One step = 32 decode tokens, one after another, each through a stack
-of 96 distinct packed layers of that shape (rb_gemv per layer, launched with
-programmatic dependent launch, captured in a CUDA graph).  The 96 layers hold
-~403 MB of sign planes, more than the 126 MB L2, so every step streams the
-planes from HBM.  Metric: packed-weight bytes read per second (GB/s).
+M = 1.  One step = 32 decode tokens, one after another; each token applies 96
+distinct, independent packed layers of that shape to its activation vector
+with rb_gemv_batch (two launches of up to 64 layers, programmatic dependent
+launch between them, captured in a CUDA graph).  The 96 layers hold ~403 MB of
+sign planes, more than the 126 MB L2, so every step streams the planes from
+HBM.  Metric: packed-weight bytes read per second (GB/s).  The same 3072
+applications issued as single-layer rb_gemv calls in one dependent chain are
+reported beside it (decode_chain).
 
 Legs (one JSON line on rank 0):
   value       device-timed (CUDA events) throughput, inputs resident in HBM;
@@ -277,38 +280,37 @@ def run_rbw(args, dist: Dist):
     lib = rbw.lib()
     import ctypes
 
-    NS = 4                                 # independent layers go round-robin over NS streams
-    streams = [torch.cuda.Stream(dev) for _ in range(NS)]
-    wss = [rbw.workspace(rbw.gemv_workspace_bytes(N_OUT, K_IN, K_PLANES, 1), dev) for _ in range(NS)]
-    ytmp = [torch.empty(1, N_OUT, dtype=torch.float32, device=dev) for _ in range(NS)]
+    # batch of the 96 layers of a token: host arrays of device pointers, built once
+    nb = LAYERS
+    lp = (ctypes.POINTER(rbw.RbLayer) * nb)(*[ctypes.pointer(structs[j]) for j in range(nb)])
+    ytmp = torch.empty(LAYERS - 1, N_OUT, dtype=torch.float32, device=dev)
+    xps = [(ctypes.c_void_p * nb)(*([X.data_ptr() + t * K_IN * 2] * nb)) for t in range(TOKENS)]
+    yps = [(ctypes.c_void_p * nb)(*([ytmp.data_ptr() + j * N_OUT * 4 for j in range(LAYERS - 1)] +
+                                    [Y_last.data_ptr() + t * N_OUT * 4])) for t in range(TOKENS)]
+    streams = [torch.cuda.Stream(dev)]
 
-    def launch(li, t, stream, wsi):
-        yp = (Y_last.data_ptr() + t * N_OUT * 4) if li == LAYERS - 1 else ytmp[wsi].data_ptr()
-        st = lib.rb_gemv(ctypes.byref(structs[li]), ctypes.c_void_p(X.data_ptr() + t * K_IN * 2), 1,
-                         ctypes.c_void_p(yp), rbw.RB_F32, ctypes.c_void_p(wss[wsi].data_ptr()),
-                         wss[wsi].numel(), None, rbw.RB_LAUNCH_PDL, ctypes.c_void_p(stream.cuda_stream))
-        if st != 0:
-            raise rbw.RbError("rb_gemv", st)
-
-    def step_streams():
-        """32 tokens x 96 independent layers; layer l on stream l % NS (fork/join on streams[0])."""
-        ev = torch.cuda.Event()
-        ev.record(streams[0])
-        for sx in streams[1:]:
-            sx.wait_event(ev)
+    def step_batched():
+        """32 tokens, one after another; per token one rb_gemv_batch over the 96 layers."""
+        sp = ctypes.c_void_p(streams[0].cuda_stream)
         for t in range(TOKENS):
-            for li in range(LAYERS):
-                launch(li, t, streams[li % NS], li % NS)
-        for sx in streams[1:]:
-            e = torch.cuda.Event()
-            e.record(sx)
-            streams[0].wait_event(e)
+            st = lib.rb_gemv_batch(ctypes.cast(lp, ctypes.c_void_p), ctypes.cast(xps[t], ctypes.c_void_p),
+                                   ctypes.cast(yps[t], ctypes.c_void_p), nb, 1, rbw.RB_F32, None,
+                                   rbw.RB_LAUNCH_PDL, sp)
+            if st != 0:
+                raise rbw.RbError("rb_gemv_batch", st)
 
     def step_chain():
-        """The same 3072 applications as one dependent chain on one stream (PDL)."""
+        """The same 3072 applications as single-layer rb_gemv calls, one dependent chain (PDL)."""
+        sp = ctypes.c_void_p(streams[0].cuda_stream)
         for t in range(TOKENS):
+            xp = ctypes.c_void_p(X.data_ptr() + t * K_IN * 2)
             for li in range(LAYERS):
-                launch(li, t, streams[0], 0)
+                yp = ctypes.c_void_p((Y_last.data_ptr() + t * N_OUT * 4) if li == LAYERS - 1
+                                     else ytmp.data_ptr() + li * N_OUT * 4)
+                st = lib.rb_gemv(ctypes.byref(structs[li]), xp, 1, yp, rbw.RB_F32, None, 0, None,
+                                 rbw.RB_LAUNCH_PDL, sp)
+                if st != 0:
+                    raise rbw.RbError("rb_gemv", st)
 
     def capture(fn, pre=None, post=None):
         with torch.cuda.stream(streams[0]):
@@ -341,12 +343,13 @@ def run_rbw(args, dist: Dist):
         dist.barrier()
         return e0.elapsed_time(e1) / 1e3
 
-    launches_per_step = TOKENS * LAYERS
+    launches_per_step = TOKENS * LAYERS          # layer applications per step
+    kernel_launches_per_step = TOKENS * ((LAYERS + 63) // 64)
     plane_bytes = layers[0].packed_bytes()
     bytes_per_step = plane_bytes * launches_per_step
     algo_bytes_per_launch = plane_bytes + 2 * K_PLANES * (N_OUT + K_IN) + 2 * K_IN + 4 * N_OUT
 
-    graph = capture(step_streams)
+    graph = capture(step_batched)
     sampler = ClockSampler(gpu_uuid(torch))
     sampler.start()
     time.sleep(0.05)
@@ -354,7 +357,7 @@ def run_rbw(args, dist: Dist):
     clocks = sampler.stop()
     t_max = dist.max(t_local, dev)
     value = throughput(bytes_per_step, dist.world, args.steps, t_max)
-    avg_launch_s = t_local / (args.steps * launches_per_step)
+    avg_launch_s = t_local / (args.steps * launches_per_step)      # per layer application
     achieved = algo_bytes_per_launch / avg_launch_s / 1e9
     del graph
 
@@ -363,13 +366,13 @@ def run_rbw(args, dist: Dist):
     t_chain = dist.max(time_graph(chain_graph, chain_steps), dev)
     chain = {"GBps": throughput(bytes_per_step, dist.world, chain_steps, t_chain),
              "us_per_layer": t_chain / (chain_steps * launches_per_step) * 1e6,
-             "what": "one stream, each rb_gemv launched with PDL after the previous one (dependent decode chain)"}
+             "what": "single-layer rb_gemv calls on one stream, each launched with PDL after the previous one (dependent decode chain)"}
     del chain_graph
 
     # ---- e2e: host X in pinned memory -> device, the step, Y of the last layer -> host
     X_pin = torch.from_numpy(X_host.view(np.int16).copy()).pin_memory()
     Y_pin = torch.empty(TOKENS, N_OUT, dtype=torch.float32).pin_memory()
-    graph_e2e = capture(step_streams, pre=lambda: X.copy_(X_pin, non_blocking=True),
+    graph_e2e = capture(step_batched, pre=lambda: X.copy_(X_pin, non_blocking=True),
                         post=lambda: Y_pin.copy_(Y_last, non_blocking=True))
     e2e_steps = max(1, min(args.steps, 200))
     t_e2e = dist.max(time_graph(graph_e2e, e2e_steps, sync_each=True), dev)
@@ -392,10 +395,12 @@ def run_rbw(args, dist: Dist):
                    "pct_of_peak": {"measured_hbm": value / dist.world / hbm_peak, "spec_8tbs": value / dist.world / 8000.0},
                    "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                                 "frac": achieved / hbm_peak, "traffic": profiled_traffic("gemv_lut_kernel<2>"),
-                                "kernel": "gemv_lut_kernel<2>", "peak_source": peak_src,
-                                "algorithmic_bytes_per_launch": algo_bytes_per_launch,
-                                "avg_launch_us": avg_launch_s * 1e6},
-                   "cpu_baseline": cb, "e2e": e2e, "gpu_launches": args.steps * launches_per_step,
+                                "kernel": "gemv_lut_kernel<2> via rb_gemv_batch", "peak_source": peak_src,
+                                "algorithmic_bytes_per_layer": algo_bytes_per_launch,
+                                "layers_per_launch": LAYERS / ((LAYERS + 63) // 64),
+                                "avg_us_per_layer": avg_launch_s * 1e6,
+                                "avg_launch_us": avg_launch_s * 1e6 * LAYERS / ((LAYERS + 63) // 64)},
+                   "cpu_baseline": cb, "e2e": e2e, "gpu_launches": args.steps * kernel_launches_per_step,
                    "decode_chain": chain,
                    "clocks": clocks, "rows": rows})
         print(json.dumps(line), flush=True)

@@ -135,6 +135,20 @@ RB_API rb_status rb_gemv(const rb_layer_t *layer, const uint16_t *X, int M,
                   int32_t *dev_status, unsigned flags, cudaStream_t stream);
 
 /*
+ * rb_gemv_batch -- rb_gemv applied to `count` independent layers of one shape
+ * (same N, K, k) in as few launches as possible, e.g. the q/k/v or gate/up
+ * projections of one decode step, or the layers of several models served at
+ * once.  layers[j], X[j], Y[j] (host arrays of device pointers) describe
+ * application j; Y[j] must not alias any other input or output of the call.
+ * For M = 1 one launch serves up to 64 layers and spreads each CTA's table
+ * build over more rows, so small layers stream at close to HBM bandwidth.
+ * Needs no workspace.
+ */
+RB_API rb_status rb_gemv_batch(const rb_layer_t *const *layers, const uint16_t *const *X, void *const *Y,
+                               int count, int M, rb_dtype y_dtype, int32_t *dev_status, unsigned flags,
+                               cudaStream_t stream);
+
+/*
  * rb_gemm -- batched (prefill) Y = X . What^T for any M >= 1 (tuned for
  * M >= 64) on the tcgen05 tensor cores: sign tiles are expanded to +-h_i
  * (fp16, exact) and multiplied with X converted to fp16 (exact in the normal

@@ -13,10 +13,10 @@
 // byte offset (byte << 8 | group << 2), one LDS fetches the entry, one FADD
 // accumulates: three instructions per eight weights.  The CTAs that share a
 // row chunk form a thread-block cluster, one CTA per group of slices; their
-// per-row sums meet over distributed shared memory after one cluster barrier
-// and are added in rank order, so the result is deterministic and no global
-// workspace is needed.  Weights and g are fetched before the
-// programmatic-dependent-launch wait; X and h are read after it.
+// per-row sums are pushed over distributed shared memory to the CTA that owns
+// the row, and after one cluster barrier added in rank order, so the result is
+// deterministic and no global workspace is needed.  Weights, g and h are
+// fetched before the programmatic-dependent-launch wait; only X after it.
 //
 // Any M <= 64, any k <= 8: generic CUDA-core kernel (lane = row, one signed
 // fused add per bit and token); it keeps every plane and token block in
@@ -44,12 +44,12 @@ __device__ __forceinline__ void lut_load_tile(uint32_t (&wd)[KP][8], const uint3
     }
 }
 
+// g as raw fp16 bits: converting here would stall on the load before the wait.
 template <int KP>
-__device__ __forceinline__ void lut_load_g(float (&gv)[KP], const uint16_t* __restrict__ g16, int64_t r, int N)
+__device__ __forceinline__ void lut_load_g(uint16_t (&gv)[KP], const uint16_t* __restrict__ g16, int64_t r, int N)
 {
 #pragma unroll
-    for (int i = 0; i < KP; ++i)
-        gv[i] = r < N ? __half2float(__ushort_as_half(g16[(int64_t)i * N + r])) : 0.0f;
+    for (int i = 0; i < KP; ++i) gv[i] = r < N ? g16[(int64_t)i * N + r] : (uint16_t)0;
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -60,20 +60,27 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_saddr, uint32_t rank) {
+__device__ __forceinline__ void st_dsmem_f32(uint32_t local_saddr, uint32_t rank, float v) {
     uint32_t remote;
-    float v;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(rank));
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-    return v;
+    asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(remote), "f"(v) : "memory");
 }
 
 // Byte tables of slice s for all KP planes (256 threads: thread (group gg,
 // part) writes bytes 32*part .. 32*part+31 of group gg).  Plane i's entry
 // (byte, group) sits at region(i/2) + byte*256 + (i%2)*128 + group*4.
 template <int KP>
-__device__ __forceinline__ void lut_build(float* lut, const uint16_t* __restrict__ h16,
-                                          const uint16_t* __restrict__ X, int64_t s, int K)
+__device__ __forceinline__ void lut_load_h(uint4 (&hr)[KP], const uint16_t* __restrict__ h16, int64_t s, int K)
+{
+    const int64_t c0 = s * 256 + (threadIdx.x & 31) * 8;
+#pragma unroll
+    for (int i = 0; i < KP; ++i)
+        hr[i] = c0 < K ? *reinterpret_cast<const uint4*>(h16 + (int64_t)i * K + c0) : make_uint4(0, 0, 0, 0);
+}
+
+template <int KP>
+__device__ __forceinline__ void lut_build(float* lut, const uint4 (&hrr)[KP], const uint16_t* __restrict__ X,
+                                          int64_t s, int K)
 {
     const int gg = threadIdx.x & 31, part = threadIdx.x >> 5;
     const int64_t c0 = s * 256 + gg * 8;
@@ -88,8 +95,7 @@ __device__ __forceinline__ void lut_build(float* lut, const uint16_t* __restrict
     }
 #pragma unroll
     for (int i = 0; i < KP; ++i) {
-        const uint4 hr = col_ok ? *reinterpret_cast<const uint4*>(h16 + (int64_t)i * K + c0) : make_uint4(0, 0, 0, 0);
-        const uint32_t hw[4] = {hr.x, hr.y, hr.z, hr.w};
+        const uint32_t hw[4] = {hrr[i].x, hrr[i].y, hrr[i].z, hrr[i].w};
         float v[8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -124,28 +130,44 @@ __device__ __forceinline__ void lut_build(float* lut, const uint16_t* __restrict
 
 // Grid: R clusters of CS CTAs.  Cluster c owns row tiles [Nt*c/R, Nt*(c+1)/R);
 // its CTA of rank j handles slices j, j+CS, j+2CS, ... < S.  Per-row slice sums
-// stay in shared memory; after one cluster barrier every CTA adds, for its
-// share of the rows, the CS partial sums read over distributed shared memory
-// (rank order) and writes Y.  With CS = 1 the CTA owns every slice.
+// stay in shared memory until each is stored into the receive area of the CTA
+// that sums that row; after one cluster barrier that CTA adds the CS partial
+// sums in rank order and writes Y.  With CS = 1 the CTA owns every slice.
+constexpr int kMaxBatch = 64;          // layers per launch of the byte-table kernel
+
+// Independent layers of one shape handled by one launch (pointers per layer).
+struct LutBatch {
+    const uint32_t* planes[kMaxBatch];
+    const uint16_t* g16[kMaxBatch];
+    const uint16_t* h16[kMaxBatch];
+    const uint16_t* X[kMaxBatch];
+    void* Y[kMaxBatch];
+};
+
 template <int KP>
 __global__ void __launch_bounds__(kLutThreads, 2)
-gemv_lut_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ g16,
-                const uint16_t* __restrict__ h16, const uint16_t* __restrict__ X,
-                int N, int K, int CS, int R, void* __restrict__ Y, int ydt)
+gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, int R, int ydt)
 {
     extern __shared__ __align__(1024) float lut[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t S = num_slices(K), Nt = num_row_tiles(N);
     const int rank = CS > 1 ? (int)cluster_rank() : 0;
-    const int chunk = blockIdx.x / CS;
+    const int layer = blockIdx.x / (CS * R);
+    const uint32_t* __restrict__ planes = batch.planes[layer];
+    const uint16_t* __restrict__ g16 = batch.g16[layer];
+    const uint16_t* __restrict__ h16 = batch.h16[layer];
+    const uint16_t* __restrict__ X = batch.X[layer];
+    void* __restrict__ Y = batch.Y[layer];
+    const int chunk = (blockIdx.x / CS) % R;
     const int64_t t_begin = Nt * chunk / R, t_end = Nt * (chunk + 1) / R;
     const int64_t chunk_rows = (t_end - t_begin) * 32;
     float* red = lut + lut_table_bytes(KP) / 4;   // per-row sums of this CTA's slices
 
-    // ---- before the dependency wait: the weights of the first slice's first
-    // tiles and their g values (neither depends on the previous kernel).
+    // ---- before the dependency wait: everything that does not depend on X --
+    // the weights of the first slice's first tiles, their g values, h.
     uint32_t wd[kLutPF][KP][8];
-    float gv[kLutPF][KP];
+    uint16_t gv[kLutPF][KP];
+    uint4 hr[KP];
     const int64_t s_first = rank;
 #pragma unroll
     for (int p = 0; p < kLutPF; ++p) {
@@ -155,6 +177,7 @@ gemv_lut_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict_
             lut_load_g<KP>(gv[p], g16, t * 32 + lane, N);
         }
     }
+    if (s_first < S) lut_load_h<KP>(hr, h16, s_first, K);
     for (int64_t x = threadIdx.x; x < chunk_rows; x += kLutThreads) red[x] = 0.0f;
 
     // Per-lane lookup constants: G[sl] byte b' = group offset ((4 sl + b') ^ lane) * 4;
@@ -179,6 +202,7 @@ gemv_lut_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict_
     for (int64_t s = s_first; s < S; s += CS) {
         if (s != s_first) {
             __syncthreads();                      // the previous slice's lookups are done with the tables
+            lut_load_h<KP>(hr, h16, s, K);
 #pragma unroll
             for (int p = 0; p < kLutPF; ++p) {
                 const int64_t t = t_begin + warp + (int64_t)p * kLutWarps;
@@ -188,41 +212,50 @@ gemv_lut_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict_
                 }
             }
         }
-        lut_build<KP>(lut, h16, X, s, K);
+        lut_build<KP>(lut, hr, X, s, K);
         __syncthreads();
 
         for (int64_t t0 = t_begin + warp; t0 < t_end; t0 += (int64_t)kLutPF * kLutWarps) {
+            // the kLutPF prefetched tiles, looked up side by side (independent chains)
+            float acc[kLutPF][KP][2];
+#pragma unroll
+            for (int p = 0; p < kLutPF; ++p)
+#pragma unroll
+                for (int i = 0; i < KP; ++i) acc[p][i][0] = acc[p][i][1] = 0.0f;
+#pragma unroll
+            for (int sl = 0; sl < 8; ++sl) {
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+#pragma unroll
+                    for (int p = 0; p < kLutPF; ++p) {
+#pragma unroll
+                        for (int i = 0; i < KP; ++i) {
+                            const uint32_t off = prmt(wd[p][i][sl], G[sl], SEL[b]);
+                            acc[p][i][b & 1] += *reinterpret_cast<const float*>(tb + (i >> 1) * 65536 + (i & 1) * 128 + off);
+                        }
+                    }
+                }
+            }
 #pragma unroll
             for (int p = 0; p < kLutPF; ++p) {
                 const int64_t t = t0 + (int64_t)p * kLutWarps;
-                if (t >= t_end) break;
-                float pr = 0.0f;
+                if (t < t_end) {
+                    float pr = 0.0f;
 #pragma unroll
-                for (int i = 0; i < KP; ++i) {
-                    float a0 = 0.0f, a1 = 0.0f;
-                    const char* tp = tb + (i >> 1) * 65536 + (i & 1) * 128;
-#pragma unroll
-                    for (int sl = 0; sl < 8; ++sl) {
-#pragma unroll
-                        for (int b = 0; b < 4; ++b) {
-                            const uint32_t off = prmt(wd[p][i][sl], G[sl], SEL[b]);
-                            const float e = *reinterpret_cast<const float*>(tp + off);
-                            if (b & 1) a1 += e; else a0 += e;
-                        }
+                    for (int i = 0; i < KP; ++i)
+                        pr += __half2float(__ushort_as_half(gv[p][i])) * (acc[p][i][0] + acc[p][i][1]);
+                    red[(t - t_begin) * 32 + lane] += pr;
+                    const int64_t tn = t + (int64_t)kLutPF * kLutWarps;   // refill this slot
+                    if (tn < t_end) {
+                        lut_load_tile<KP>(wd[p], planes, s, tn, S, Nt, lane);
+                        lut_load_g<KP>(gv[p], g16, tn * 32 + lane, N);
                     }
-                    pr += gv[p][i] * (a0 + a1);
-                }
-                red[(t - t_begin) * 32 + lane] += pr;
-                const int64_t tn = t + (int64_t)kLutPF * kLutWarps;   // refill this slot
-                if (tn < t_end) {
-                    lut_load_tile<KP>(wd[p], planes, s, tn, S, Nt, lane);
-                    lut_load_g<KP>(gv[p], g16, tn * 32 + lane, N);
                 }
             }
         }
     }
 
-    // ---- cross-slice sum (every CTA of the cluster reaches both barriers)
+    // ---- cross-slice sum
     if (CS == 1) {
         __syncthreads();
         for (int64_t x = threadIdx.x; x < chunk_rows; x += kLutThreads) {
@@ -231,20 +264,28 @@ gemv_lut_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict_
         }
         return;
     }
+    // Rows [x0(j), x1(j)) of the chunk are summed by rank j.  Every CTA stores its
+    // partial of such a row into rank j's receive area, slot (own rank, row);
+    // one cluster barrier (release / acquire) later each CTA adds its rows'
+    // CS partials from local shared memory, in rank order.
+    float* recv = red + chunk_rows;
+    const uint32_t recv_s = smem_u32(recv);
+    __syncthreads();                              // red[] complete within the CTA
+    for (int64_t x = threadIdx.x; x < chunk_rows; x += kLutThreads) {
+        // owner = max{j : floor(chunk_rows*j/CS) <= x}
+        const int owner = (int)(((x + 1) * CS - 1) / chunk_rows);
+        const int64_t xo = x - chunk_rows * owner / CS;
+        const int64_t span = chunk_rows * (owner + 1) / CS - chunk_rows * owner / CS;
+        st_dsmem_f32(recv_s + (uint32_t)((rank * span + xo) * 4), (uint32_t)owner, red[x]);
+    }
     cluster_sync_all();
     const int64_t x0 = chunk_rows * rank / CS, x1 = chunk_rows * (rank + 1) / CS;
-    const uint32_t red_s = smem_u32(red);
-    for (int64_t x = x0 + threadIdx.x; x < x1; x += kLutThreads) {
-        float v[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = j < CS ? ld_dsmem_f32(red_s + (uint32_t)x * 4u, (uint32_t)j) : 0.0f;
+    for (int64_t xo = threadIdx.x; xo < x1 - x0; xo += kLutThreads) {
         float y = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) y += v[j];
-        const int64_t r = t_begin * 32 + x;
+        for (int j = 0; j < CS; ++j) y += recv[j * (x1 - x0) + xo];
+        const int64_t r = t_begin * 32 + x0 + xo;
         if (r < N) store_y(Y, ydt, r, y);
     }
-    cluster_sync_all();                           // peers keep their shared memory until every read is done
 }
 
 // ---------------------------------------------------------------- generic kernel
@@ -321,10 +362,10 @@ struct LutPlan {
     int smem;        // dynamic shared memory bytes
 };
 
-cudaLaunchConfig_t lut_config(const LutPlan& p, cudaLaunchAttribute* attr, bool pdl, cudaStream_t stream)
+cudaLaunchConfig_t lut_config(const LutPlan& p, int count, cudaLaunchAttribute* attr, bool pdl, cudaStream_t stream)
 {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.CS * p.R));
+    cfg.gridDim = dim3((unsigned)(count * p.CS * p.R));
     cfg.blockDim = dim3(kLutThreads);
     cfg.dynamicSmemBytes = (size_t)p.smem;
     cfg.stream = stream;
@@ -346,17 +387,28 @@ cudaLaunchConfig_t lut_config(const LutPlan& p, cudaLaunchAttribute* attr, bool 
     return cfg;
 }
 
-// Slices per CTA = ceil(S/16), CS = ceil(S / that) CTAs per cluster; as many
-// clusters (row chunks) as fit one CTA per SM, capped by how many clusters of
-// that size the GPU keeps resident at once and by the number of row tiles.
+// Per-row sums (red) plus, with a cluster, the receive area of the rows this CTA
+// sums: CS slots of at most ceil(rows/CS) rows, which never exceeds rows + CS.
+int lut_row_bytes(int64_t Nt, int R, int CS)
+{
+    const int64_t rows = ((Nt + R - 1) / R) * 32;
+    return (int)((CS > 1 ? 2 * rows + CS : rows) * 4);
+}
+
+// Slices per CTA = ceil(S/16), CS = ceil(S / that) CTAs per cluster.  Row
+// chunks per layer (R): a single layer takes as many as fill the SMs (lowest
+// latency); a batch of `count` layers takes as few as keep about two CTAs per
+// SM busy, so each CTA's table build is spread over more rows.  R is capped by
+// the clusters the GPU keeps resident, the row tiles and shared memory.
 template <int KP>
-rb_status lut_plan(int N, int K, LutPlan* plan)
+rb_status lut_plan(int N, int K, int count, LutPlan* plan)
 {
     const int64_t S = num_slices(K), Nt = num_row_tiles(N);
     const int spc = (int)((S + 15) / 16);
     const int CS = (int)((S + spc - 1) / spc);
     const int sms = num_sms();
     int R = CS > 1 ? sms / CS : sms;
+    if (count > 1) R = (int)((2 * sms + (int64_t)count * CS - 1) / ((int64_t)count * CS));
     if (R < 1) R = 1;
     if (R > Nt) R = (int)Nt;
     static bool attr_set[64] = {};
@@ -370,15 +422,17 @@ rb_status lut_plan(int N, int K, LutPlan* plan)
             return RB_ERR_CUDA;
         attr_set[dev] = true;
     }
-    LutPlan p{CS, R, lut_table_bytes(KP) + (int)(((Nt + R - 1) / R) * 32 * 4)};
-    if (CS > 1) {
+    // shared memory: at most ~105 KB per CTA so that two CTAs fit on an SM
+    while (R < Nt && lut_table_bytes(KP) + lut_row_bytes(Nt, R, CS) > 105 * 1024) ++R;
+    LutPlan p{CS, R, lut_table_bytes(KP) + lut_row_bytes(Nt, R, CS)};
+    if (CS > 1 && count == 1) {
         cudaLaunchAttribute attr[2];
-        cudaLaunchConfig_t cfg = lut_config(p, attr, false, 0);
+        cudaLaunchConfig_t cfg = lut_config(p, 1, attr, false, 0);
         int active = 0;
         if (cudaOccupancyMaxActiveClusters(&active, gemv_lut_kernel<KP>, &cfg) == cudaSuccess && active > 0 &&
             active < R) {
             p.R = active;
-            p.smem = lut_table_bytes(KP) + (int)(((Nt + p.R - 1) / p.R) * 32 * 4);
+            p.smem = lut_table_bytes(KP) + lut_row_bytes(Nt, p.R, CS);
         }
     }
     if (p.smem > 227 * 1024) return RB_ERR_UNSUPPORTED;
@@ -387,16 +441,30 @@ rb_status lut_plan(int N, int K, LutPlan* plan)
 }
 
 template <int KP>
-rb_status launch_lut(const rb_layer_t* L, const uint16_t* X, void* Y, int ydt, bool pdl, cudaStream_t stream)
+rb_status launch_lut(const rb_layer_t* const* layers, const uint16_t* const* X, void* const* Y, int count,
+                     int ydt, bool pdl, cudaStream_t stream)
 {
-    LutPlan plan;
-    rb_status st = lut_plan<KP>(L->n_out, L->k_in, &plan);
-    if (st != RB_OK) return st;
-    cudaLaunchAttribute attr[2];
-    cudaLaunchConfig_t cfg = lut_config(plan, attr, pdl, stream);
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel<KP>, L->planes, L->g16, L->h16, X,
-                                             (int)L->n_out, (int)L->k_in, plan.CS, plan.R, Y, ydt);
-    return e == cudaSuccess ? RB_OK : RB_ERR_CUDA;
+    const rb_layer_t* L0 = layers[0];
+    for (int base = 0; base < count; base += kMaxBatch) {
+        const int n = count - base < kMaxBatch ? count - base : kMaxBatch;
+        LutPlan plan;
+        rb_status st = lut_plan<KP>(L0->n_out, L0->k_in, n, &plan);
+        if (st != RB_OK) return st;
+        LutBatch b = {};
+        for (int j = 0; j < n; ++j) {
+            b.planes[j] = layers[base + j]->planes;
+            b.g16[j] = layers[base + j]->g16;
+            b.h16[j] = layers[base + j]->h16;
+            b.X[j] = X[base + j];
+            b.Y[j] = Y[base + j];
+        }
+        cudaLaunchAttribute attr[2];
+        cudaLaunchConfig_t cfg = lut_config(plan, n, attr, pdl, stream);
+        if (cudaLaunchKernelEx(&cfg, gemv_lut_kernel<KP>, b, (int)L0->n_out, (int)L0->k_in, plan.CS, plan.R, ydt) !=
+            cudaSuccess)
+            return RB_ERR_CUDA;
+    }
+    return RB_OK;
 }
 
 template <int KP>
@@ -422,6 +490,45 @@ extern "C" size_t rb_gemv_workspace_bytes(int n_out, int k_in, int k_planes, int
     return 0;          // every rb_gemv path keeps its partial sums on chip
 }
 
+static rb_status gemv_dispatch(const rb_layer_t* const* layers, const uint16_t* const* X, void* const* Y,
+                               int count, int M, rb_dtype y_dtype, unsigned flags, cudaStream_t stream)
+{
+    const rb_layer_t* L0 = layers[0];
+    for (int j = 0; j < count; ++j) {
+        rb_status st = check_apply_args(layers[j], X[j], M, Y[j], y_dtype, flags);
+        if (st != RB_OK) return st;
+        if (layers[j]->n_out != L0->n_out || layers[j]->k_in != L0->k_in || layers[j]->k_planes != L0->k_planes)
+            return RB_ERR_SHAPE;
+    }
+    if (M > 64) return RB_ERR_SHAPE;
+    if (!device_is_sm100()) return RB_ERR_UNSUPPORTED;
+    const bool pdl = (flags & RB_LAUNCH_PDL) != 0;
+    const int ydt = (int)y_dtype;
+    if (use_lut(L0, M)) {
+        switch (L0->k_planes) {
+            case 1: return launch_lut<1>(layers, X, Y, count, ydt, pdl, stream);
+            case 2: return launch_lut<2>(layers, X, Y, count, ydt, pdl, stream);
+            case 3: return launch_lut<3>(layers, X, Y, count, ydt, pdl, stream);
+            default: return launch_lut<4>(layers, X, Y, count, ydt, pdl, stream);
+        }
+    }
+    for (int j = 0; j < count; ++j) {
+        rb_status st;
+        switch (L0->k_planes) {
+            case 1: st = launch_generic<1>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
+            case 2: st = launch_generic<2>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
+            case 3: st = launch_generic<3>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
+            case 4: st = launch_generic<4>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
+            case 5: st = launch_generic<5>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
+            case 6: st = launch_generic<6>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
+            case 7: st = launch_generic<7>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
+            default: st = launch_generic<8>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
+        }
+        if (st != RB_OK) return st;
+    }
+    return RB_OK;
+}
+
 extern "C" rb_status rb_gemv(const rb_layer_t* layer, const uint16_t* X, int M, void* Y,
                              rb_dtype y_dtype, void* workspace, size_t workspace_bytes,
                              int32_t* dev_status, unsigned flags, cudaStream_t stream)
@@ -429,28 +536,17 @@ extern "C" rb_status rb_gemv(const rb_layer_t* layer, const uint16_t* X, int M, 
     (void)dev_status;
     (void)workspace;
     (void)workspace_bytes;
-    rb_status st = check_apply_args(layer, X, M, Y, y_dtype, flags);
-    if (st != RB_OK) return st;
-    if (M > 64) return RB_ERR_SHAPE;
-    if (!device_is_sm100()) return RB_ERR_UNSUPPORTED;
-    const bool pdl = (flags & RB_LAUNCH_PDL) != 0;
-    const int ydt = (int)y_dtype;
-    if (use_lut(layer, M)) {
-        switch (layer->k_planes) {
-            case 1: return launch_lut<1>(layer, X, Y, ydt, pdl, stream);
-            case 2: return launch_lut<2>(layer, X, Y, ydt, pdl, stream);
-            case 3: return launch_lut<3>(layer, X, Y, ydt, pdl, stream);
-            default: return launch_lut<4>(layer, X, Y, ydt, pdl, stream);
-        }
-    }
-    switch (layer->k_planes) {
-        case 1: return launch_generic<1>(layer, X, M, Y, ydt, pdl, stream);
-        case 2: return launch_generic<2>(layer, X, M, Y, ydt, pdl, stream);
-        case 3: return launch_generic<3>(layer, X, M, Y, ydt, pdl, stream);
-        case 4: return launch_generic<4>(layer, X, M, Y, ydt, pdl, stream);
-        case 5: return launch_generic<5>(layer, X, M, Y, ydt, pdl, stream);
-        case 6: return launch_generic<6>(layer, X, M, Y, ydt, pdl, stream);
-        case 7: return launch_generic<7>(layer, X, M, Y, ydt, pdl, stream);
-        default: return launch_generic<8>(layer, X, M, Y, ydt, pdl, stream);
-    }
+    if (!layer) return RB_ERR_ARG;
+    return gemv_dispatch(&layer, &X, &Y, 1, M, y_dtype, flags, stream);
+}
+
+extern "C" rb_status rb_gemv_batch(const rb_layer_t* const* layers, const uint16_t* const* X, void* const* Y,
+                                   int count, int M, rb_dtype y_dtype, int32_t* dev_status, unsigned flags,
+                                   cudaStream_t stream)
+{
+    (void)dev_status;
+    if (!layers || !X || !Y || count < 1) return RB_ERR_ARG;
+    for (int j = 0; j < count; ++j)
+        if (!layers[j]) return RB_ERR_ARG;
+    return gemv_dispatch(layers, X, Y, count, M, y_dtype, flags, stream);
 }

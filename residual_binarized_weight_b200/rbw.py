@@ -29,6 +29,7 @@ SIGNATURES = {
     "rb_pack": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "rb_gemv_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
     "rb_gemv": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _u32, _vp]),
+    "rb_gemv_batch": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _u32, _vp]),
     "rb_gemm_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
     "rb_gemm": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _u32, _vp]),
     "rb_svid_workspace_bytes": (_sz, [_i32, _i32]),
@@ -146,6 +147,21 @@ def gemv(layer: PackedLayer, X, Y=None, ws=None, flags=0, dev_status=None, strea
     if Y is None:
         Y = torch.empty(X.shape[0], layer.n_out, dtype=y_dtype, device=X.device)
     return _apply("rb_gemv", layer, X, Y, ws, flags, dev_status, stream)
+
+
+def gemv_batch(layers, Xs, Ys, flags=0, dev_status=None, stream=None):
+    """rb_gemv_batch: independent layers of one shape; Xs[j] bf16 [M][K], Ys[j] [M][N] (CUDA tensors)."""
+    n = len(layers)
+    structs = (RbLayer * n)(*[L.struct() for L in layers])
+    lp = (ctypes.POINTER(RbLayer) * n)(*[ctypes.pointer(structs[j]) for j in range(n)])
+    xp = (ctypes.c_void_p * n)(*[X.data_ptr() for X in Xs])
+    yp = (ctypes.c_void_p * n)(*[Y.data_ptr() for Y in Ys])
+    M = Xs[0].shape[0]
+    ydt = RB_BF16 if Ys[0].dtype == torch.bfloat16 else RB_F32
+    st = lib().rb_gemv_batch(ctypes.cast(lp, ctypes.c_void_p), ctypes.cast(xp, ctypes.c_void_p),
+                             ctypes.cast(yp, ctypes.c_void_p), n, M, ydt, _ptr(dev_status), flags, _stream(stream))
+    _check("rb_gemv_batch", st)
+    return Ys
 
 
 def gemm(layer: PackedLayer, X, Y=None, ws=None, flags=0, dev_status=None, stream=None, y_dtype=torch.float32):

@@ -106,3 +106,42 @@ def test_gemv_errors_on_device():
     with pytest.raises(rbw.RbError) as e:
         rbw.gemv(L, Xbad)
     assert e.value.status == rbw.RB_ERR_ALIGN
+
+
+@pytest.mark.parametrize("N,K,k,count", [(4096, 4096, 2, 5), (300, 800, 1, 3), (1000, 11008, 2, 2), (64, 256, 3, 70)])
+def test_gemv_batch_matches_single_and_oracle(N, K, k, count):
+    """rb_gemv_batch over independent layers gives each layer exactly what rb_gemv gives,
+    and both match the oracle."""
+    rng = np.random.default_rng(N + K + count)
+    layers, Xs, refs = [], [], []
+    for j in range(min(count, 4)):
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+        g, h = oracle.svid_greedy(W, k, iters=6)
+        planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+        layers.append(cases.upload_layer(planes, g16, h16, N, K, k))
+        X = synth.activations(1, K, seed=j + 7)
+        Xs.append(X)
+        refs.append((planes, g16, h16))
+    idx = [j % len(layers) for j in range(count)]              # more applications than distinct layers
+    Xd = [cases.to_dev(Xs[i]) for i in idx]
+    Ys = [torch.empty(1, N, dtype=torch.float32, device="cuda") for _ in idx]
+    rbw.gemv_batch([layers[i] for i in idx], Xd, Ys)
+    torch.cuda.synchronize()
+    for j, i in enumerate(idx):
+        single = rbw.gemv(layers[i], Xd[j])
+        torch.cuda.synchronize()
+        assert torch.equal(Ys[j], single), "batch and single-layer results differ for application %d" % j
+        if j < len(layers):
+            planes, g16, h16 = refs[i]
+            Yr = oracle.apply(planes, g16, h16, N, K, k, Xs[i])
+            cases.check_y(Ys[j].cpu().numpy().astype(np.float64), Yr, cases.abs_bound(g16, h16, Xs[i]), bf16=False)
+
+
+def test_gemv_batch_rejects_mixed_shapes():
+    a = rbw.PackedLayer(64, 256, 2)
+    b = rbw.PackedLayer(64, 512, 2)
+    X = [torch.zeros(1, 256, dtype=torch.int16, device="cuda"), torch.zeros(1, 512, dtype=torch.int16, device="cuda")]
+    Y = [torch.empty(1, 64, device="cuda") for _ in range(2)]
+    with pytest.raises(rbw.RbError) as e:
+        rbw.gemv_batch([a, b], X, Y)
+    assert e.value.status == rbw.RB_ERR_SHAPE
