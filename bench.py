@@ -477,7 +477,8 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="skip the extra per-row timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--mode", choices=["full", "gemv-kernel", "pack-kernel", "gemm-kernel"], default="full",
+    ap.add_argument("--mode", choices=["full", "gemv-kernel", "gemv-batch-kernel", "pack-kernel", "gemm-kernel"],
+                    default="full",
                     help="kernel-only modes run one kernel a few times (used for ncu captures)")
     ap.add_argument("--launches", type=int, default=20)
     ap.add_argument("--M", type=int, default=1)
@@ -520,6 +521,10 @@ def run_kernel_mode(args):
             ws = rbw.workspace(rbw.gemv_workspace_bytes(N_OUT, K_IN, K_PLANES, M), dev)
             for j in range(args.launches):
                 rbw.gemv(layers[j % nl], X, Y=Y, ws=ws)
+        elif args.mode == "gemv-batch-kernel":
+            Ys = [torch.empty(M, N_OUT, dtype=torch.float32, device=dev) for _ in range(nl)]
+            for j in range(args.launches):
+                rbw.gemv_batch(layers, [X] * nl, Ys)
         else:
             ws = rbw.workspace(rbw.gemm_workspace_bytes(N_OUT, K_IN, K_PLANES, M), dev)
             for j in range(args.launches):

@@ -29,6 +29,7 @@ namespace {
 constexpr int kLutThreads = 256;
 constexpr int kLutWarps = kLutThreads / 32;
 constexpr int kLutPF = 2;              // row tiles per warp held in registers ahead of use
+constexpr int kLutPD = 6;              // row tiles per warp prefetched into L2 ahead of use
 
 __host__ __device__ constexpr int lut_table_bytes(int kp) { return ((kp + 1) / 2) * 65536; }
 
@@ -41,6 +42,19 @@ __device__ __forceinline__ void lut_load_tile(uint32_t (&wd)[KP][8], const uint3
         const uint32_t* blk = planes + block_index(i, s, t, S, Nt) * 256 + lane;
 #pragma unroll
         for (int sl = 0; sl < 8; ++sl) wd[i][sl] = __ldcs(blk + sl * 32);
+    }
+}
+
+// L2 prefetch of one row tile's sign words (KP blocks of 1 KB = 8 lines each):
+// lane l < 8*KP touches line l%8 of plane l/8.  Keeps DRAM busy further ahead
+// than the register-held tiles can.
+template <int KP>
+__device__ __forceinline__ void lut_prefetch_tile(const uint32_t* __restrict__ planes, int64_t s, int64_t t,
+                                                  int64_t S, int64_t Nt, int lane)
+{
+    if (lane < 8 * KP) {
+        const uint32_t* p = planes + block_index(lane >> 3, s, t, S, Nt) * 256 + (lane & 7) * 32;
+        asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
     }
 }
 
@@ -177,7 +191,14 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
             lut_load_g<KP>(gv[p], g16, t * 32 + lane, N);
         }
     }
-    if (s_first < S) lut_load_h<KP>(hr, h16, s_first, K);
+    if (s_first < S) {
+        lut_load_h<KP>(hr, h16, s_first, K);
+#pragma unroll
+        for (int p = kLutPF; p < kLutPD; ++p) {
+            const int64_t t = t_begin + warp + (int64_t)p * kLutWarps;
+            if (t < t_end) lut_prefetch_tile<KP>(planes, s_first, t, S, Nt, lane);
+        }
+    }
     for (int64_t x = threadIdx.x; x < chunk_rows; x += kLutThreads) red[x] = 0.0f;
 
     // Per-lane lookup constants: G[sl] byte b' = group offset ((4 sl + b') ^ lane) * 4;
@@ -245,6 +266,8 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
                     for (int i = 0; i < KP; ++i)
                         pr += __half2float(__ushort_as_half(gv[p][i])) * (acc[p][i][0] + acc[p][i][1]);
                     red[(t - t_begin) * 32 + lane] += pr;
+                    const int64_t tp = t + (int64_t)kLutPD * kLutWarps;   // L2 prefetch further ahead
+                    if (tp < t_end) lut_prefetch_tile<KP>(planes, s, tp, S, Nt, lane);
                     const int64_t tn = t + (int64_t)kLutPF * kLutWarps;   // refill this slot
                     if (tn < t_end) {
                         lut_load_tile<KP>(wd[p], planes, s, tn, S, Nt, lane);
