@@ -66,6 +66,27 @@ __device__ __forceinline__ void lut_load_g(uint16_t (&gv)[KP], const uint16_t* _
     for (int i = 0; i < KP; ++i) gv[i] = r < N ? g16[(int64_t)i * N + r] : (uint16_t)0;
 }
 
+// Shared-window address of dynamic shared memory in a kernel without static
+// shared memory on sm_100 (the first 1 KB is reserved).  The byte tables start
+// there, so a lookup is one LDS with the PRMT result as register and the table
+// base folded into the immediate.  The kernel checks the base at entry and uses
+// a register add instead if it ever differs.
+constexpr uint32_t kDynSmemBase = 1024;
+
+template <uint32_t IMM>
+__device__ __forceinline__ float lds_imm(uint32_t off) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(off), "n"(IMM));
+    return v;
+}
+
+template <bool FAST, int I>
+__device__ __forceinline__ float lut_entry(uint32_t tbase, uint32_t off) {
+    constexpr uint32_t C = (uint32_t)((I >> 1) * 65536 + (I & 1) * 128);
+    if constexpr (FAST) return lds_imm<kDynSmemBase + C>(off);
+    else return lds_f32(tbase + C + off);
+}
+
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -138,6 +159,87 @@ __device__ __forceinline__ void lut_build(float* lut, const uint4 (&hrr)[KP], co
         for (int j = 0; j < 32; ++j) {
             const int b = 32 * part + j;
             *reinterpret_cast<float*>(base + b * 256) = L[b & 15] + Hh[(b >> 4) & 1];
+        }
+    }
+}
+
+// All lookups of the kLutPF register-held tiles: for each word slot, the PRMT
+// offsets of 4 bytes x kLutPF tiles x KP planes are formed first, then all the
+// LDS are issued, then the FADDs, so each warp keeps 4*kLutPF*KP independent
+// table reads in flight.
+template <int KP, bool FAST>
+__device__ __forceinline__ void lut_lookups(float (&acc)[kLutPF][KP][2], const uint32_t (&wd)[kLutPF][KP][8],
+                                            const uint32_t (&G)[8], const uint32_t (&SEL)[4], uint32_t tbase)
+{
+#pragma unroll
+    for (int sl = 0; sl < 8; ++sl) {
+        uint32_t off[4][kLutPF][KP];
+        float e[4][kLutPF][KP];
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+            for (int p = 0; p < kLutPF; ++p)
+#pragma unroll
+                for (int i = 0; i < KP; ++i) off[b][p][i] = prmt(wd[p][i][sl], G[sl], SEL[b]);
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+            for (int p = 0; p < kLutPF; ++p) {
+                e[b][p][0] = lut_entry<FAST, 0>(tbase, off[b][p][0]);
+                if constexpr (KP > 1) e[b][p][1] = lut_entry<FAST, 1>(tbase, off[b][p][1]);
+                if constexpr (KP > 2) e[b][p][2] = lut_entry<FAST, 2>(tbase, off[b][p][2]);
+                if constexpr (KP > 3) e[b][p][3] = lut_entry<FAST, 3>(tbase, off[b][p][3]);
+            }
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+            for (int p = 0; p < kLutPF; ++p)
+#pragma unroll
+                for (int i = 0; i < KP; ++i) acc[p][i][b & 1] += e[b][p][i];
+    }
+}
+
+template <int KP, bool FAST>
+__device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_t (&gv)[kLutPF][KP],
+                                          const uint32_t (&G)[8], const uint32_t (&SEL)[4], uint32_t tbase,
+                                          float* red, const uint32_t* __restrict__ planes,
+                                          const uint16_t* __restrict__ g16, int64_t s, int64_t S, int64_t Nt,
+                                          int N, int tb, int te, int warp, int lane)
+{
+    const uint32_t* pbase[KP];
+#pragma unroll
+    for (int i = 0; i < KP; ++i) pbase[i] = planes + block_index(i, s, 0, S, Nt) * 256 + lane;
+    // this lane's L2-prefetch line: plane lane/8, line lane%8 of a tile block
+    const uint32_t* pf_base = lane < 8 * KP
+        ? planes + block_index(lane >> 3, s, 0, S, Nt) * 256 + (lane & 7) * 32 : planes;
+    for (int t0 = tb + warp; t0 < te; t0 += kLutPF * kLutWarps) {
+        float acc[kLutPF][KP][2];
+#pragma unroll
+        for (int p = 0; p < kLutPF; ++p)
+#pragma unroll
+            for (int i = 0; i < KP; ++i) acc[p][i][0] = acc[p][i][1] = 0.0f;
+        lut_lookups<KP, FAST>(acc, wd, G, SEL, tbase);
+#pragma unroll
+        for (int p = 0; p < kLutPF; ++p) {
+            const int t = t0 + p * kLutWarps;
+            if (t < te) {
+                float pr = 0.0f;
+#pragma unroll
+                for (int i = 0; i < KP; ++i)
+                    pr += __half2float(__ushort_as_half(gv[p][i])) * (acc[p][i][0] + acc[p][i][1]);
+                red[(t - tb) * 32 + lane] += pr;
+                const int tp = t + kLutPD * kLutWarps;                  // L2 prefetch further ahead
+                if (tp < te && lane < 8 * KP)
+                    asm volatile("prefetch.global.L2 [%0];" :: "l"(pf_base + (size_t)tp * 256));
+                const int tn = t + kLutPF * kLutWarps;                  // refill this slot
+                if (tn < te) {
+#pragma unroll
+                    for (int i = 0; i < KP; ++i)
+#pragma unroll
+                        for (int sl = 0; sl < 8; ++sl) wd[p][i][sl] = __ldcs(pbase[i] + (size_t)tn * 256 + sl * 32);
+                    lut_load_g<KP>(gv[p], g16, (int64_t)tn * 32 + lane, N);
+                }
+            }
         }
     }
 }
@@ -215,8 +317,9 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
     for (int b = 0; b < 4; ++b)
         SEL[b] = (uint32_t)(4 + b) | ((uint32_t)(b ^ (lane & 3)) << 4) |
                  ((uint32_t)(12 + b) << 8) | ((uint32_t)(12 + b) << 12);
-    const char* tb = reinterpret_cast<const char*>(lut);
 
+    const uint32_t tbase = smem_u32(lut);
+    const bool fast_base = tbase == kDynSmemBase;
     pdl_launch_dependents();
     pdl_wait();
 
@@ -236,46 +339,10 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
         lut_build<KP>(lut, hr, X, s, K);
         __syncthreads();
 
-        for (int64_t t0 = t_begin + warp; t0 < t_end; t0 += (int64_t)kLutPF * kLutWarps) {
-            // the kLutPF prefetched tiles, looked up side by side (independent chains)
-            float acc[kLutPF][KP][2];
-#pragma unroll
-            for (int p = 0; p < kLutPF; ++p)
-#pragma unroll
-                for (int i = 0; i < KP; ++i) acc[p][i][0] = acc[p][i][1] = 0.0f;
-#pragma unroll
-            for (int sl = 0; sl < 8; ++sl) {
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-#pragma unroll
-                    for (int p = 0; p < kLutPF; ++p) {
-#pragma unroll
-                        for (int i = 0; i < KP; ++i) {
-                            const uint32_t off = prmt(wd[p][i][sl], G[sl], SEL[b]);
-                            acc[p][i][b & 1] += *reinterpret_cast<const float*>(tb + (i >> 1) * 65536 + (i & 1) * 128 + off);
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int p = 0; p < kLutPF; ++p) {
-                const int64_t t = t0 + (int64_t)p * kLutWarps;
-                if (t < t_end) {
-                    float pr = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < KP; ++i)
-                        pr += __half2float(__ushort_as_half(gv[p][i])) * (acc[p][i][0] + acc[p][i][1]);
-                    red[(t - t_begin) * 32 + lane] += pr;
-                    const int64_t tp = t + (int64_t)kLutPD * kLutWarps;   // L2 prefetch further ahead
-                    if (tp < t_end) lut_prefetch_tile<KP>(planes, s, tp, S, Nt, lane);
-                    const int64_t tn = t + (int64_t)kLutPF * kLutWarps;   // refill this slot
-                    if (tn < t_end) {
-                        lut_load_tile<KP>(wd[p], planes, s, tn, S, Nt, lane);
-                        lut_load_g<KP>(gv[p], g16, tn * 32 + lane, N);
-                    }
-                }
-            }
-        }
+        if (fast_base)
+            lut_tiles<KP, true>(wd, gv, G, SEL, tbase, red, planes, g16, s, S, Nt, N, (int)t_begin, (int)t_end, warp, lane);
+        else
+            lut_tiles<KP, false>(wd, gv, G, SEL, tbase, red, planes, g16, s, S, Nt, N, (int)t_begin, (int)t_end, warp, lane);
     }
 
     // ---- cross-slice sum
