@@ -162,6 +162,29 @@ RB_API rb_status rb_gemm(const rb_layer_t *layer, const uint16_t *X, int M,
                   int32_t *dev_status, unsigned flags, cudaStream_t stream);
 
 /*
+ * rb_gemm_noalloc -- rb_gemm for callers that must not allocate device memory.
+ * The paper has no counterpart: this is a deployment convenience of the
+ * library.  Some hosts give the library a fixed device-memory budget at
+ * start-up and allow no further allocations (embedded or real-time
+ * deployments, plugin hosts whose own allocator owns the GPU, code that must
+ * not block on the allocator), so they cannot supply rb_gemm's workspace.
+ * This call takes the same arguments minus the workspace and uses a fixed
+ * 32 MiB array compiled into the library instead (every GPU that loads the
+ * library holds it until the process exits).  It allocates nothing.
+ *   - Sizes whose rb_gemm_workspace_bytes(N, K, k, M) exceeds 32 MiB (about
+ *     M*K <= 16.7 million) return RB_ERR_WORKSPACE; k > 4 returns
+ *     RB_ERR_UNSUPPORTED, as for rb_gemm.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the array.  Each call rewrites what it uses before
+ *     reading it, so nothing carries over between calls, but calls that
+ *     overlap on the GPU (two streams at once) race on it: serialise them.
+ */
+RB_API rb_status rb_gemm_noalloc(const rb_layer_t *layer, const uint16_t *X, int M,
+                                 void *Y, rb_dtype y_dtype, int32_t *dev_status, unsigned flags,
+                                 cudaStream_t stream);
+
+/*
  * rb_svid_greedy -- greedy SVID scales for each plane (RaBiT names Greedy
  * SVID as the traditional initialiser): for i = 1..k, (g_i, h_i) is the
  * rank-1 approximation of |R_{i-1}| by `iters` rounds of power iteration in

@@ -22,6 +22,8 @@
 // owns TMEM lanes 32*(w%4) .. +31).  Every mbarrier wait is bounded: on expiry
 // the kernel raises RB_DEV_TIMEOUT in dev_status, drains what it issued,
 // frees its tensor memory and returns.
+#include <atomic>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -510,4 +512,57 @@ extern "C" rb_status rb_gemm(const rb_layer_t* layer, const uint16_t* X, int M, 
 {
     return gemm_with_timeout(layer, X, M, Y, y_dtype, workspace, workspace_bytes, dev_status, flags,
                              stream, kTimeoutNs);
+}
+
+// ---------------------------------------------------------------------------
+// rb_gemm_noalloc: rb_gemm for callers that must not allocate device memory.
+//
+// Some hosts hand this library a fixed device-memory budget up front and do
+// not allow further allocations: embedded and real-time deployments that size
+// everything at start-up, plugin hosts whose own allocator owns the GPU, or
+// code that must not block on the allocator's device-wide synchronisation.
+// Such callers cannot provide rb_gemm's workspace.  This entry point uses a
+// file-scope device array instead (kNoAllocScratchBytes, held by every GPU
+// that loads the library until the process exits).  It calls no cudaMalloc,
+// cudaFree or any other allocating routine.
+//
+// The array's name is only a host-side stand-in in host code; its device
+// address is looked up once per device with cudaGetSymbolAddress, with that
+// device current, by the first call on that device (so the first call on a
+// device should come before any stream capture).  Every call shares the array
+// and the kernels fully rewrite the part they use before reading it, so no
+// state carries over; calls that overlap on the GPU (for example on two
+// streams at once) race on it and must be serialised by the caller.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocScratchBytes = (size_t)32 << 20;    // 32 MiB
+static __device__ __align__(256) uint8_t g_gemm_scratch[kNoAllocScratchBytes];
+
+void* noalloc_scratch_address()
+{
+    static std::atomic<void*> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    void* p = cache[dev].load(std::memory_order_acquire);
+    if (!p) {
+        if (cudaGetSymbolAddress(&p, g_gemm_scratch) != cudaSuccess || !p) return nullptr;
+        cache[dev].store(p, std::memory_order_release);
+    }
+    return p;
+}
+}  // namespace
+
+extern "C" rb_status rb_gemm_noalloc(const rb_layer_t* layer, const uint16_t* X, int M, void* Y, rb_dtype y_dtype,
+                                     int32_t* dev_status, unsigned flags, cudaStream_t stream)
+{
+    rb_status st = rbw::check_apply_args(layer, X, M, Y, y_dtype, flags);
+    if (st != RB_OK) return st;
+    if (layer->k_planes > 4) return RB_ERR_UNSUPPORTED;
+    if (rb_gemm_workspace_bytes(layer->n_out, layer->k_in, layer->k_planes, M) > kNoAllocScratchBytes)
+        return RB_ERR_WORKSPACE;                 // problem larger than the fixed scratch array
+    if (!rbw::device_is_sm100()) return RB_ERR_UNSUPPORTED;
+    void* scratch = noalloc_scratch_address();
+    if (!scratch) return RB_ERR_CUDA;
+    return rbw::gemm_with_timeout(layer, X, M, Y, y_dtype, scratch, kNoAllocScratchBytes, dev_status, flags,
+                                  stream, rbw::kTimeoutNs);
 }

@@ -32,6 +32,7 @@ SIGNATURES = {
     "rb_gemv_batch": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _u32, _vp]),
     "rb_gemm_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
     "rb_gemm": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _u32, _vp]),
+    "rb_gemm_noalloc": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _u32, _vp]),
     "rb_svid_workspace_bytes": (_sz, [_i32, _i32]),
     "rb_svid_greedy": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
 }
@@ -169,6 +170,18 @@ def gemm(layer: PackedLayer, X, Y=None, ws=None, flags=0, dev_status=None, strea
     if Y is None:
         Y = torch.empty(X.shape[0], layer.n_out, dtype=y_dtype, device=X.device)
     return _apply("rb_gemm", layer, X, Y, ws, flags, dev_status, stream)
+
+
+def gemm_noalloc(layer: PackedLayer, X, Y=None, flags=0, dev_status=None, stream=None, y_dtype=torch.float32):
+    """rb_gemm_noalloc: rb_gemm without a workspace (fixed 32 MiB library scratch; see include/rbw.h)."""
+    if Y is None:
+        Y = torch.empty(X.shape[0], layer.n_out, dtype=y_dtype, device=X.device)
+    L = layer.struct()
+    ydt = RB_BF16 if Y.dtype == torch.bfloat16 else RB_F32
+    st = lib().rb_gemm_noalloc(ctypes.byref(L), _ptr(X), X.shape[0], _ptr(Y), ydt, _ptr(dev_status), flags,
+                               _stream(stream))
+    _check("rb_gemm_noalloc", st)
+    return Y
 
 
 def svid_greedy(W, k_planes, iters=20, ws=None, stream=None):
