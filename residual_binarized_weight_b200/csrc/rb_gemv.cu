@@ -360,19 +360,23 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
     // CS partials from local shared memory, in rank order.
     float* recv = red + chunk_rows;
     const uint32_t recv_s = smem_u32(recv);
+    const int rows = (int)chunk_rows;             // <= 32 * Nt, fits 32 bits
     __syncthreads();                              // red[] complete within the CTA
-    for (int64_t x = threadIdx.x; x < chunk_rows; x += kLutThreads) {
-        // owner = max{j : floor(chunk_rows*j/CS) <= x}
-        const int owner = (int)(((x + 1) * CS - 1) / chunk_rows);
-        const int64_t xo = x - chunk_rows * owner / CS;
-        const int64_t span = chunk_rows * (owner + 1) / CS - chunk_rows * owner / CS;
-        st_dsmem_f32(recv_s + (uint32_t)((rank * span + xo) * 4), (uint32_t)owner, red[x]);
+    {                                             // rows [x0(j), x1(j)) go to rank j
+        const int tpo = kLutThreads / CS;         // threads per destination rank
+        const int j = threadIdx.x / tpo;
+        if (j < CS) {
+            const int jx0 = rows * j / CS, span = rows * (j + 1) / CS - jx0;
+            const uint32_t dst = recv_s + (uint32_t)(rank * span) * 4u;
+            for (int xo = threadIdx.x - j * tpo; xo < span; xo += tpo)
+                st_dsmem_f32(dst + (uint32_t)xo * 4u, (uint32_t)j, red[jx0 + xo]);
+        }
     }
     cluster_sync_all();
-    const int64_t x0 = chunk_rows * rank / CS, x1 = chunk_rows * (rank + 1) / CS;
-    for (int64_t xo = threadIdx.x; xo < x1 - x0; xo += kLutThreads) {
+    const int x0 = rows * rank / CS, my_span = rows * (rank + 1) / CS - x0;
+    for (int xo = threadIdx.x; xo < my_span; xo += kLutThreads) {
         float y = 0.0f;
-        for (int j = 0; j < CS; ++j) y += recv[j * (x1 - x0) + xo];
+        for (int j = 0; j < CS; ++j) y += recv[j * my_span + xo];
         const int64_t r = t_begin * 32 + x0 + xo;
         if (r < N) store_y(Y, ydt, r, y);
     }
