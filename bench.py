@@ -5,8 +5,8 @@ Workload: the Llama-7B q_proj shape, N = K = 4096 with k = 2 residual sign
 planes (W ~ N(0, 0.02) with 0.1% x20 outliers, greedy-SVID scales), decode
 M = 1.  One step = 32 decode tokens, one after another; each token applies 96
 distinct, independent packed layers of that shape to its activation vector
-with rb_gemv_batch (two launches of up to 64 layers, programmatic dependent
-launch between them, captured in a CUDA graph).  The 96 layers hold ~403 MB of
+with one rb_gemv_batch call (one launch; programmatic dependent launch between
+the tokens' launches; captured in a CUDA graph).  The 96 layers hold ~403 MB of
 sign planes, more than the 126 MB L2, so every step streams the planes from
 HBM.  Metric: packed-weight bytes read per second (GB/s).  The same 3072
 applications issued as single-layer rb_gemv calls in one dependent chain are
@@ -117,14 +117,22 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
 
+REJECT_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region.
+
+    Each sample is stamped on arrival; only samples that arrive between begin()
+    and end() (the host-side bracket of the timed region) count.
+    """
 
     def __init__(self, gpu_id: str | None, interval_ms=20):
         self.gpu_id, self.interval_ms = gpu_id, interval_ms
         self.proc, self.lines = None, []
+        self.t0 = self.t1 = None
 
-    def start(self):
+    def start(self, wait_s=5.0):
         cmd = ["nvidia-smi", "--query-gpu=clocks.sm,clocks.max.sm,utilization.gpu,power.draw,clocks_event_reasons.active",
                "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)]
         if self.gpu_id:
@@ -135,10 +143,21 @@ class ClockSampler:
             self.reader.start()
         except Exception:
             self.proc = None
+            return
+        deadline = time.monotonic() + wait_s          # the first sample marks a running sampler
+        while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def begin(self):
+        self.t0 = time.monotonic()
+
+    def end(self):
+        self.t1 = time.monotonic()
+        time.sleep(2.5 * self.interval_ms / 1e3)     # let the last in-window sample arrive
 
     def stop(self):
         if self.proc is None:
@@ -149,27 +168,29 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.reader.join(timeout=2)
+        t0 = self.t0 if self.t0 is not None else float("-inf")
+        t1 = self.t1 if self.t1 is not None else float("inf")
         sm, mx, reasons = [], [], set()
-        for ln in self.lines:
+        for ts, ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 5:
                 continue
             try:
-                s, m, util = float(parts[0]), float(parts[1]), float(parts[2])
+                s, m = float(parts[0]), float(parts[1])
                 bits = int(parts[4], 16) if parts[4].lower().startswith("0x") else int(parts[4])
             except ValueError:
                 continue
             mx.append(m)
-            if util >= 50:
+            if t0 <= ts <= t1:
                 sm.append(s)
                 for b, name in REASON_BITS.items():
                     if bits & b and name != "gpu_idle":
                         reasons.add(name)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
-                    "samples_under_load": 0}
+                    "samples_in_timed_region": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples_under_load": len(sm)}
+                "samples_in_timed_region": len(sm)}
 
 
 def kernel_sources_sha() -> str:
@@ -181,7 +202,7 @@ def kernel_sources_sha() -> str:
 
 
 def profiled_traffic(kernel_tag: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current source."""
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current source."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -194,8 +215,9 @@ def profiled_traffic(kernel_tag: str):
 
 
 # ---------------------------------------------------------------- CPU oracle legs
-def oracle_sample(seconds_budget=15.0, max_layers=64):
-    """Time the oracle's float64 apply on the workload layer (bounded sample)."""
+def oracle_sample(seconds_budget=12.0, max_layers=TOKENS * LAYERS):
+    """Time the oracle's float64 apply on the workload layer: applications until
+    about seconds_budget of CPU work has run, at most one step's worth."""
     import oracle
     from residual_binarized_weight_b200 import synth
     wl = synth.workload(WORKLOAD)
@@ -282,6 +304,7 @@ def run_rbw(args, dist: Dist):
 
     # batch of the 96 layers of a token: host arrays of device pointers, built once
     nb = LAYERS
+    PER_LAUNCH = 96                          # layers per rb_gemv_batch call (one call per token)
     lp = (ctypes.POINTER(rbw.RbLayer) * nb)(*[ctypes.pointer(structs[j]) for j in range(nb)])
     ytmp = torch.empty(LAYERS - 1, N_OUT, dtype=torch.float32, device=dev)
     xps = [(ctypes.c_void_p * nb)(*([X.data_ptr() + t * K_IN * 2] * nb)) for t in range(TOKENS)]
@@ -293,11 +316,14 @@ def run_rbw(args, dist: Dist):
         """32 tokens, one after another; per token one rb_gemv_batch over the 96 layers."""
         sp = ctypes.c_void_p(streams[0].cuda_stream)
         for t in range(TOKENS):
-            st = lib.rb_gemv_batch(ctypes.cast(lp, ctypes.c_void_p), ctypes.cast(xps[t], ctypes.c_void_p),
-                                   ctypes.cast(yps[t], ctypes.c_void_p), nb, 1, rbw.RB_F32, None,
-                                   rbw.RB_LAUNCH_PDL, sp)
-            if st != 0:
-                raise rbw.RbError("rb_gemv_batch", st)
+            for b in range(0, nb, PER_LAUNCH):
+                n = min(PER_LAUNCH, nb - b)
+                st = lib.rb_gemv_batch(ctypes.c_void_p(ctypes.addressof(lp) + b * ctypes.sizeof(ctypes.c_void_p)),
+                                       ctypes.c_void_p(ctypes.addressof(xps[t]) + b * ctypes.sizeof(ctypes.c_void_p)),
+                                       ctypes.c_void_p(ctypes.addressof(yps[t]) + b * ctypes.sizeof(ctypes.c_void_p)),
+                                       n, 1, rbw.RB_F32, None, rbw.RB_LAUNCH_PDL, sp)
+                if st != 0:
+                    raise rbw.RbError("rb_gemv_batch", st)
 
     def step_chain():
         """The same 3072 applications as single-layer rb_gemv calls, one dependent chain (PDL)."""
@@ -326,13 +352,15 @@ def run_rbw(args, dist: Dist):
         torch.cuda.synchronize()
         return gr
 
-    def time_graph(gr, steps, sync_each=False):
+    def time_graph(gr, steps, sync_each=False, sampler=None):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(streams[0]):
             for _ in range(max(3, args.warmup)):
                 gr.replay()
             torch.cuda.synchronize()
             dist.barrier()
+            if sampler:
+                sampler.begin()
             e0.record(streams[0])
             for _ in range(steps):
                 gr.replay()
@@ -340,21 +368,27 @@ def run_rbw(args, dist: Dist):
                     streams[0].synchronize()       # the host reads each step's result
             e1.record(streams[0])
         torch.cuda.synchronize()
+        if sampler:
+            sampler.end()
         dist.barrier()
         return e0.elapsed_time(e1) / 1e3
 
     launches_per_step = TOKENS * LAYERS          # layer applications per step
-    kernel_launches_per_step = TOKENS * ((LAYERS + 63) // 64)
+    kernel_launches_per_step = TOKENS * ((LAYERS + PER_LAUNCH - 1) // PER_LAUNCH)
     plane_bytes = layers[0].packed_bytes()
     bytes_per_step = plane_bytes * launches_per_step
     algo_bytes_per_launch = plane_bytes + 2 * K_PLANES * (N_OUT + K_IN) + 2 * K_IN + 4 * N_OUT
 
     graph = capture(step_batched)
-    sampler = ClockSampler(gpu_uuid(torch))
-    sampler.start()
-    time.sleep(0.05)
-    t_local = time_graph(graph, args.steps)
-    clocks = sampler.stop()
+    for attempt in range(2):                 # a run that saw thermal or hardware slowdown is taken once more
+        sampler = ClockSampler(gpu_uuid(torch))
+        sampler.start()
+        t_local = time_graph(graph, args.steps, sampler=sampler)
+        clocks = sampler.stop()
+        if not (clocks and set(clocks["reasons"]) & REJECT_REASONS):
+            break
+        if clocks:
+            clocks["retaken"] = True
     t_max = dist.max(t_local, dev)
     value = throughput(bytes_per_step, dist.world, args.steps, t_max)
     avg_launch_s = t_local / (args.steps * launches_per_step)      # per layer application
@@ -395,11 +429,12 @@ def run_rbw(args, dist: Dist):
                    "pct_of_peak": {"measured_hbm": value / dist.world / hbm_peak, "spec_8tbs": value / dist.world / 8000.0},
                    "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                                 "frac": achieved / hbm_peak, "traffic": profiled_traffic("gemv_lut_kernel<2>"),
+                                "traffic_unit": "DRAM bytes per launch of %d layers (ncu)" % PER_LAUNCH,
                                 "kernel": "gemv_lut_kernel<2> via rb_gemv_batch", "peak_source": peak_src,
                                 "algorithmic_bytes_per_layer": algo_bytes_per_launch,
-                                "layers_per_launch": LAYERS / ((LAYERS + 63) // 64),
+                                "layers_per_launch": PER_LAUNCH,
                                 "avg_us_per_layer": avg_launch_s * 1e6,
-                                "avg_launch_us": avg_launch_s * 1e6 * LAYERS / ((LAYERS + 63) // 64)},
+                                "avg_launch_us": avg_launch_s * 1e6 * PER_LAUNCH},
                    "cpu_baseline": cb, "e2e": e2e, "gpu_launches": args.steps * kernel_launches_per_step,
                    "decode_chain": chain,
                    "clocks": clocks, "rows": rows})
@@ -476,7 +511,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["rbw", "reference"], default="rbw")
     ap.add_argument("--quick", action="store_true", help="skip the extra per-row timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--mode", choices=["full", "gemv-kernel", "gemv-batch-kernel", "pack-kernel", "gemm-kernel"],
                     default="full",
                     help="kernel-only modes run one kernel a few times (used for ncu captures)")
@@ -506,7 +541,7 @@ def run_kernel_mode(args):
         for _ in range(args.launches):
             rbw.pack(W, g, h, K_PLANES, out=base)
     else:
-        nl = 32
+        nl = 48                             # distinct layers: 48 x 4.2 MB of planes, larger than L2
         layers = []
         for _ in range(nl):
             L = rbw.PackedLayer(N_OUT, K_IN, K_PLANES, dev)

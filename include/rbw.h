@@ -140,9 +140,12 @@ RB_API rb_status rb_gemv(const rb_layer_t *layer, const uint16_t *X, int M,
  * projections of one decode step, or the layers of several models served at
  * once.  layers[j], X[j], Y[j] (host arrays of device pointers) describe
  * application j; Y[j] must not alias any other input or output of the call.
- * For M = 1 one launch serves up to 64 layers and spreads each CTA's table
- * build over more rows, so small layers stream at close to HBM bandwidth.
- * Needs no workspace.
+ * For M = 1 one launch serves up to 128 layers; its shape (CTAs per cluster,
+ * row chunks per layer) is chosen for the whole batch so that every SM stays
+ * busy and each CTA's table builds are spread over many rows.  The per-slice
+ * sums are therefore associated differently than in rb_gemv for the same layer,
+ * so results may differ from rb_gemv's in the last bits; both are
+ * deterministic for a given count.  Needs no workspace.
  */
 RB_API rb_status rb_gemv_batch(const rb_layer_t *const *layers, const uint16_t *const *X, void *const *Y,
                                int count, int M, rb_dtype y_dtype, int32_t *dev_status, unsigned flags,

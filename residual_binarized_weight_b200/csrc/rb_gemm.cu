@@ -34,7 +34,7 @@ namespace {
 
 constexpr int kBR = 128;          // output rows per CTA (MMA M, TMEM lanes)
 constexpr int kBK = 64;           // K per pipeline stage (one 128-byte swizzle row of fp16)
-constexpr int kSX = 8;            // X stages
+constexpr int kSX = 8;            // X stages (at most; fewer when h pairs of a long K need the room)
 constexpr int kThreads = 192;
 constexpr uint64_t kTimeoutNs = 1000000000ull;   // 1 s per wait
 
@@ -155,7 +155,22 @@ __host__ __device__ constexpr int gemm_sa(int kp) { return kp <= 2 ? 4 : 2; }
 __host__ __device__ constexpr int gemm_tmem_cols(int kp) {
     return (kp * gemm_bt(kp) + gemm_sa(kp) * kp * 32) <= 256 ? 256 : 512;
 }
-__host__ __device__ constexpr int gemm_smem_bytes(int kp) { return kSX * gemm_bt(kp) * 128 + 1024 + 256; }
+// With three or more planes the expansion warps are the bottleneck and read the
+// h pairs of the whole layer from shared memory (one bulk copy per CTA) with the
+// sign words a slice ahead; with one or two planes the k-block-ahead loads from
+// global memory measured faster.
+__host__ __device__ constexpr bool gemm_hp_in_smem(int kp) { return kp >= 3; }
+// Shared memory: nsx X stages, the h pairs when they live there (kp * K/2 words), barriers.
+__host__ __device__ inline int gemm_hp_bytes(int kp, int K) {
+    return gemm_hp_in_smem(kp) ? ((kp * (K / 2) * 4) + 127) / 128 * 128 : 0;
+}
+__host__ __device__ inline int gemm_smem_bytes(int kp, int K, int nsx) {
+    return nsx * gemm_bt(kp) * 128 + gemm_hp_bytes(kp, K) + 1024 + 256;
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
 
 // ---------------------------------------------------------------- pre-pass
 // X16[m][32q + 2j + e] = fp16(X[m][32q + j + 16e]);  hperm[i][16q + j] = (h[32q+j], h[32q+j+16]).
@@ -208,7 +223,8 @@ template <int KP>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ planes,
                const uint16_t* __restrict__ g16, const uint32_t* __restrict__ hperm,
-               int N, int K, int M, void* __restrict__ Y, int ydt, int32_t* dev_status, uint64_t timeout_ns)
+               int N, int K, int M, void* __restrict__ Y, int ydt, int32_t* dev_status, uint64_t timeout_ns,
+               int nsx)
 {
     constexpr int BT = gemm_bt(KP), SA = gemm_sa(KP), NCOLS = gemm_tmem_cols(KP);
     constexpr uint32_t X_STAGE = BT * 128;
@@ -220,14 +236,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (sbase - smem_u32(smem_raw));
     const uint32_t xs0 = sbase;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + kSX * X_STAGE);
+    const uint32_t hp_bytes = (uint32_t)gemm_hp_bytes(KP, K);
+    const uint32_t hps = sbase + (uint32_t)nsx * X_STAGE;           // h pairs, [plane][K/2]
+    const uint32_t* hsm = reinterpret_cast<const uint32_t*>(gbase + (size_t)nsx * X_STAGE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + (size_t)nsx * X_STAGE + hp_bytes);
     const uint32_t bar0 = smem_u32(bars);
     auto full_x = [&](int s) { return bar0 + 8u * s; };
     auto empty_x = [&](int s) { return bar0 + 8u * (kSX + s); };
     auto full_a = [&](int s) { return bar0 + 8u * (2 * kSX + s); };
     auto empty_a = [&](int s) { return bar0 + 8u * (2 * kSX + SA + s); };
     const uint32_t acc_full = bar0 + 8u * (2 * kSX + 2 * SA);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kSX + 2 * SA + 1);
+    const uint32_t hp_full = bar0 + 8u * (2 * kSX + 2 * SA + 1);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kSX + 2 * SA + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -238,6 +258,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
         for (int s = 0; s < kSX; ++s) { mbar_init(full_x(s), 1); mbar_init(empty_x(s), 1); }
         for (int s = 0; s < SA; ++s) { mbar_init(full_a(s), 128); mbar_init(empty_a(s), 1); }
         mbar_init(acc_full, 1);
+        mbar_init(hp_full, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(&tmap_x) : "memory");
@@ -256,25 +277,34 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
 
     if (warp == 0) {
         if (lane == 0) {                          // ---------------- TMA producer
-            int issued = 0;
+            if constexpr (gemm_hp_in_smem(KP)) {
+                mbar_arrive_expect_tx(hp_full, (uint32_t)(KP * (K / 2) * 4));
+                bulk_load(hps, hperm, (uint32_t)(KP * (K / 2) * 4), hp_full);
+            }
+            // stage s and its fill count j (phase = j & 1) advance without divisions
+            int issued = 0, s = 0, j = 0;
             for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % kSX, j = kb / kSX;
                 if (j > 0 && !mbar_wait(empty_x(s), (j - 1) & 1, abort_flag, dev_status, timeout_ns)) break;
                 mbar_arrive_expect_tx(full_x(s), X_STAGE);
                 tma_load_2d(xs0 + s * X_STAGE, &tmap_x, full_x(s), kb * kBK, m0);
                 ++issued;
+                if (++s == nsx) { s = 0; ++j; }
             }
             if (*abort_flag) {                    // drain the loads this thread issued (bounded)
                 const uint64_t t0 = globaltimer_ns();
-                for (int kb = issued - kSX < 0 ? 0 : issued - kSX; kb < issued; ++kb)
-                    while (!mbar_try_wait(full_x(kb % kSX), (kb / kSX) & 1) && globaltimer_ns() - t0 < timeout_ns) {}
+                for (int kb = issued - nsx < 0 ? 0 : issued - nsx; kb < issued; ++kb)
+                    while (!mbar_try_wait(full_x(kb % nsx), (kb / nsx) & 1) && globaltimer_ns() - t0 < timeout_ns) {}
+                if constexpr (gemm_hp_in_smem(KP))
+                    while (!mbar_try_wait(hp_full, 0) && globaltimer_ns() - t0 < timeout_ns) {}
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {                          // ---------------- MMA issuer
+            int s = 0;
+            uint32_t xphase = 0;
             for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % kSX, sa = kb % SA;
-                if (!mbar_wait(full_x(s), (kb / kSX) & 1, abort_flag, dev_status, timeout_ns)) break;
+                const int sa = kb % SA;
+                if (!mbar_wait(full_x(s), xphase, abort_flag, dev_status, timeout_ns)) break;
                 if (!mbar_wait(full_a(sa), (kb / SA) & 1, abort_flag, dev_status, timeout_ns)) break;
                 tc_fence_after();
                 const uint32_t xaddr = xs0 + s * X_STAGE;
@@ -290,6 +320,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
                 }
                 tc_commit(empty_x(s));
                 tc_commit(empty_a(sa));
+                if (++s == nsx) { s = 0; xphase ^= 1u; }
             }
             tc_commit(acc_full);                  // arrives once every MMA issued above is done
         }
@@ -301,62 +332,121 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
         const int64_t tile = n >> 5;
         const bool tile_ok = tile < Nt;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        // sign words and +-h pairs of one k-block, fetched one k-block ahead
-        auto load_kb = [&](int kb, uint32_t (&wv)[KP][2], uint32_t (&hp)[KP][32]) {
-            const int64_t sl = kb / 4;
-            const int w0 = (kb & 3) * 2;
-#pragma unroll
-            for (int i = 0; i < KP; ++i) {
-#pragma unroll
-                for (int ww = 0; ww < 2; ++ww) {
-                    const int64_t col0 = (int64_t)kb * kBK + ww * 32;
-                    wv[i][ww] = (tile_ok && col0 < K)
-                        ? planes[block_index(i, sl, tile, S, Nt) * 256 + (((w0 + ww) ^ (lane >> 2)) * 32) + lane]
-                        : 0u;
-                }
-                const int64_t hbase = (int64_t)i * (K / 2) + (int64_t)kb * 32;
-#pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    uint4 u = make_uint4(0, 0, 0, 0);
-                    if ((int64_t)kb * 32 + 4 * v < K / 2) u = *reinterpret_cast<const uint4*>(hperm + hbase + 4 * v);
-                    hp[i][4 * v] = u.x; hp[i][4 * v + 1] = u.y; hp[i][4 * v + 2] = u.z; hp[i][4 * v + 3] = u.w;
-                }
-            }
-        };
-        uint32_t wv[KP][2], hp[KP][32];
-        load_kb(0, wv, hp);
         bool ok = true;
-        for (int kb = 0; kb < nkb && ok; ++kb) {
-            const int sa = kb % SA;
-            uint32_t cw[KP][2], ch[KP][32];
+        if constexpr (!gemm_hp_in_smem(KP)) {
+            // Sign words and +-h pairs of one k-block, fetched one k-block ahead from
+            // global memory (L1/L2 hits: every row of the CTA reads the same h pairs).
+            auto load_kb = [&](int kb, uint32_t (&wv)[KP][2], uint32_t (&hp)[KP][32]) {
+                const int64_t sl = kb / 4;
+                const int w0 = (kb & 3) * 2;
 #pragma unroll
-            for (int i = 0; i < KP; ++i) {
-                cw[i][0] = wv[i][0];
-                cw[i][1] = wv[i][1];
+                for (int i = 0; i < KP; ++i) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) ch[i][j] = hp[i][j];
-            }
-            if (kb + 1 < nkb) load_kb(kb + 1, wv, hp);
-            if (kb >= SA) {
-                if (!mbar_wait_warp(empty_a(sa), ((kb / SA) - 1) & 1, abort_flag, dev_status, timeout_ns)) {
-                    ok = false;
-                    break;
+                    for (int ww = 0; ww < 2; ++ww) {
+                        const int64_t col0 = (int64_t)kb * kBK + ww * 32;
+                        wv[i][ww] = (tile_ok && col0 < K)
+                            ? planes[block_index(i, sl, tile, S, Nt) * 256 + (((w0 + ww) ^ (lane >> 2)) * 32) + lane]
+                            : 0u;
+                    }
+                    const int64_t hbase = (int64_t)i * (K / 2) + (int64_t)kb * 32;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        uint4 u = make_uint4(0, 0, 0, 0);
+                        if ((int64_t)kb * 32 + 4 * v < K / 2) u = *reinterpret_cast<const uint4*>(hperm + hbase + 4 * v);
+                        hp[i][4 * v] = u.x; hp[i][4 * v + 1] = u.y; hp[i][4 * v + 2] = u.z; hp[i][4 * v + 3] = u.w;
+                    }
                 }
-                tc_fence_after();
+            };
+            uint32_t wv[KP][2], hp[KP][32];
+            load_kb(0, wv, hp);
+            for (int kb = 0; kb < nkb && ok; ++kb) {
+                const int sa = kb % SA;
+                uint32_t cw[KP][2], ch[KP][32];
+#pragma unroll
+                for (int i = 0; i < KP; ++i) {
+                    cw[i][0] = wv[i][0];
+                    cw[i][1] = wv[i][1];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) ch[i][j] = hp[i][j];
+                }
+                if (kb + 1 < nkb) load_kb(kb + 1, wv, hp);
+                if (kb >= SA) {
+                    if (!mbar_wait_warp(empty_a(sa), ((kb / SA) - 1) & 1, abort_flag, dev_status, timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+#pragma unroll
+                for (int i = 0; i < KP; ++i) {
+                    uint32_t a[32];
+#pragma unroll
+                    for (int ww = 0; ww < 2; ++ww)
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            a[ww * 16 + j] = lop3_sign(cw[i][ww] << (15 - j), ch[i][ww * 16 + j]);
+                    tc_st_32x32b_x32(tmem + lane_base + (uint32_t)(KP * BT + (sa * KP + i) * 32), a);
+                }
+                tc_wait_st();
+                tc_fence_before();
+                mbar_arrive(full_a(sa));
             }
-#pragma unroll
-            for (int i = 0; i < KP; ++i) {
-                uint32_t a[32];
-#pragma unroll
-                for (int ww = 0; ww < 2; ++ww)
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        a[ww * 16 + j] = lop3_sign(cw[i][ww] << (15 - j), ch[i][ww * 16 + j]);
-                tc_st_32x32b_x32(tmem + lane_base + (uint32_t)(KP * BT + (sa * KP + i) * 32), a);
+        } else {
+            // Sign words: the 8 logical words of a 256-column slice (4 k-blocks) per
+            // plane, loaded one slice ahead.  h pairs: from shared memory.
+            auto load_slice = [&](int64_t sl, uint32_t (&wv)[KP][8]) {
+    #pragma unroll
+                for (int i = 0; i < KP; ++i) {
+                    const uint32_t* blk = planes + block_index(i, sl, tile, S, Nt) * 256 + lane;
+    #pragma unroll
+                    for (int w = 0; w < 8; ++w)
+                        wv[i][w] = (tile_ok && sl * 256 + w * 32 < K) ? blk[((w ^ (lane >> 2)) * 32)] : 0u;
+                }
+            };
+            uint32_t cur[KP][8], nxt[KP][8];
+            load_slice(0, cur);
+            ok = mbar_wait_warp(hp_full, 0, abort_flag, dev_status, timeout_ns);
+            for (int64_t sl = 0; sl < S && ok; ++sl) {
+                if (sl + 1 < S) load_slice(sl + 1, nxt);
+    #pragma unroll
+                for (int qk = 0; qk < 4; ++qk) {
+                    const int kb = (int)sl * 4 + qk;
+                    if (kb >= nkb || !ok) break;
+                    const int sa = kb % SA;
+                    if (kb >= SA) {
+                        if (!mbar_wait_warp(empty_a(sa), ((kb / SA) - 1) & 1, abort_flag, dev_status, timeout_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+    #pragma unroll
+                    for (int i = 0; i < KP; ++i) {
+                        uint32_t hp[32];
+                        const uint32_t* hrow = hsm + (size_t)i * (K / 2) + (size_t)kb * 32;
+    #pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            uint4 u = make_uint4(0, 0, 0, 0);
+                            if (kb * 32 + 4 * v < K / 2) u = *reinterpret_cast<const uint4*>(hrow + 4 * v);
+                            hp[4 * v] = u.x; hp[4 * v + 1] = u.y; hp[4 * v + 2] = u.z; hp[4 * v + 3] = u.w;
+                        }
+                        uint32_t a[32];
+    #pragma unroll
+                        for (int ww = 0; ww < 2; ++ww)
+    #pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                a[ww * 16 + j] = lop3_sign(cur[i][2 * qk + ww] << (15 - j), hp[ww * 16 + j]);
+                        tc_st_32x32b_x32(tmem + lane_base + (uint32_t)(KP * BT + (sa * KP + i) * 32), a);
+                    }
+                    tc_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(full_a(sa));
+                }
+    #pragma unroll
+                for (int i = 0; i < KP; ++i)
+    #pragma unroll
+                    for (int w = 0; w < 8; ++w) cur[i][w] = nxt[i][w];
             }
-            tc_wait_st();
-            tc_fence_before();
-            mbar_arrive(full_a(sa));
         }
         // ---- epilogue
         if (ok && mbar_wait_warp(acc_full, 0, abort_flag, dev_status, timeout_ns)) {
@@ -370,14 +460,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
                 float y[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) y[j] = 0.0f;
+                uint32_t v[KP][32];
 #pragma unroll
-                for (int i = 0; i < KP; ++i) {
-                    uint32_t v[32];
-                    tc_ld_32x32b_x32(tmem + lane_base + (uint32_t)(i * BT + c * 32), v);
-                    tc_wait_ld();
+                for (int i = 0; i < KP; ++i) tc_ld_32x32b_x32(tmem + lane_base + (uint32_t)(i * BT + c * 32), v[i]);
+                tc_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) y[j] = fmaf(gi[i], __uint_as_float(v[j]), y[j]);
-                }
+                for (int i = 0; i < KP; ++i)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) y[j] = fmaf(gi[i], __uint_as_float(v[i][j]), y[j]);
                 if (n < N) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
@@ -454,15 +544,19 @@ rb_status launch_gemm(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    const int smem = gemm_smem_bytes(KP);
+    constexpr int kMaxSmem = 227 * 1024;
+    int nsx = kSX;
+    while (nsx > 2 && gemm_smem_bytes(KP, L->k_in, nsx) > kMaxSmem) --nsx;
+    const int smem = gemm_smem_bytes(KP, L->k_in, nsx);
+    if (smem > kMaxSmem) return RB_ERR_UNSUPPORTED;          // K too long for the h pairs in shared memory
     if (dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(gemm_tc_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        if (cudaFuncSetAttribute(gemm_tc_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem) != cudaSuccess)
             return RB_ERR_CUDA;
         attr_set[dev] = true;
     }
     dim3 grid((unsigned)((L->n_out + kBR - 1) / kBR), (unsigned)((M + BT - 1) / BT));
     return launch(gemm_tc_kernel<KP>, grid, dim3(kThreads), (size_t)smem, stream, pdl, map, L->planes,
-                  L->g16, (const uint32_t*)ws.hperm, L->n_out, L->k_in, M, Y, ydt, dev_status, timeout_ns);
+                  L->g16, (const uint32_t*)ws.hperm, L->n_out, L->k_in, M, Y, ydt, dev_status, timeout_ns, nsx);
 }
 
 }  // namespace

@@ -23,6 +23,8 @@
 // registers and needs no workspace.
 #include "rbw_internal.cuh"
 
+#include <mutex>
+
 namespace rbw {
 namespace {
 
@@ -99,6 +101,15 @@ __device__ __forceinline__ void st_dsmem_f32(uint32_t local_saddr, uint32_t rank
     uint32_t remote;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(rank));
     asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(remote), "f"(v) : "memory");
+}
+
+// Per-row sums (red) plus, with a cluster, the receive area of the rows this CTA
+// sums: CS slots of at most ceil(rows/CS) rows, which never exceeds rows + CS;
+// rounded up to 16 bytes.
+__host__ __device__ inline int lut_row_bytes(int64_t Nt, int R, int CS)
+{
+    const int64_t rows = ((Nt + R - 1) / R) * 32;
+    return (int)(((CS > 1 ? 2 * rows + CS : rows) + 3) / 4 * 16);
 }
 
 // Byte tables of slice s for all KP planes (256 threads: thread (group gg,
@@ -203,15 +214,20 @@ template <int KP, bool FAST>
 __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_t (&gv)[kLutPF][KP],
                                           const uint32_t (&G)[8], const uint32_t (&SEL)[4], uint32_t tbase,
                                           float* red, const uint32_t* __restrict__ planes,
-                                          const uint16_t* __restrict__ g16, int64_t s, int64_t S, int64_t Nt,
-                                          int N, int tb, int te, int warp, int lane)
+                                          const uint16_t* __restrict__ g16, int64_t s, int64_t s_next,
+                                          int64_t S, int64_t Nt, int N, int tb, int te, int warp, int lane)
 {
     const uint32_t* pbase[KP];
 #pragma unroll
     for (int i = 0; i < KP; ++i) pbase[i] = planes + block_index(i, s, 0, S, Nt) * 256 + lane;
-    // this lane's L2-prefetch line: plane lane/8, line lane%8 of a tile block
+    // this lane's L2-prefetch line: plane lane/8, line lane%8 of a tile block, in
+    // this slice and in the CTA's next one (prefetches run on into it: a warp's
+    // tiles there are the same t as here, its sequence restarting at tb + warp)
     const uint32_t* pf_base = lane < 8 * KP
         ? planes + block_index(lane >> 3, s, 0, S, Nt) * 256 + (lane & 7) * 32 : planes;
+    const uint32_t* pf_next = (lane < 8 * KP && s_next < S)
+        ? planes + block_index(lane >> 3, s_next, 0, S, Nt) * 256 + (lane & 7) * 32 : nullptr;
+    const int wrap = te - tb > warp ? ((te - tb - warp + kLutWarps - 1) / kLutWarps) * kLutWarps : 0;
     for (int t0 = tb + warp; t0 < te; t0 += kLutPF * kLutWarps) {
         float acc[kLutPF][KP][2];
 #pragma unroll
@@ -229,8 +245,11 @@ __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_
                     pr += __half2float(__ushort_as_half(gv[p][i])) * (acc[p][i][0] + acc[p][i][1]);
                 red[(t - tb) * 32 + lane] += pr;
                 const int tp = t + kLutPD * kLutWarps;                  // L2 prefetch further ahead
-                if (tp < te && lane < 8 * KP)
-                    asm volatile("prefetch.global.L2 [%0];" :: "l"(pf_base + (size_t)tp * 256));
+                if (tp < te) {
+                    if (lane < 8 * KP) asm volatile("prefetch.global.L2 [%0];" :: "l"(pf_base + (size_t)tp * 256));
+                } else if (pf_next != nullptr && tp - wrap < te) {
+                    asm volatile("prefetch.global.L2 [%0];" :: "l"(pf_next + (size_t)(tp - wrap) * 256));
+                }
                 const int tn = t + kLutPF * kLutWarps;                  // refill this slot
                 if (tn < te) {
 #pragma unroll
@@ -249,7 +268,7 @@ __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_
 // stay in shared memory until each is stored into the receive area of the CTA
 // that sums that row; after one cluster barrier that CTA adds the CS partial
 // sums in rank order and writes Y.  With CS = 1 the CTA owns every slice.
-constexpr int kMaxBatch = 64;          // layers per launch of the byte-table kernel
+constexpr int kMaxBatch = 128;         // layers per launch of the byte-table kernel
 
 // Independent layers of one shape handled by one launch (pointers per layer).
 struct LutBatch {
@@ -340,9 +359,11 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
         __syncthreads();
 
         if (fast_base)
-            lut_tiles<KP, true>(wd, gv, G, SEL, tbase, red, planes, g16, s, S, Nt, N, (int)t_begin, (int)t_end, warp, lane);
+            lut_tiles<KP, true>(wd, gv, G, SEL, tbase, red, planes, g16, s, s + CS, S, Nt, N, (int)t_begin,
+                                (int)t_end, warp, lane);
         else
-            lut_tiles<KP, false>(wd, gv, G, SEL, tbase, red, planes, g16, s, S, Nt, N, (int)t_begin, (int)t_end, warp, lane);
+            lut_tiles<KP, false>(wd, gv, G, SEL, tbase, red, planes, g16, s, s + CS, S, Nt, N, (int)t_begin,
+                                 (int)t_end, warp, lane);
     }
 
     // ---- cross-slice sum
@@ -481,56 +502,148 @@ cudaLaunchConfig_t lut_config(const LutPlan& p, int count, cudaLaunchAttribute* 
     return cfg;
 }
 
-// Per-row sums (red) plus, with a cluster, the receive area of the rows this CTA
-// sums: CS slots of at most ceil(rows/CS) rows, which never exceeds rows + CS.
-int lut_row_bytes(int64_t Nt, int R, int CS)
-{
-    const int64_t rows = ((Nt + R - 1) / R) * 32;
-    return (int)((CS > 1 ? 2 * rows + CS : rows) * 4);
-}
-
-// Slices per CTA = ceil(S/16), CS = ceil(S / that) CTAs per cluster.  Row
-// chunks per layer (R): a single layer takes as many as fill the SMs (lowest
-// latency); a batch of `count` layers takes as few as keep about two CTAs per
-// SM busy, so each CTA's table build is spread over more rows.  R is capped by
-// the clusters the GPU keeps resident, the row tiles and shared memory.
 template <int KP>
-rb_status lut_plan(int N, int K, int count, LutPlan* plan)
+bool lut_set_attributes()
 {
-    const int64_t S = num_slices(K), Nt = num_row_tiles(N);
-    const int spc = (int)((S + 15) / 16);
-    const int CS = (int)((S + spc - 1) / spc);
-    const int sms = num_sms();
-    int R = CS > 1 ? sms / CS : sms;
-    if (count > 1) R = (int)((2 * sms + (int64_t)count * CS - 1) / ((int64_t)count * CS));
-    if (R < 1) R = 1;
-    if (R > Nt) R = (int)Nt;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) return RB_ERR_UNSUPPORTED;
+    if (dev < 0 || dev >= 64) return false;
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(gemv_lut_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
-            return RB_ERR_CUDA;
+            return false;
         if (cudaFuncSetAttribute(gemv_lut_kernel<KP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-            return RB_ERR_CUDA;
+            return false;
         attr_set[dev] = true;
     }
-    // shared memory: at most ~105 KB per CTA so that two CTAs fit on an SM
-    while (R < Nt && lut_table_bytes(KP) + lut_row_bytes(Nt, R, CS) > 105 * 1024) ++R;
-    LutPlan p{CS, R, lut_table_bytes(KP) + lut_row_bytes(Nt, R, CS)};
-    if (CS > 1 && count == 1) {
-        cudaLaunchAttribute attr[2];
-        cudaLaunchConfig_t cfg = lut_config(p, 1, attr, false, 0);
-        int active = 0;
-        if (cudaOccupancyMaxActiveClusters(&active, gemv_lut_kernel<KP>, &cfg) == cudaSuccess && active > 0 &&
-            active < R) {
-            p.R = active;
-            p.smem = lut_table_bytes(KP) + lut_row_bytes(Nt, p.R, CS);
+    return true;
+}
+
+// Clusters of CS CTAs (CTAs when CS = 1) the GPU keeps resident with `smem`
+// bytes per CTA, or 0 if the query fails.
+template <int KP>
+int lut_resident(int CS, int smem)
+{
+    LutPlan p{CS, 1, smem};
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = lut_config(p, 1, attr, false, 0);
+    int n = 0;
+    if (CS > 1) {
+        if (cudaOccupancyMaxActiveClusters(&n, gemv_lut_kernel<KP>, &cfg) != cudaSuccess) n = 0;
+    } else {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_lut_kernel<KP>, kLutThreads, (size_t)smem) !=
+            cudaSuccess)
+            n = 0;
+        n *= num_sms();
+    }
+    return n;
+}
+
+// Cost of one slice's table build, in units of one row tile's lookups per warp
+// (64 stores and ~80 arithmetic instructions per thread plus the barriers).
+constexpr int kLutBuildTiles = 8;
+
+// Single layer (count == 1): lowest latency.  Slices per CTA = ceil(S/16),
+// CS = ceil(S / that) CTAs per cluster, as many row chunks (R) as the GPU keeps
+// clusters resident, one wave.
+// Batch: CS (a power of two) and R minimise the modelled time waves * (time of
+// one CTA), where a CTA builds ceil(S/CS) tables and runs ceil(rows/R) row
+// tiles through each, and the count * R clusters run in ceil(count * R /
+// resident) waves of the clusters the GPU keeps resident (fewer for larger
+// clusters: a cluster's CTAs share a GPC).  A single wave that leaves resident
+// slots empty is charged for them in part (x 1 + (empty fraction) / 2): the
+// CTAs then crowd some SMs while others idle.  Measured on 4096 x 4096 layers,
+// full waves of 8-CTA clusters with all rows per CTA came out fastest.
+template <int KP>
+rb_status lut_plan_uncached(int N, int K, int count, LutPlan* plan)
+{
+    const int64_t S = num_slices(K), Nt = num_row_tiles(N);
+    constexpr int kSmemCap = 105 * 1024;        // two CTAs per SM, when the tables leave room
+    const int cap = lut_table_bytes(KP) < 96 * 1024 ? kSmemCap : 227 * 1024;
+    if (count == 1) {
+        const int spc = (int)((S + 15) / 16);
+        const int CS = (int)((S + spc - 1) / spc);
+        const int sms = num_sms();
+        int R = CS > 1 ? sms / CS : sms;
+        if (R < 1) R = 1;
+        if (R > Nt) R = (int)Nt;
+        while (R < Nt && lut_table_bytes(KP) + lut_row_bytes(Nt, R, CS) > cap) ++R;
+        LutPlan p{CS, R, lut_table_bytes(KP) + lut_row_bytes(Nt, R, CS)};
+        if (CS > 1) {
+            const int active = lut_resident<KP>(CS, p.smem);
+            if (active > 0 && active < R) {
+                p.R = active;
+                p.smem = lut_table_bytes(KP) + lut_row_bytes(Nt, p.R, CS);
+            }
+        }
+        if (p.smem > 227 * 1024) return RB_ERR_UNSUPPORTED;
+        *plan = p;
+        return RB_OK;
+    }
+    LutPlan best{0, 0, 0};
+    double best_cost = 1e300;
+    for (int CS = 1; CS <= 16 && (CS == 1 || CS <= S); CS *= 2) {
+        const int64_t spc = (S + CS - 1) / CS;
+        int resident = -1;
+        const int rmax = (int)(Nt < 4096 ? Nt : 4096);
+        for (int R = 1; R <= rmax; ++R) {
+            const int smem = lut_table_bytes(KP) + lut_row_bytes(Nt, R, CS);
+            if (smem > cap) continue;
+            if (resident < 0) resident = lut_resident<KP>(CS, smem);   // a lower bound for larger R (less smem)
+            if (resident <= 0) break;
+            const int64_t units = (int64_t)count * R;
+            const int64_t waves = (units + resident - 1) / resident;
+            const int64_t tiles = (Nt + R - 1) / R;
+            const int64_t per_cta = spc * (kLutBuildTiles + (tiles + kLutWarps - 1) / kLutWarps * kLutWarps);
+            double cost = (double)(waves * per_cta);
+            if (units < resident) cost *= 1.0 + 0.5 * (double)(resident - units) / (double)resident;
+            if (cost < best_cost) {
+                best_cost = cost;
+                best = LutPlan{CS, R, smem};
+            }
+            if (units >= 4 * (int64_t)resident) break;      // later R only add waves
         }
     }
-    if (p.smem > 227 * 1024) return RB_ERR_UNSUPPORTED;
-    *plan = p;
+    if (best.CS == 0) return RB_ERR_UNSUPPORTED;
+    *plan = best;
+    return RB_OK;
+}
+
+// Plans are cached per (device, k, N, K, count): the occupancy queries behind
+// them cost more host time than a launch.
+struct LutPlanKey {
+    int dev, kp, N, K, count;
+    bool operator==(const LutPlanKey& o) const {
+        return dev == o.dev && kp == o.kp && N == o.N && K == o.K && count == o.count;
+    }
+};
+constexpr int kPlanCache = 256;
+std::mutex g_plan_mu;
+LutPlanKey g_plan_keys[kPlanCache];
+LutPlan g_plan_vals[kPlanCache];
+int g_plan_n = 0;
+
+template <int KP>
+rb_status lut_plan(int N, int K, int count, LutPlan* plan)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RB_ERR_CUDA;
+    if (!lut_set_attributes<KP>()) return RB_ERR_CUDA;
+    const LutPlanKey key{dev, KP, N, K, count};
+    {
+        std::lock_guard<std::mutex> lk(g_plan_mu);
+        for (int j = 0; j < g_plan_n; ++j)
+            if (g_plan_keys[j] == key) {
+                *plan = g_plan_vals[j];
+                return RB_OK;
+            }
+    }
+    rb_status st = lut_plan_uncached<KP>(N, K, count, plan);
+    if (st != RB_OK) return st;
+    std::lock_guard<std::mutex> lk(g_plan_mu);
+    const int j = g_plan_n < kPlanCache ? g_plan_n++ : (int)((unsigned)(N ^ K ^ count) % kPlanCache);
+    g_plan_keys[j] = key;
+    g_plan_vals[j] = *plan;
     return RB_OK;
 }
 
