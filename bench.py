@@ -541,7 +541,7 @@ def run_kernel_mode(args):
         for _ in range(args.launches):
             rbw.pack(W, g, h, K_PLANES, out=base)
     else:
-        nl = 48                             # distinct layers: 48 x 4.2 MB of planes, larger than L2
+        nl = LAYERS                         # distinct layers: 96 x 4.2 MB of planes, larger than L2
         layers = []
         for _ in range(nl):
             L = rbw.PackedLayer(N_OUT, K_IN, K_PLANES, dev)

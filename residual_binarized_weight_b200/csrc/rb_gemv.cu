@@ -210,6 +210,14 @@ __device__ __forceinline__ void lut_lookups(float (&acc)[kLutPF][KP][2], const u
     }
 }
 
+// The row tiles of one slice for this warp: t = tb + warp + 8 j, j < nw, kLutPF
+// at a time from registers.  Each slot is refilled right after its lookups:
+// with the tile kLutPF further on, clamped to the warp's last tile when that
+// runs past the end (the slot is then not used), and after the last group with
+// tile j = slot of the CTA's next slice, so a slice starts on loaded registers.
+// L2 prefetches run kLutPD tiles ahead in the same sequence, on into the next
+// slice.  Tile validity only gates the red[] update, so no load is guarded by
+// a branch.
 template <int KP, bool FAST>
 __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_t (&gv)[kLutPF][KP],
                                           const uint32_t (&G)[8], const uint32_t (&SEL)[4], uint32_t tbase,
@@ -217,47 +225,57 @@ __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_
                                           const uint16_t* __restrict__ g16, int64_t s, int64_t s_next,
                                           int64_t S, int64_t Nt, int N, int tb, int te, int warp, int lane)
 {
-    const uint32_t* pbase[KP];
+    const int nw = te - tb > warp ? (te - tb - warp + kLutWarps - 1) / kLutWarps : 0;
+    const int iters = (nw + kLutPF - 1) / kLutPF;
+    const bool has_next = s_next < S;
+    const uint32_t* cur[KP];
+    const uint32_t* nxt[KP];
 #pragma unroll
-    for (int i = 0; i < KP; ++i) pbase[i] = planes + block_index(i, s, 0, S, Nt) * 256 + lane;
-    // this lane's L2-prefetch line: plane lane/8, line lane%8 of a tile block, in
-    // this slice and in the CTA's next one (prefetches run on into it: a warp's
-    // tiles there are the same t as here, its sequence restarting at tb + warp)
-    const uint32_t* pf_base = lane < 8 * KP
-        ? planes + block_index(lane >> 3, s, 0, S, Nt) * 256 + (lane & 7) * 32 : planes;
-    const uint32_t* pf_next = (lane < 8 * KP && s_next < S)
-        ? planes + block_index(lane >> 3, s_next, 0, S, Nt) * 256 + (lane & 7) * 32 : nullptr;
-    const int wrap = te - tb > warp ? ((te - tb - warp + kLutWarps - 1) / kLutWarps) * kLutWarps : 0;
-    for (int t0 = tb + warp; t0 < te; t0 += kLutPF * kLutWarps) {
+    for (int i = 0; i < KP; ++i) {
+        cur[i] = planes + block_index(i, s, 0, S, Nt) * 256 + lane;
+        nxt[i] = has_next ? planes + block_index(i, s_next, 0, S, Nt) * 256 + lane : cur[i];
+    }
+    // this lane's L2-prefetch line: plane lane/8, line lane%8 of a tile block
+    const bool pf_lane = lane < 8 * KP;
+    const uint32_t* pf_cur = planes + block_index(pf_lane ? lane >> 3 : 0, s, 0, S, Nt) * 256 + (lane & 7) * 32;
+    const uint32_t* pf_nxt = has_next
+        ? planes + block_index(pf_lane ? lane >> 3 : 0, s_next, 0, S, Nt) * 256 + (lane & 7) * 32 : pf_cur;
+    const int t_w = tb + warp;                    // the warp's first tile
+    for (int it = 0; it < iters; ++it) {
         float acc[kLutPF][KP][2];
 #pragma unroll
         for (int p = 0; p < kLutPF; ++p)
 #pragma unroll
             for (int i = 0; i < KP; ++i) acc[p][i][0] = acc[p][i][1] = 0.0f;
         lut_lookups<KP, FAST>(acc, wd, G, SEL, tbase);
+        const bool last = it + 1 == iters;
 #pragma unroll
         for (int p = 0; p < kLutPF; ++p) {
-            const int t = t0 + p * kLutWarps;
-            if (t < te) {
-                float pr = 0.0f;
+            const int j = it * kLutPF + p;
+            float pr = 0.0f;
 #pragma unroll
-                for (int i = 0; i < KP; ++i)
-                    pr += __half2float(__ushort_as_half(gv[p][i])) * (acc[p][i][0] + acc[p][i][1]);
-                red[(t - tb) * 32 + lane] += pr;
-                const int tp = t + kLutPD * kLutWarps;                  // L2 prefetch further ahead
-                if (tp < te) {
-                    if (lane < 8 * KP) asm volatile("prefetch.global.L2 [%0];" :: "l"(pf_base + (size_t)tp * 256));
-                } else if (pf_next != nullptr && tp - wrap < te) {
-                    asm volatile("prefetch.global.L2 [%0];" :: "l"(pf_next + (size_t)(tp - wrap) * 256));
+            for (int i = 0; i < KP; ++i)
+                pr += __half2float(__ushort_as_half(gv[p][i])) * (acc[p][i][0] + acc[p][i][1]);
+            if (j < nw) red[(j * kLutWarps + warp) * 32 + lane] += pr;
+            const int jp = j + kLutPD;
+            const bool pf_here = jp < nw;
+            if (pf_lane && (pf_here || (has_next && jp - nw < nw))) {
+                const uint32_t* q = pf_here ? pf_cur + (size_t)(t_w + jp * kLutWarps) * 256
+                                            : pf_nxt + (size_t)(t_w + (jp - nw) * kLutWarps) * 256;
+                asm volatile("prefetch.global.L2 [%0];" :: "l"(q));
+            }
+            if (!last || (has_next && p < nw)) {
+                const int jn = last ? p : min(j + kLutPF, nw - 1);
+                const size_t tn = (size_t)(t_w + jn * kLutWarps);
+#pragma unroll
+                for (int i = 0; i < KP; ++i) {
+                    const uint32_t* q = (last ? nxt[i] : cur[i]) + tn * 256;
+#pragma unroll
+                    for (int sl = 0; sl < 8; ++sl) wd[p][i][sl] = __ldcs(q + sl * 32);
                 }
-                const int tn = t + kLutPF * kLutWarps;                  // refill this slot
-                if (tn < te) {
+                const int64_t r = min((int64_t)tn * 32 + lane, (int64_t)N - 1);
 #pragma unroll
-                    for (int i = 0; i < KP; ++i)
-#pragma unroll
-                        for (int sl = 0; sl < 8; ++sl) wd[p][i][sl] = __ldcs(pbase[i] + (size_t)tn * 256 + sl * 32);
-                    lut_load_g<KP>(gv[p], g16, (int64_t)tn * 32 + lane, N);
-                }
+                for (int i = 0; i < KP; ++i) gv[p][i] = g16[(int64_t)i * N + r];
             }
         }
     }
@@ -310,6 +328,13 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
         if (t < t_end && s_first < S) {
             lut_load_tile<KP>(wd[p], planes, s_first, t, S, Nt, lane);
             lut_load_g<KP>(gv[p], g16, t * 32 + lane, N);
+        } else {                                  // an unused slot: defined values for its lookups
+#pragma unroll
+            for (int i = 0; i < KP; ++i) {
+#pragma unroll
+                for (int sl = 0; sl < 8; ++sl) wd[p][i][sl] = 0u;
+                gv[p][i] = 0;
+            }
         }
     }
     if (s_first < S) {
@@ -345,15 +370,7 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
     for (int64_t s = s_first; s < S; s += CS) {
         if (s != s_first) {
             __syncthreads();                      // the previous slice's lookups are done with the tables
-            lut_load_h<KP>(hr, h16, s, K);
-#pragma unroll
-            for (int p = 0; p < kLutPF; ++p) {
-                const int64_t t = t_begin + warp + (int64_t)p * kLutWarps;
-                if (t < t_end) {
-                    lut_load_tile<KP>(wd[p], planes, s, t, S, Nt, lane);
-                    lut_load_g<KP>(gv[p], g16, t * 32 + lane, N);
-                }
-            }
+            lut_load_h<KP>(hr, h16, s, K);        // (its tiles are in registers already)
         }
         lut_build<KP>(lut, hr, X, s, K);
         __syncthreads();
