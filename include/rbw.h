@@ -117,17 +117,18 @@ RB_API rb_status rb_pack(const float *W, const float *g, const float *h,
 
 /*
  * rb_gemv -- decode-time Y = sum_i g_i .* (B_i (h_i .* X)) for 1 <= M <= 64
- * tokens (tuned for M = 1; RaBiT "matmul-free" evaluation, additions and
- * element-wise scaling only).
+ * tokens (RaBiT, "Residual binarization": the k binary paths run side by side
+ * and are summed after the element-wise scaling).
  *   X   [M][K] bfloat16 bit patterns.
  *   Y   [M][N] fp32 or bfloat16 (y_dtype), written, never read.
- *   workspace: rb_gemv_workspace_bytes(N, K, k, M) bytes of device memory
- *   (0 when the call needs none).  It holds per-slice fp32 partial sums and
- *   per-row-tile arrival counters; it must be zero-filled before its first
- *   use, and every call returns the counters to zero, so later calls need no
- *   clearing.  Calls that share a workspace must not overlap on the GPU
- *   (same stream, with or without RB_LAUNCH_PDL, is fine).
- * h_i .* x is formed exactly in fp32 and every sum is accumulated in fp32.
+ *   workspace: rb_gemv_workspace_bytes(...) returns 0; every path keeps its
+ *   partial sums on chip, and the workspace arguments are ignored.
+ * M = 1 and k <= 4: byte tables; h_i .* x is formed exactly in fp32 and every
+ * sum is accumulated in fp32 (CUDA cores, additions only).
+ * Otherwise: tensor cores (mma.sync, fp16 operands, fp32 accumulation).  The
+ * +-h_i operands are exact in fp16 and X is converted to fp16 (exact for bf16
+ * values of magnitude 2^-14 .. 65504; smaller ones lose low bits, larger ones
+ * overflow), so every product is exact and only the accumulation rounds.
  */
 RB_API size_t rb_gemv_workspace_bytes(int n_out, int k_in, int k_planes, int M);
 RB_API rb_status rb_gemv(const rb_layer_t *layer, const uint16_t *X, int M,

@@ -18,9 +18,9 @@
 // deterministic and no global workspace is needed.  Weights, g and h are
 // fetched before the programmatic-dependent-launch wait; only X after it.
 //
-// Any M <= 64, any k <= 8: generic CUDA-core kernel (lane = row, one signed
-// fused add per bit and token); it keeps every plane and token block in
-// registers and needs no workspace.
+// M >= 2 (up to 64), and M = 1 with k > 4: tensor-core kernel (mma.sync,
+// fp16 operands, fp32 accumulation) with the sign words expanded to +-h in
+// registers; see gemv_mma_kernel.
 #include "rbw_internal.cuh"
 
 #include <mutex>
@@ -420,70 +420,243 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
     }
 }
 
-// ---------------------------------------------------------------- generic kernel
-constexpr int kGenThreads = 128;       // 4 warps = 4 row tiles
-constexpr int kGenMT = 4;              // tokens per CTA
+// ---------------------------------------------------------------- tensor-core decode kernel
+// M >= 2 (up to 64), and M = 1 with k > 4.  mma.sync m16n8k16, fp16 operands,
+// fp32 accumulation: A = the signed scales +-h_i expanded from the sign words in
+// registers, B = the activations converted to fp16, D = one accumulator per
+// plane; Y = sum_i g_i * D_i.  Products of two fp16 values are exact in fp32.
+//
+// K order inside a 32-column word: MMA k index 2j + e is column j + 16e (the
+// order of the h pairs (h[j], h[j+16])), so one shift brings sign bits j and
+// j+16 to the sign positions of an fp16 pair and one LOP3 applies them; the
+// staged activations use the same order.
+//
+// Grid: per layer, row groups of 8 tiles (one 32-row tile per warp) x CS CTAs
+// along K (a cluster; rank j takes the contiguous slices [j*spc, (j+1)*spc)) x
+// token groups of 8*NT tokens (grid.y).  Partial sums of a row group go over
+// distributed shared memory to the rank that owns the row and are added there
+// in rank order (deterministic, no workspace).
+constexpr int kMmaWarps = 8;
+constexpr int kMmaThreads = kMmaWarps * 32;
+constexpr int kMmaRows = kMmaWarps * 32;        // rows per CTA
 
-template <int KP>
-__global__ void __launch_bounds__(kGenThreads)
-gemv_generic_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ g16,
-                    const uint16_t* __restrict__ h16, const uint16_t* __restrict__ X,
-                    int N, int K, int M, void* __restrict__ Y, int ydt)
+__host__ __device__ constexpr int mma_xs(int spc) { return spc * 256 + 8; }   // halves per staged token row
+__host__ __device__ inline int mma_smem_bytes(int kp, int nt, int spc, int CS)
 {
-    __shared__ float hx[KP][kGenMT][8][33];
+    const int x = 8 * nt * mma_xs(spc) * 2;                  // staged X, fp16
+    const int hq = kp * spc * 8 * 4 * 16;                    // h pairs, 16 B per (plane, word, t)
+    const int recv = CS > 1 ? kMmaRows * 8 * nt * 4 : 0;     // partial sums received from the cluster
+    return (x + 15) / 16 * 16 + hq + recv;
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// (~shifted & 0x80008000) ^ hpair: a clear sign bit turns +h into -h.
+__device__ __forceinline__ uint32_t sign_pair(uint32_t shifted, uint32_t hpair)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xA6;" : "=r"(d) : "r"(shifted), "r"(0x80008000u), "r"(hpair));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t bf16_to_f16_bits(uint16_t v)
+{
+    return (uint32_t)__half_as_ushort(__float2half_rn(bf16_bits_to_f32(v)));
+}
+
+// The 8 logical words of plane i, slice s, tile T for row `lane` (zero past the tiles).
+template <int KP>
+__device__ __forceinline__ void mma_load_words(uint32_t (&w)[KP][8], const uint32_t* __restrict__ planes,
+                                               int64_t s, int64_t T, int64_t S, int64_t Nt, int lane)
+{
+#pragma unroll
+    for (int i = 0; i < KP; ++i) {
+        const uint32_t* blk = planes + block_index(i, s, T, S, Nt) * 256 + lane;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) w[i][q] = T < Nt ? __ldcs(blk + ((q ^ (lane >> 2)) * 32)) : 0u;
+    }
+}
+
+template <int KP, int NT>
+__global__ void __launch_bounds__(kMmaThreads, 1)
+gemv_mma_kernel(const __grid_constant__ LutBatch batch, int N, int K, int M, int CS, int groups, int ydt)
+{
+    constexpr int TG = 8 * NT;
+    extern __shared__ __align__(16) uint8_t msm[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
     const int64_t S = num_slices(K), Nt = num_row_tiles(N);
-    const int64_t t = (int64_t)blockIdx.x * (kGenThreads / 32) + warp;
-    const int m0 = blockIdx.y * kGenMT;
+    const int rank = CS > 1 ? (int)cluster_rank() : 0;
+    const int cl = blockIdx.x / CS;
+    const int layer = cl / groups, grp = cl % groups;
+    const uint32_t* __restrict__ planes = batch.planes[layer];
+    const uint16_t* __restrict__ g16 = batch.g16[layer];
+    const uint16_t* __restrict__ h16 = batch.h16[layer];
+    const uint16_t* __restrict__ X = batch.X[layer];
+    void* __restrict__ Y = batch.Y[layer];
+    const int spc = (int)((S + CS - 1) / CS);
+    const int64_t s0 = (int64_t)rank * spc;
+    const int nsl = (int)(s0 < S ? (S - s0 < spc ? S - s0 : spc) : 0);
+    const int m0 = blockIdx.y * TG;
+    const int XS = mma_xs(spc);
+    uint16_t* xs = reinterpret_cast<uint16_t*>(msm);                                  // [TG][XS]
+    uint4* hq = reinterpret_cast<uint4*>(msm + (TG * XS * 2 + 15) / 16 * 16);         // [KP][spc*8][4]
+    float* recv = reinterpret_cast<float*>(hq + KP * spc * 8 * 4);                     // [CS][rows/CS][TG]
+    const int64_t T = (int64_t)grp * kMmaWarps + warp;                               // this warp's tile
+
+    // ---- before the dependency wait: the first slice's sign words and the h pairs
+    uint32_t cw[KP][8];
+    if (nsl > 0) mma_load_words<KP>(cw, planes, s0, T, S, Nt, lane);
+    for (int idx = threadIdx.x; idx < KP * nsl * 32; idx += kMmaThreads) {
+        const int i = idx / (nsl * 32), wl = (idx / 4) % (nsl * 8), tt = idx & 3;
+        const int64_t c0 = s0 * 256 + 32 * wl;
+        uint32_t pr[4] = {0u, 0u, 0u, 0u};
+        if (c0 < K) {
+            const uint16_t* hb = h16 + (int64_t)i * K + c0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) pr[q] = (uint32_t)hb[tt + 4 * q] | ((uint32_t)hb[tt + 4 * q + 16] << 16);
+        }
+        hq[(i * spc * 8 + wl) * 4 + tt] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+    }
     pdl_launch_dependents();
     pdl_wait();
+    // ---- activations of the CTA's columns, fp16, pair order (j, j+16) per word
+    for (int idx = threadIdx.x; idx < TG * nsl * 128; idx += kMmaThreads) {
+        const int m = idx / (nsl * 128), rem = idx % (nsl * 128), wl = rem >> 4, j = rem & 15;
+        const int64_t c0 = s0 * 256 + 32 * wl + j;
+        uint32_t v = 0u;
+        if (m0 + m < M && c0 < K) {
+            const uint16_t* xr = X + (int64_t)(m0 + m) * K + c0;
+            v = bf16_to_f16_bits(xr[0]) | (bf16_to_f16_bits(xr[16]) << 16);
+        }
+        *reinterpret_cast<uint32_t*>(xs + m * XS + 32 * wl + 2 * j) = v;
+    }
+    __syncthreads();
 
-    float acc[KP][kGenMT];
+    float acc[KP][2][NT][4];
 #pragma unroll
     for (int i = 0; i < KP; ++i)
 #pragma unroll
-        for (int m = 0; m < kGenMT; ++m) acc[i][m] = 0.0f;
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[i][hf][nt][q] = 0.0f;
 
-    for (int64_t s = 0; s < S; ++s) {
-        for (int idx = threadIdx.x; idx < KP * kGenMT * 256; idx += kGenThreads) {
-            const int cc = idx & 255, m = (idx >> 8) % kGenMT, i = idx / (256 * kGenMT);
-            const int64_t c = s * 256 + cc;
-            float v = 0.0f;
-            if (c < K && m0 + m < M)
-                v = __half2float(__ushort_as_half(h16[(int64_t)i * K + c])) *
-                    bf16_bits_to_f32(X[(int64_t)(m0 + m) * K + c]);
-            hx[i][m][cc >> 5][cc & 31] = v;
-        }
-        __syncthreads();
-        if (t < Nt) {
+    const uint16_t* xg = xs + g * XS + 2 * t;       // this thread's token row g, k pair 2t
+    for (int sl = 0; sl < nsl; ++sl) {
+        uint32_t nw[KP][8];
+        if (sl + 1 < nsl) mma_load_words<KP>(nw, planes, s0 + sl + 1, T, S, Nt, lane);
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            const int wl = sl * 8 + w;
+            uint32_t b[2][NT][2];
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint16_t* xp = xg + nt * 8 * XS + 32 * wl + 16 * ks;
+                    b[ks][nt][0] = *reinterpret_cast<const uint32_t*>(xp);
+                    b[ks][nt][1] = *reinterpret_cast<const uint32_t*>(xp + 8);
+                }
 #pragma unroll
             for (int i = 0; i < KP; ++i) {
-                const uint32_t* blk = planes + block_index(i, s, t, S, Nt) * 256 + lane;
-                for (int sl = 0; sl < 8; ++sl) {
-                    const uint32_t word = blk[sl * 32];
-                    const int wl = sl ^ (lane >> 2);
-#pragma unroll 8
-                    for (int j = 0; j < 32; ++j) {
-                        const float sg = ((word >> j) & 1u) ? 1.0f : -1.0f;
+                const uint4 hv = hq[(i * spc * 8 + wl) * 4 + t];      // pairs j = t, t+4, t+8, t+12
 #pragma unroll
-                        for (int m = 0; m < kGenMT; ++m) acc[i][m] = fmaf(sg, hx[i][m][wl][j], acc[i][m]);
+                for (int hf = 0; hf < 2; ++hf) {
+                    const uint32_t wa = __shfl_sync(0xffffffffu, cw[i][w], 16 * hf + g);
+                    const uint32_t wb = __shfl_sync(0xffffffffu, cw[i][w], 16 * hf + g + 8);
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const int j0 = 8 * ks + t;
+                        const uint32_t h0 = ks ? hv.z : hv.x, h1 = ks ? hv.w : hv.y;
+                        const uint32_t a0 = sign_pair(wa << (15 - j0), h0), a1 = sign_pair(wb << (15 - j0), h0);
+                        const uint32_t a2 = sign_pair(wa << (11 - j0), h1), a3 = sign_pair(wb << (11 - j0), h1);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+                            mma_16816(acc[i][hf][nt], a0, a1, a2, a3, b[ks][nt][0], b[ks][nt][1]);
                     }
                 }
             }
         }
-        __syncthreads();
-    }
-    const int64_t r = t * 32 + lane;
-    if (t < Nt && r < N) {
-#pragma unroll
-        for (int m = 0; m < kGenMT; ++m) {
-            if (m0 + m >= M) break;
-            float y = 0.0f;
+        if (sl + 1 < nsl) {
 #pragma unroll
             for (int i = 0; i < KP; ++i)
-                y += __half2float(__ushort_as_half(g16[(int64_t)i * N + r])) * acc[i][m];
-            store_y(Y, ydt, (int64_t)(m0 + m) * N + r, y);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) cw[i][q] = nw[i][q];
         }
+    }
+
+    // ---- y[row][token] = sum_i g_i[row] * acc_i; thread rows 16hf + g + 8e, tokens 8nt + 2t + q
+    float y[2][2][NT][2];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int64_t r = T * 32 + 16 * hf + g + 8 * e;
+            float gi[KP];
+#pragma unroll
+            for (int i = 0; i < KP; ++i)
+                gi[i] = r < N ? __half2float(__ushort_as_half(g16[(int64_t)i * N + r])) : 0.0f;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    float v = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < KP; ++i) v += gi[i] * acc[i][hf][nt][2 * e + q];
+                    y[hf][e][nt][q] = v;
+                }
+        }
+    if (CS == 1) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int64_t r = T * 32 + 16 * hf + g + 8 * e;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int m = m0 + 8 * nt + 2 * t + q;
+                        if (r < N && m < M) store_y(Y, ydt, (int64_t)m * N + r, y[hf][e][nt][q]);
+                    }
+            }
+        return;
+    }
+    // Rows [j*RPO, (j+1)*RPO) of the CTA's 256 belong to rank j; slot (source rank, row, token).
+    const int RPO = kMmaRows / CS;
+    const uint32_t recv_s = smem_u32(recv);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int cr = warp * 32 + 16 * hf + g + 8 * e;
+            const int owner = cr / RPO, lr = cr - owner * RPO;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int tok = 8 * nt + 2 * t + q;
+                    st_dsmem_f32(recv_s + (uint32_t)(((rank * RPO + lr) * TG + tok) * 4), (uint32_t)owner,
+                                 y[hf][e][nt][q]);
+                }
+        }
+    cluster_sync_all();
+    for (int idx = threadIdx.x; idx < RPO * TG; idx += kMmaThreads) {
+        const int tok = idx / RPO, lr = idx % RPO;
+        float v = 0.0f;
+        for (int j = 0; j < CS; ++j) v += recv[(j * RPO + lr) * TG + tok];
+        const int64_t r = (int64_t)grp * kMmaRows + rank * RPO + lr;
+        const int m = m0 + tok;
+        if (r < N && m < M) store_y(Y, ydt, (int64_t)m * N + r, v);
     }
 }
 
@@ -691,14 +864,87 @@ rb_status launch_lut(const rb_layer_t* const* layers, const uint16_t* const* X, 
     return RB_OK;
 }
 
-template <int KP>
-rb_status launch_generic(const rb_layer_t* L, const uint16_t* X, int M, void* Y, int ydt,
-                         bool pdl, cudaStream_t stream)
+// Tensor-core decode: tokens per group 8*NT with k*NT <= 8 (accumulator
+// registers); CS = the smallest power of two that fits the staged activations
+// (at most 96 KB) and gives about two CTAs per SM, at most min(16, S).
+template <int KP, int NT>
+rb_status launch_mma_nt(const LutBatch& b, int n, int N, int K, int M, int ydt, bool pdl, cudaStream_t stream)
 {
-    const int64_t Nt = num_row_tiles(L->n_out);
-    dim3 grid((unsigned)((Nt + 3) / 4), (unsigned)((M + kGenMT - 1) / kGenMT));
-    return launch(gemv_generic_kernel<KP>, grid, dim3(kGenThreads), 0, stream, pdl,
-                  L->planes, L->g16, L->h16, X, L->n_out, L->k_in, M, Y, ydt);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RB_ERR_CUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(gemv_mma_kernel<KP, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 227 * 1024) != cudaSuccess ||
+            cudaFuncSetAttribute(gemv_mma_kernel<KP, NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess)
+            return RB_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    const int64_t S = num_slices(K), Nt = num_row_tiles(N);
+    const int groups = (int)((Nt + kMmaWarps - 1) / kMmaWarps);
+    const int tgroups = (M + 8 * NT - 1) / (8 * NT);
+    const int64_t want = 2LL * num_sms();
+    int CS = 1;
+    while (CS < 16 && CS < S &&
+           (8 * NT * mma_xs((int)((S + CS - 1) / CS)) * 2 > 96 * 1024 || (int64_t)n * groups * tgroups * CS < want))
+        CS *= 2;
+    const int spc = (int)((S + CS - 1) / CS);
+    const int smem = mma_smem_bytes(KP, NT, spc, CS);
+    if (smem > 227 * 1024) return RB_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(n * groups * CS), (unsigned)tgroups);
+    cfg.blockDim = dim3(kMmaThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (CS > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)CS;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    if (cudaLaunchKernelEx(&cfg, gemv_mma_kernel<KP, NT>, b, N, K, M, CS, groups, ydt) != cudaSuccess)
+        return RB_ERR_CUDA;
+    return RB_OK;
+}
+
+template <int KP>
+rb_status launch_mma(const rb_layer_t* const* layers, const uint16_t* const* X, void* const* Y, int count, int M,
+                     int ydt, bool pdl, cudaStream_t stream)
+{
+    constexpr int NTMAX = KP <= 2 ? 4 : (KP <= 4 ? 2 : 1);
+    const rb_layer_t* L0 = layers[0];
+    for (int base = 0; base < count; base += kMaxBatch) {
+        const int n = count - base < kMaxBatch ? count - base : kMaxBatch;
+        LutBatch b = {};
+        for (int j = 0; j < n; ++j) {
+            b.planes[j] = layers[base + j]->planes;
+            b.g16[j] = layers[base + j]->g16;
+            b.h16[j] = layers[base + j]->h16;
+            b.X[j] = X[base + j];
+            b.Y[j] = Y[base + j];
+        }
+        const int need = (M + 7) / 8;                 // n-tiles for all tokens in one group
+        rb_status st;
+        if (need >= 4 && NTMAX >= 4)
+            st = launch_mma_nt<KP, (NTMAX >= 4 ? 4 : 1)>(b, n, L0->n_out, L0->k_in, M, ydt, pdl, stream);
+        else if (need >= 2 && NTMAX >= 2)
+            st = launch_mma_nt<KP, (NTMAX >= 2 ? 2 : 1)>(b, n, L0->n_out, L0->k_in, M, ydt, pdl, stream);
+        else
+            st = launch_mma_nt<KP, 1>(b, n, L0->n_out, L0->k_in, M, ydt, pdl, stream);
+        if (st != RB_OK) return st;
+    }
+    return RB_OK;
 }
 
 bool use_lut(const rb_layer_t* L, int M) { return M == 1 && L->k_planes <= 4; }
@@ -736,21 +982,16 @@ static rb_status gemv_dispatch(const rb_layer_t* const* layers, const uint16_t* 
             default: return launch_lut<4>(layers, X, Y, count, ydt, pdl, stream);
         }
     }
-    for (int j = 0; j < count; ++j) {
-        rb_status st;
-        switch (L0->k_planes) {
-            case 1: st = launch_generic<1>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
-            case 2: st = launch_generic<2>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
-            case 3: st = launch_generic<3>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
-            case 4: st = launch_generic<4>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
-            case 5: st = launch_generic<5>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
-            case 6: st = launch_generic<6>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
-            case 7: st = launch_generic<7>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
-            default: st = launch_generic<8>(layers[j], X[j], M, Y[j], ydt, pdl, stream); break;
-        }
-        if (st != RB_OK) return st;
+    switch (L0->k_planes) {
+        case 1: return launch_mma<1>(layers, X, Y, count, M, ydt, pdl, stream);
+        case 2: return launch_mma<2>(layers, X, Y, count, M, ydt, pdl, stream);
+        case 3: return launch_mma<3>(layers, X, Y, count, M, ydt, pdl, stream);
+        case 4: return launch_mma<4>(layers, X, Y, count, M, ydt, pdl, stream);
+        case 5: return launch_mma<5>(layers, X, Y, count, M, ydt, pdl, stream);
+        case 6: return launch_mma<6>(layers, X, Y, count, M, ydt, pdl, stream);
+        case 7: return launch_mma<7>(layers, X, Y, count, M, ydt, pdl, stream);
+        default: return launch_mma<8>(layers, X, Y, count, M, ydt, pdl, stream);
     }
-    return RB_OK;
 }
 
 extern "C" rb_status rb_gemv(const rb_layer_t* layer, const uint16_t* X, int M, void* Y,
