@@ -466,11 +466,6 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t shifted, uint32_t hpair)
     return d;
 }
 
-__device__ __forceinline__ uint32_t bf16_to_f16_bits(uint16_t v)
-{
-    return (uint32_t)__half_as_ushort(__float2half_rn(bf16_bits_to_f32(v)));
-}
-
 // The 8 logical words of plane i, slice s, tile T for row `lane` (zero past the tiles).
 template <int KP>
 __device__ __forceinline__ void mma_load_words(uint32_t (&w)[KP][8], const uint32_t* __restrict__ planes,
@@ -514,29 +509,59 @@ gemv_mma_kernel(const __grid_constant__ LutBatch batch, int N, int K, int M, int
     // ---- before the dependency wait: the first slice's sign words and the h pairs
     uint32_t cw[KP][8];
     if (nsl > 0) mma_load_words<KP>(cw, planes, s0, T, S, Nt, lane);
-    for (int idx = threadIdx.x; idx < KP * nsl * 32; idx += kMmaThreads) {
-        const int i = idx / (nsl * 32), wl = (idx / 4) % (nsl * 8), tt = idx & 3;
+    // one (plane, word) per item: 64 B of h, 16 pairs (h[j], h[j+16]), four 16 B entries
+    for (int idx = threadIdx.x; idx < KP * nsl * 8; idx += kMmaThreads) {
+        const int i = idx / (nsl * 8), wl = idx % (nsl * 8);
         const int64_t c0 = s0 * 256 + 32 * wl;
-        uint32_t pr[4] = {0u, 0u, 0u, 0u};
+        uint32_t hw[16];                              // h[c0 + 2e], h[c0 + 2e + 1] in word e
         if (c0 < K) {
-            const uint16_t* hb = h16 + (int64_t)i * K + c0;
+            const uint4* hb = reinterpret_cast<const uint4*>(h16 + (int64_t)i * K + c0);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) pr[q] = (uint32_t)hb[tt + 4 * q] | ((uint32_t)hb[tt + 4 * q + 16] << 16);
+            for (int q = 0; q < 4; ++q) {
+                const uint4 v = hb[q];
+                hw[4 * q] = v.x; hw[4 * q + 1] = v.y; hw[4 * q + 2] = v.z; hw[4 * q + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) hw[e] = 0u;
         }
-        hq[(i * spc * 8 + wl) * 4 + tt] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+        uint4* dst = hq + (i * spc * 8 + wl) * 4;
+#pragma unroll
+        for (int tt = 0; tt < 4; ++tt) {
+            uint32_t pr[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int j = tt + 4 * q;             // pair (h[j], h[j+16])
+                pr[q] = prmt(hw[j >> 1], hw[(j + 16) >> 1], (j & 1) ? 0x7632u : 0x5410u);
+            }
+            dst[tt] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+        }
     }
     pdl_launch_dependents();
     pdl_wait();
-    // ---- activations of the CTA's columns, fp16, pair order (j, j+16) per word
-    for (int idx = threadIdx.x; idx < TG * nsl * 128; idx += kMmaThreads) {
-        const int m = idx / (nsl * 128), rem = idx % (nsl * 128), wl = rem >> 4, j = rem & 15;
-        const int64_t c0 = s0 * 256 + 32 * wl + j;
-        uint32_t v = 0u;
+    // ---- activations of the CTA's columns, fp16, pair order (j, j+16) per word;
+    // one item = token m, word wl, half q: pairs j = 8q .. 8q+7 from two 16 B loads
+    for (int idx = threadIdx.x; idx < TG * nsl * 16; idx += kMmaThreads) {
+        const int m = idx / (nsl * 16), rem = idx % (nsl * 16), wl = rem >> 1, q = rem & 1;
+        const int64_t c0 = s0 * 256 + 32 * wl + 8 * q;
+        uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
         if (m0 + m < M && c0 < K) {
             const uint16_t* xr = X + (int64_t)(m0 + m) * K + c0;
-            v = bf16_to_f16_bits(xr[0]) | (bf16_to_f16_bits(xr[16]) << 16);
+            lo = *reinterpret_cast<const uint4*>(xr);          // columns 8q .. 8q+7 of the word
+            hi = *reinterpret_cast<const uint4*>(xr + 16);     // columns 16+8q .. 16+8q+7
         }
-        *reinterpret_cast<uint32_t*>(xs + m * XS + 32 * wl + 2 * j) = v;
+        const uint32_t lw[4] = {lo.x, lo.y, lo.z, lo.w}, hw[4] = {hi.x, hi.y, hi.z, hi.w};
+        uint32_t pr[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t a = (e & 1) ? (lw[e >> 1] & 0xffff0000u) : (lw[e >> 1] << 16);
+            const uint32_t b = (e & 1) ? (hw[e >> 1] & 0xffff0000u) : (hw[e >> 1] << 16);
+            const __half2 h2 = __floats2half2_rn(__uint_as_float(a), __uint_as_float(b));
+            pr[e] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(xs + m * XS + 32 * wl + 16 * q);
+        dst[0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+        dst[1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
     }
     __syncthreads();
 
