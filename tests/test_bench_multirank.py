@@ -1,0 +1,64 @@
+"""Host logic of bench.py's multi-rank path on CPU: two gloo ranks, the
+max-over-ranks step time, the whole-job throughput, the reference arm that
+runs on rank 0 only, and the keys of the JSON line."""
+import json
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_path):
+    os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    d = bench.Dist()
+    d.init("gloo")
+    d.barrier()
+    t_local = 1.0 + 0.5 * rank                 # rank 1 is the slow one
+    t_max = d.max(t_local)
+    value = bench.throughput(1e9, d.world, 10, t_max)
+    d.barrier()
+    if d.rank == 0:
+        with open(out_path, "w") as f:
+            json.dump({"t_max": t_max, "value": value, "world": d.world}, f)
+    d.close()
+
+
+def test_two_gloo_ranks_take_the_max_time(tmp_path):
+    out = str(tmp_path / "r0.json")
+    mp.start_processes(_rank_main, args=(2, _free_port(), out), nprocs=2, join=True, start_method="spawn")
+    r = json.load(open(out))
+    assert r["world"] == 2
+    assert r["t_max"] == pytest.approx(1.5)
+    # whole-job GB/s: both ranks' bytes over the slowest rank's time
+    assert r["value"] == pytest.approx(1e9 * 2 * 10 / 1.5 / 1e9)
+
+
+class _FakeDist:
+    def __init__(self, rank, world):
+        self.rank, self.world, self.pg = rank, world, False
+
+
+def test_reference_arm_runs_on_rank0_only(capsys):
+    ns = type("A", (), {"steps": 1, "warmup": 0, "gpus": 2})()
+    assert bench.run_reference(ns, _FakeDist(1, 2)) == 0
+    assert capsys.readouterr().out == ""          # a non-zero rank does no work and prints nothing
+
+
+def test_json_line_carries_the_contract_keys():
+    line = bench.assemble_line(value=1.0, unit="GB/s", n_gpus=2, steps=3, warmup=3, ms_per_step=1.0,
+                               extra={"config": bench.config_dict()})
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config"):
+        assert k in line
+    assert line["scaling"] == "weak" and line["higher_is_better"] is True
+    assert line["config"]["workload"] == bench.WORKLOAD
