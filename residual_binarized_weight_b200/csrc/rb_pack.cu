@@ -22,6 +22,43 @@ namespace {
 
 constexpr int kPackThreads = 256;
 
+template <int KP, bool FULL>
+__device__ __forceinline__ void pack_item(const float* __restrict__ W, const float* __restrict__ g,
+                                          const float* __restrict__ h, int N, int K, int t, int c,
+                                          int lane, uint32_t (&mine)[KP], int& bad)
+{
+    float hv[KP], gv[KP];
+    const int my_row = t * 32 + lane;
+#pragma unroll
+    for (int i = 0; i < KP; ++i) {
+        hv[i] = h[(int64_t)i * K + c];
+        gv[i] = (FULL || my_row < N) ? g[(int64_t)i * N + my_row] : 0.0f;
+    }
+    // all 32 row segments in flight at once (4 KB per warp) before any arithmetic
+    const float* p = W + (int64_t)t * 32 * K + c;
+    float wv[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) wv[j] = (FULL || t * 32 + j < N) ? __ldcs(p + (int64_t)j * K) : 0.0f;
+    float nonfinite = 0.0f;                   // stays 0 unless some W is NaN or +-inf
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        float R = wv[j];
+        nonfinite = fmaf(R, 0.0f, nonfinite);
+#pragma unroll
+        for (int i = 0; i < KP; ++i) {
+            const float gi = __shfl_sync(0xffffffffu, gv[i], j);
+            const float tt = __fmul_rn(gi, hv[i]);
+            const bool b = R >= 0.0f;                   // sign(0) = +1, -0.0 too
+            R = __fadd_rn(R, b ? -tt : tt);             // R - t or R + t, one rounding
+            const uint32_t word = __ballot_sync(0xffffffffu, b);
+            mine[i] = lane == j ? word : mine[i];
+        }
+    }
+    bad |= nonfinite != 0.0f;
+}
+
+// Items are (row tile t, slice s, word w), numbered t-major so that the warps
+// of a CTA stream neighbouring columns of the same rows; 32-bit index math.
 template <int KP>
 __global__ void __launch_bounds__(kPackThreads, 2)
 pack_kernel(const float* __restrict__ W, const float* __restrict__ g,
@@ -29,62 +66,43 @@ pack_kernel(const float* __restrict__ W, const float* __restrict__ g,
             uint32_t* __restrict__ planes, int32_t* dev_status)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t S = num_slices(K), Nt = num_row_tiles(N);
-    const int64_t items = Nt * S * 8;
-    const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int S = (int)num_slices(K), Nt = (int)num_row_tiles(N);
+    const int words = K / 32;                     // valid words per row
+    const int items = Nt * words;
+    const int gwarp = (int)((blockIdx.x * (unsigned)blockDim.x + threadIdx.x) >> 5);
+    const int nwarps = (int)((gridDim.x * (unsigned)blockDim.x) >> 5);
+    const int full_tiles = N / 32;
     int bad = 0;
 
-    for (int64_t it = gwarp; it < items; it += nwarps) {
-        const int w = (int)(it & 7);              // logical word within the slice
-        const int64_t s = (it >> 3) % S;
-        const int64_t t = (it >> 3) / S;
-        const int64_t col0 = s * 256 + (int64_t)w * 32;
-        const int64_t c = col0 + lane;
+    for (int it = gwarp; it < items; it += nwarps) {
+        const int t = it / words, wg = it - t * words;      // word wg of the row = slice wg/8, word wg%8
+        const int c = wg * 32 + lane;
         uint32_t mine[KP];
 #pragma unroll
         for (int i = 0; i < KP; ++i) mine[i] = 0u;
-
-        if (col0 < K) {                           // K % 32 == 0: whole word valid
-            float hv[KP], gv[KP];
-            const int64_t my_row = t * 32 + lane;
-#pragma unroll
-            for (int i = 0; i < KP; ++i) {
-                hv[i] = h[(int64_t)i * K + c];
-                gv[i] = my_row < N ? g[(int64_t)i * N + my_row] : 0.0f;
-            }
-            // all 32 row segments in flight at once (4 KB per warp) before any arithmetic
-            float wv[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int64_t r = t * 32 + j;
-                wv[j] = r < N ? __ldcs(W + r * K + c) : 0.0f;
-            }
-            float nonfinite = 0.0f;               // stays 0 unless some W is NaN or +-inf
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                float R = wv[j];
-                nonfinite = fmaf(R, 0.0f, nonfinite);
-                const bool mine_row = lane == j;
-#pragma unroll
-                for (int i = 0; i < KP; ++i) {
-                    const float gi = __shfl_sync(0xffffffffu, gv[i], j);
-                    const float tt = __fmul_rn(gi, hv[i]);
-                    const bool b = R >= 0.0f;               // sign(0) = +1, -0.0 too
-                    R = __fadd_rn(R, b ? -tt : tt);         // R - t or R + t, one rounding
-                    const uint32_t word = __ballot_sync(0xffffffffu, b);
-                    if (mine_row) mine[i] = word;
-                }
-            }
-            bad |= nonfinite != 0.0f;
+        if (t < full_tiles) {
+            pack_item<KP, true>(W, g, h, N, K, t, c, lane, mine, bad);
+        } else {
+            pack_item<KP, false>(W, g, h, N, K, t, c, lane, mine, bad);
             if (t * 32 + lane >= N) {
 #pragma unroll
                 for (int i = 0; i < KP; ++i) mine[i] = 0u;   // padding rows of the last tile
             }
         }
+        const int s = wg >> 3, w = wg & 7;
 #pragma unroll
         for (int i = 0; i < KP; ++i)
             planes[word_offset(i, s, t * 32 + lane, w, S, Nt)] = mine[i];
+    }
+    // padding words of a ragged last slice (K % 256 != 0) stay zero
+    const int pad_words = S * 8 - words;
+    if (pad_words > 0) {
+        for (int it = gwarp; it < Nt * pad_words; it += nwarps) {
+            const int t = it / pad_words, wg = words + (it - t * pad_words);
+#pragma unroll
+            for (int i = 0; i < KP; ++i)
+                planes[word_offset(i, wg >> 3, t * 32 + lane, wg & 7, S, Nt)] = 0u;
+        }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_dev_status(dev_status, RB_DEV_NONFINITE);
 }
@@ -113,6 +131,7 @@ rb_status launch_pack(const float* W, const float* g, const float* h, int N, int
                       uint32_t* planes, int32_t* dev_status, cudaStream_t stream)
 {
     const int64_t items = num_row_tiles(N) * num_slices(K) * 8;
+    if (items > INT32_MAX / 2) return RB_ERR_UNSUPPORTED;          // 32-bit item numbering
     const int64_t warps_per_cta = kPackThreads / 32;
     int64_t ctas = (items + warps_per_cta - 1) / warps_per_cta;
     const int64_t cap = (int64_t)num_sms() * 8;
