@@ -121,14 +121,20 @@ RB_API rb_status rb_pack(const float *W, const float *g, const float *h,
  * and are summed after the element-wise scaling).
  *   X   [M][K] bfloat16 bit patterns.
  *   Y   [M][N] fp32 or bfloat16 (y_dtype), written, never read.
- *   workspace: rb_gemv_workspace_bytes(...) returns 0; every path keeps its
- *   partial sums on chip, and the workspace arguments are ignored.
+ *   workspace: rb_gemv_workspace_bytes(N, K, k, M) bytes of 16-byte aligned
+ *   device memory (0 when no path needs one; then NULL is fine).  It holds X
+ *   converted to fp16 and the h pairs for the tcgen05 path; no clearing needed.
+ *   Calls that share a workspace must not overlap on the GPU.
  * M = 1 and k <= 4: byte tables; h_i .* x is formed exactly in fp32 and every
  * sum is accumulated in fp32 (CUDA cores, additions only).
- * Otherwise: tensor cores (mma.sync, fp16 operands, fp32 accumulation).  The
- * +-h_i operands are exact in fp16 and X is converted to fp16 (exact for bf16
- * values of magnitude 2^-14 .. 65504; smaller ones lose low bits, larger ones
- * overflow), so every product is exact and only the accumulation rounds.
+ * M >= 32 and k <= 4 with the workspace: the tcgen05 kernel of rb_gemm with
+ * 16/32/64-token tiles and K split over a thread-block cluster.
+ * Otherwise (no workspace, or k > 4): mma.sync kernel.  Both tensor-core paths
+ * use fp16 operands with fp32 accumulation: the +-h_i operands are exact in
+ * fp16 and X is converted to fp16 (exact for bf16 values of magnitude
+ * 2^-14 .. 65504; smaller ones lose low bits, larger ones overflow; the
+ * tcgen05 path flags |x| >= 65520 with RB_DEV_RANGE), so every product is
+ * exact and only the accumulation rounds.
  */
 RB_API size_t rb_gemv_workspace_bytes(int n_out, int k_in, int k_planes, int M);
 RB_API rb_status rb_gemv(const rb_layer_t *layer, const uint16_t *X, int M,

@@ -130,6 +130,14 @@ __device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[3
                  : "r"(taddr) : "memory");
 }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+                   "=r"(v[14]), "=r"(v[15])
+                 : "r"(taddr));
+}
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ uint32_t lop3_sign(uint32_t shifted, uint32_t hpair) {
     // (~shifted & 0x80008000) ^ hpair : a clear sign bit flips +h to -h
@@ -152,9 +160,6 @@ __host__ __device__ constexpr uint32_t idesc_f16(int bt) {
 
 __host__ __device__ constexpr int gemm_bt(int kp) { return kp <= 2 ? 128 : 64; }
 __host__ __device__ constexpr int gemm_sa(int kp) { return kp <= 2 ? 4 : 2; }
-__host__ __device__ constexpr int gemm_tmem_cols(int kp) {
-    return (kp * gemm_bt(kp) + gemm_sa(kp) * kp * 32) <= 256 ? 256 : 512;
-}
 // With three or more planes the expansion warps are the bottleneck and read the
 // h pairs of the whole layer from shared memory (one bulk copy per CTA) with the
 // sign words a slice ahead; with one or two planes the k-block-ahead loads from
@@ -164,8 +169,9 @@ __host__ __device__ constexpr bool gemm_hp_in_smem(int kp) { return kp >= 3; }
 __host__ __device__ inline int gemm_hp_bytes(int kp, int K) {
     return gemm_hp_in_smem(kp) ? ((kp * (K / 2) * 4) + 127) / 128 * 128 : 0;
 }
-__host__ __device__ inline int gemm_smem_bytes(int kp, int K, int nsx) {
-    return nsx * gemm_bt(kp) * 128 + gemm_hp_bytes(kp, K) + 1024 + 256;
+// ks > 1 adds the receive area of the cluster reduction (128 rows x bt tokens fp32).
+__host__ __device__ inline int gemm_smem_bytes(int kp, int bt, int K, int nsx, int ks) {
+    return nsx * bt * 128 + gemm_hp_bytes(kp, K) + 1024 + 256 + (ks > 1 ? ks * ((kBR + ks - 1) / ks) * bt * 4 : 0);
 }
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
@@ -219,14 +225,19 @@ __global__ void gemm_prepass_kernel(const uint16_t* __restrict__ X, const uint16
 }
 
 // ---------------------------------------------------------------- main kernel
-template <int KP>
-__global__ void __launch_bounds__(kThreads, 1)
+// BT tokens per tile (the MMA's N), SA A stages.  gridDim.z = ks > 1 splits K:
+// the ks CTAs of a cluster (1, 1, ks) take kb_per k-blocks each, push their
+// partial sums (Y contributions of 128 rows x BT tokens) over distributed
+// shared memory to the rank that owns the row, and that rank adds them in
+// rank order.
+template <int KP, int BT, int SA>
+__global__ void __launch_bounds__(kThreads, (KP <= 2 && BT <= 64) ? 2 : 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ planes,
                const uint16_t* __restrict__ g16, const uint32_t* __restrict__ hperm,
                int N, int K, int M, void* __restrict__ Y, int ydt, int32_t* dev_status, uint64_t timeout_ns,
-               int nsx)
+               int nsx, int kb_per)
 {
-    constexpr int BT = gemm_bt(KP), SA = gemm_sa(KP), NCOLS = gemm_tmem_cols(KP);
+    constexpr int NCOLS = (KP * BT + SA * KP * 32) <= 256 ? 256 : 512;
     constexpr uint32_t X_STAGE = BT * 128;
     constexpr uint32_t IDESC = idesc_f16(BT);
     static_assert(KP * BT + SA * KP * 32 <= NCOLS, "tensor memory budget");
@@ -253,6 +264,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * kBR, m0 = blockIdx.y * BT;
     const int nkb = (K + kBK - 1) / kBK;
+    const int ks = (int)gridDim.z, rank = (int)blockIdx.z;
+    const int kb0 = rank * kb_per;
+    const int kb1 = kb0 + kb_per < nkb ? kb0 + kb_per : nkb;      // kb0 < kb1 (host guarantees)
+    const int nloc = kb1 - kb0;
+    float* recv = reinterpret_cast<float*>(gbase + (size_t)nsx * X_STAGE + hp_bytes + 256);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSX; ++s) { mbar_init(full_x(s), 1); mbar_init(empty_x(s), 1); }
@@ -283,7 +299,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
             }
             // stage s and its fill count j (phase = j & 1) advance without divisions
             int issued = 0, s = 0, j = 0;
-            for (int kb = 0; kb < nkb; ++kb) {
+            for (int kb = kb0; kb < kb1; ++kb) {
                 if (j > 0 && !mbar_wait(empty_x(s), (j - 1) & 1, abort_flag, dev_status, timeout_ns)) break;
                 mbar_arrive_expect_tx(full_x(s), X_STAGE);
                 tma_load_2d(xs0 + s * X_STAGE, &tmap_x, full_x(s), kb * kBK, m0);
@@ -302,10 +318,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
         if (lane == 0) {                          // ---------------- MMA issuer
             int s = 0;
             uint32_t xphase = 0;
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int sa = kb % SA;
+            for (int it = 0; it < nloc; ++it) {
+                const int sa = it % SA;
                 if (!mbar_wait(full_x(s), xphase, abort_flag, dev_status, timeout_ns)) break;
-                if (!mbar_wait(full_a(sa), (kb / SA) & 1, abort_flag, dev_status, timeout_ns)) break;
+                if (!mbar_wait(full_a(sa), (it / SA) & 1, abort_flag, dev_status, timeout_ns)) break;
                 tc_fence_after();
                 const uint32_t xaddr = xs0 + s * X_STAGE;
 #pragma unroll
@@ -315,7 +331,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
                         const uint32_t a_t = tmem + (uint32_t)(KP * BT + (sa * KP + i) * 32 + kk * 8);
                         const uint32_t d_t = tmem + (uint32_t)(i * BT);
                         tc_mma_f16_ts(d_t, a_t, smem_desc_sw128(xaddr + kk * 32), IDESC,
-                                      (kb > 0 || kk > 0) ? 1u : 0u);
+                                      (it > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
                 tc_commit(empty_x(s));
@@ -358,9 +374,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
                 }
             };
             uint32_t wv[KP][2], hp[KP][32];
-            load_kb(0, wv, hp);
-            for (int kb = 0; kb < nkb && ok; ++kb) {
-                const int sa = kb % SA;
+            load_kb(kb0, wv, hp);
+            for (int kb = kb0; kb < kb1 && ok; ++kb) {
+                const int it = kb - kb0, sa = it % SA;
                 uint32_t cw[KP][2], ch[KP][32];
 #pragma unroll
                 for (int i = 0; i < KP; ++i) {
@@ -369,9 +385,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
 #pragma unroll
                     for (int j = 0; j < 32; ++j) ch[i][j] = hp[i][j];
                 }
-                if (kb + 1 < nkb) load_kb(kb + 1, wv, hp);
-                if (kb >= SA) {
-                    if (!mbar_wait_warp(empty_a(sa), ((kb / SA) - 1) & 1, abort_flag, dev_status, timeout_ns)) {
+                if (kb + 1 < kb1) load_kb(kb + 1, wv, hp);
+                if (it >= SA) {
+                    if (!mbar_wait_warp(empty_a(sa), ((it / SA) - 1) & 1, abort_flag, dev_status, timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -404,17 +420,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
                 }
             };
             uint32_t cur[KP][8], nxt[KP][8];
-            load_slice(0, cur);
+            load_slice(kb0 / 4, cur);
             ok = mbar_wait_warp(hp_full, 0, abort_flag, dev_status, timeout_ns);
-            for (int64_t sl = 0; sl < S && ok; ++sl) {
-                if (sl + 1 < S) load_slice(sl + 1, nxt);
+            for (int64_t sl = kb0 / 4; sl * 4 < kb1 && ok; ++sl) {
+                if ((sl + 1) * 4 < kb1) load_slice(sl + 1, nxt);
     #pragma unroll
                 for (int qk = 0; qk < 4; ++qk) {
                     const int kb = (int)sl * 4 + qk;
-                    if (kb >= nkb || !ok) break;
-                    const int sa = kb % SA;
-                    if (kb >= SA) {
-                        if (!mbar_wait_warp(empty_a(sa), ((kb / SA) - 1) & 1, abort_flag, dev_status, timeout_ns)) {
+                    if (kb >= kb1 || !ok) break;
+                    const int it = kb - kb0, sa = it % SA;
+                    if (it >= SA) {
+                        if (!mbar_wait_warp(empty_a(sa), ((it / SA) - 1) & 1, abort_flag, dev_status, timeout_ns)) {
                             ok = false;
                             break;
                         }
@@ -455,27 +471,54 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
 #pragma unroll
             for (int i = 0; i < KP; ++i)
                 gi[i] = n < N ? __half2float(__ushort_as_half(g16[(int64_t)i * N + n])) : 0.0f;
+            constexpr int CW = BT < 32 ? BT : 32;            // tokens per TMEM load
 #pragma unroll 1
-            for (int c = 0; c < BT / 32; ++c) {
-                float y[32];
+            for (int c = 0; c < BT / CW; ++c) {
+                float y[CW];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) y[j] = 0.0f;
-                uint32_t v[KP][32];
+                for (int j = 0; j < CW; ++j) y[j] = 0.0f;
+                uint32_t v[KP][CW];
 #pragma unroll
-                for (int i = 0; i < KP; ++i) tc_ld_32x32b_x32(tmem + lane_base + (uint32_t)(i * BT + c * 32), v[i]);
+                for (int i = 0; i < KP; ++i) {
+                    if constexpr (CW == 32) tc_ld_32x32b_x32(tmem + lane_base + (uint32_t)(i * BT + c * CW), v[i]);
+                    else tc_ld_32x32b_x16(tmem + lane_base + (uint32_t)(i * BT + c * CW), v[i]);
+                }
                 tc_wait_ld();
 #pragma unroll
                 for (int i = 0; i < KP; ++i)
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) y[j] = fmaf(gi[i], __uint_as_float(v[i][j]), y[j]);
-                if (n < N) {
+                    for (int j = 0; j < CW; ++j) y[j] = fmaf(gi[i], __uint_as_float(v[i][j]), y[j]);
+                if (ks == 1) {
+                    if (n < N) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int64_t m = (int64_t)m0 + c * 32 + j;
-                        if (m < M) store_y(Y, ydt, m * N + n, y[j]);
+                        for (int j = 0; j < CW; ++j) {
+                            const int64_t m = (int64_t)m0 + c * CW + j;
+                            if (m < M) store_y(Y, ydt, m * N + n, y[j]);
+                        }
                     }
+                } else {                          // slot (this rank, row, tokens c*CW ..) at the row's owner
+                    // rank j owns rows [ceil(128 j / ks), ceil(128 (j+1) / ks)); any ks <= 16
+                    const int rpo = (kBR + ks - 1) / ks, owner = (r * ks) / kBR;
+                    const int lr = r - (kBR * owner + ks - 1) / ks;
+                    const uint32_t dst = smem_u32(recv) + (uint32_t)(((rank * rpo + lr) * BT + c * CW) * 4);
+#pragma unroll
+                    for (int j = 0; j < CW; j += 4)
+                        st_dsmem_v4(dst + (uint32_t)(j * 4), (uint32_t)owner, y[j], y[j + 1], y[j + 2], y[j + 3]);
                 }
             }
+        }
+    }
+
+    if (ks > 1) {                                 // every CTA arrives, also one that gave up
+        cluster_sync_all();
+        const int rpo = (kBR + ks - 1) / ks;
+        const int row0 = (kBR * rank + ks - 1) / ks, nrow = (kBR * (rank + 1) + ks - 1) / ks - row0;
+        for (int idx = threadIdx.x; idx < nrow * BT; idx += kThreads) {
+            const int tok = idx / nrow, lr = idx - tok * nrow;
+            float v = 0.0f;
+            for (int j = 0; j < ks; ++j) v += recv[(j * rpo + lr) * BT + tok];
+            const int64_t n = (int64_t)n0 + row0 + lr, m = (int64_t)m0 + tok;
+            if (n < N && m < M) store_y(Y, ydt, m * N + n, v);
         }
     }
 
@@ -525,11 +568,12 @@ GemmWs gemm_ws_layout(int K, int kp, int M, void* base)
     return w;
 }
 
-template <int KP>
+// ks > 1: K split over clusters of (1, 1, ks); every rank gets a whole number
+// of 256-column slices and at least one k-block.
+template <int KP, int BT, int SA>
 rb_status launch_gemm(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs& ws,
-                      int32_t* dev_status, bool pdl, cudaStream_t stream, uint64_t timeout_ns)
+                      int32_t* dev_status, bool pdl, cudaStream_t stream, uint64_t timeout_ns, int ks)
 {
-    constexpr int BT = gemm_bt(KP);
     PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
     if (!enc) return RB_ERR_CUDA;
     CUtensorMap map;
@@ -541,34 +585,82 @@ rb_status launch_gemm(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return RB_ERR_CUDA;
+    const int nkb = (L->k_in + kBK - 1) / kBK;
+    int kb_per = (nkb + ks - 1) / ks;
+    kb_per = (kb_per + 3) / 4 * 4;                            // whole slices per rank
+    ks = (nkb + kb_per - 1) / kb_per;                         // no rank without k-blocks
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     constexpr int kMaxSmem = 227 * 1024;
     int nsx = kSX;
-    while (nsx > 2 && gemm_smem_bytes(KP, L->k_in, nsx) > kMaxSmem) --nsx;
-    const int smem = gemm_smem_bytes(KP, L->k_in, nsx);
+    while (nsx > 2 && gemm_smem_bytes(KP, BT, L->k_in, nsx, ks) > kMaxSmem) --nsx;
+    const int smem = gemm_smem_bytes(KP, BT, L->k_in, nsx, ks);
     if (smem > kMaxSmem) return RB_ERR_UNSUPPORTED;          // K too long for the h pairs in shared memory
     if (dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(gemm_tc_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem) != cudaSuccess)
+        if (cudaFuncSetAttribute(gemm_tc_kernel<KP, BT, SA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMaxSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_tc_kernel<KP, BT, SA>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess)
             return RB_ERR_CUDA;
         attr_set[dev] = true;
     }
-    dim3 grid((unsigned)((L->n_out + kBR - 1) / kBR), (unsigned)((M + BT - 1) / BT));
-    return launch(gemm_tc_kernel<KP>, grid, dim3(kThreads), (size_t)smem, stream, pdl, map, L->planes,
-                  L->g16, (const uint32_t*)ws.hperm, L->n_out, L->k_in, M, Y, ydt, dev_status, timeout_ns, nsx);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((L->n_out + kBR - 1) / kBR), (unsigned)((M + BT - 1) / BT), (unsigned)ks);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (ks > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 1;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = (unsigned)ks;
+        ++na;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<KP, BT, SA>, map, L->planes, L->g16, (const uint32_t*)ws.hperm,
+                           (int)L->n_out, (int)L->k_in, M, Y, ydt, dev_status, timeout_ns, nsx, kb_per) !=
+        cudaSuccess)
+        return RB_ERR_CUDA;
+    return RB_OK;
+}
+
+// Decode-sized M (<= 64): tokens per tile 16, 32 or 64, two A stages, and the
+// K split that gives about two CTAs per SM (at most 16 ranks).
+template <int KP>
+rb_status launch_gemm_decode(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs& ws,
+                             int32_t* dev_status, cudaStream_t stream, uint64_t timeout_ns)
+{
+    const int bt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    const int64_t ctas = (int64_t)((L->n_out + kBR - 1) / kBR) * ((M + bt - 1) / bt);
+    const int nkb = (L->k_in + kBK - 1) / kBK;
+    int ks = 1;
+    while (ks < 16 && ks * 4 < nkb && ctas * ks < 2LL * num_sms()) ks *= 2;
+    if (bt == 16) return launch_gemm<KP, 16, 2>(L, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, ks);
+    if (bt == 32) return launch_gemm<KP, 32, 2>(L, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, ks);
+    return launch_gemm<KP, 64, 2>(L, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, ks);
 }
 
 }  // namespace
 
-// rb_gemm with a caller-chosen bound on every device-side wait.
+// rb_gemm with a caller-chosen bound on every device-side wait; decode = the
+// small-M tile shapes with the K split (rb_gemv for M >= 2 with a workspace).
 rb_status gemm_with_timeout(const rb_layer_t* layer, const uint16_t* X, int M, void* Y, rb_dtype y_dtype,
                                void* workspace, size_t workspace_bytes, int32_t* dev_status, unsigned flags,
-                               cudaStream_t stream, uint64_t timeout_ns)
+                               cudaStream_t stream, uint64_t timeout_ns, bool decode)
 {
     rb_status st = check_apply_args(layer, X, M, Y, y_dtype, flags);
     if (st != RB_OK) return st;
     if (layer->k_planes > 4) return RB_ERR_UNSUPPORTED;
+    if (decode && M > 64) return RB_ERR_SHAPE;
     if (dev_status && !aligned16(dev_status)) return RB_ERR_ALIGN;
     GemmWs ws = gemm_ws_layout(layer->k_in, layer->k_planes, M, workspace);
     if (!workspace || workspace_bytes < ws.bytes) return RB_ERR_WORKSPACE;
@@ -582,13 +674,24 @@ rb_status gemm_with_timeout(const rb_layer_t* layer, const uint16_t* X, int M, v
     st = launch(gemm_prepass_kernel, dim3((unsigned)ctas), dim3(256), 0, stream, pdl, X, layer->h16, M,
                 layer->k_in, layer->k_planes, ws.x16, ws.hperm, dev_status);
     if (st != RB_OK) return st;
+    const int ydt = (int)y_dtype;
+    if (decode) {
+        switch (layer->k_planes) {
+            case 1: return launch_gemm_decode<1>(layer, M, Y, ydt, ws, dev_status, stream, timeout_ns);
+            case 2: return launch_gemm_decode<2>(layer, M, Y, ydt, ws, dev_status, stream, timeout_ns);
+            case 3: return launch_gemm_decode<3>(layer, M, Y, ydt, ws, dev_status, stream, timeout_ns);
+            default: return launch_gemm_decode<4>(layer, M, Y, ydt, ws, dev_status, stream, timeout_ns);
+        }
+    }
     switch (layer->k_planes) {
-        case 1: return launch_gemm<1>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, timeout_ns);
-        case 2: return launch_gemm<2>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, timeout_ns);
-        case 3: return launch_gemm<3>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, timeout_ns);
-        default: return launch_gemm<4>(layer, M, Y, (int)y_dtype, ws, dev_status, true, stream, timeout_ns);
+        case 1: return launch_gemm<1, gemm_bt(1), gemm_sa(1)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+        case 2: return launch_gemm<2, gemm_bt(2), gemm_sa(2)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+        case 3: return launch_gemm<3, gemm_bt(3), gemm_sa(3)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+        default: return launch_gemm<4, gemm_bt(4), gemm_sa(4)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
     }
 }
+
+size_t gemm_workspace(int k_in, int k_planes, int M) { return gemm_ws_layout(k_in, k_planes, M, nullptr).bytes; }
 
 }  // namespace rbw
 
@@ -605,7 +708,7 @@ extern "C" rb_status rb_gemm(const rb_layer_t* layer, const uint16_t* X, int M, 
                              cudaStream_t stream)
 {
     return gemm_with_timeout(layer, X, M, Y, y_dtype, workspace, workspace_bytes, dev_status, flags,
-                             stream, kTimeoutNs);
+                             stream, kTimeoutNs, false);
 }
 
 // ---------------------------------------------------------------------------
@@ -658,5 +761,5 @@ extern "C" rb_status rb_gemm_noalloc(const rb_layer_t* layer, const uint16_t* X,
     void* scratch = noalloc_scratch_address();
     if (!scratch) return RB_ERR_CUDA;
     return rbw::gemm_with_timeout(layer, X, M, Y, y_dtype, scratch, kNoAllocScratchBytes, dev_status, flags,
-                                  stream, rbw::kTimeoutNs);
+                                  stream, rbw::kTimeoutNs, false);
 }

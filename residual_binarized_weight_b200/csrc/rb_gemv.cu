@@ -89,19 +89,6 @@ __device__ __forceinline__ float lut_entry(uint32_t tbase, uint32_t off) {
     else return lds_f32(tbase + C + off);
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void st_dsmem_f32(uint32_t local_saddr, uint32_t rank, float v) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(rank));
-    asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(remote), "f"(v) : "memory");
-}
 
 // Per-row sums (red) plus, with a cluster, the receive area of the rows this CTA
 // sums: CS slots of at most ceil(rows/CS) rows, which never exceeds rows + CS;
@@ -979,10 +966,14 @@ bool use_lut(const rb_layer_t* L, int M) { return M == 1 && L->k_planes <= 4; }
 
 using namespace rbw;
 
+// From this many tokens (and k <= 4) rb_gemv runs on the tcgen05 kernel when
+// the caller passes the workspace it needs (X in fp16 and the h pairs).
+constexpr int kTcMinM = 32;
+
 extern "C" size_t rb_gemv_workspace_bytes(int n_out, int k_in, int k_planes, int M)
 {
-    (void)n_out; (void)k_in; (void)k_planes; (void)M;
-    return 0;          // every rb_gemv path keeps its partial sums on chip
+    if (n_out < 1 || k_in < 32 || k_in % 32 != 0 || M < kTcMinM || M > 64 || k_planes < 1 || k_planes > 4) return 0;
+    return gemm_workspace(k_in, k_planes, M);
 }
 
 static rb_status gemv_dispatch(const rb_layer_t* const* layers, const uint16_t* const* X, void* const* Y,
@@ -1023,10 +1014,11 @@ extern "C" rb_status rb_gemv(const rb_layer_t* layer, const uint16_t* X, int M, 
                              rb_dtype y_dtype, void* workspace, size_t workspace_bytes,
                              int32_t* dev_status, unsigned flags, cudaStream_t stream)
 {
-    (void)dev_status;
-    (void)workspace;
-    (void)workspace_bytes;
     if (!layer) return RB_ERR_ARG;
+    if (M >= kTcMinM && M <= 64 && layer->k_planes <= 4 && workspace != nullptr &&
+        workspace_bytes >= rb_gemv_workspace_bytes(layer->n_out, layer->k_in, layer->k_planes, M))
+        return gemm_with_timeout(layer, X, M, Y, y_dtype, workspace, workspace_bytes, dev_status, flags, stream,
+                                 kWaitTimeoutNs, true);
     return gemv_dispatch(&layer, &X, &Y, 1, M, y_dtype, flags, stream);
 }
 

@@ -29,6 +29,27 @@ __host__ __device__ inline int64_t word_offset(int i, int64_t s, int64_t r, int 
 }
 
 // ---------------------------------------------------------------- device helpers
+// Thread-block cluster: rank, a full barrier (release / acquire), and stores
+// into another CTA's shared memory at the same offset as a local address.
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void st_dsmem_f32(uint32_t local_saddr, uint32_t rank, float v) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(rank));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(remote), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_dsmem_v4(uint32_t local_saddr, uint32_t rank, float a, float b, float c, float d) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(rank));
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" :: "r"(remote), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
 __device__ __forceinline__ void pdl_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
@@ -96,6 +117,13 @@ inline rb_status check_apply_args(const rb_layer_t* L, const void* X, int M, con
 }
 
 int num_sms();                 // of the current device (cached per device)
+
+// The tcgen05 kernel (rb_gemm.cu); decode = small-M tiles with a K split.
+constexpr uint64_t kWaitTimeoutNs = 1000000000ull;    // bound on each device-side wait (1 s)
+rb_status gemm_with_timeout(const rb_layer_t* layer, const uint16_t* X, int M, void* Y, rb_dtype y_dtype,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status, unsigned flags,
+                            cudaStream_t stream, uint64_t timeout_ns, bool decode);
+size_t gemm_workspace(int k_in, int k_planes, int M);  // bytes of its workspace (X in fp16, h pairs)
 bool device_is_sm100();        // current device is compute capability 10.x
 
 }  // namespace rbw

@@ -181,6 +181,30 @@ def test_gemv_batch_multi_token(N, K, k, M, count):
                       per_elem=per_elem(M, k))
 
 
+@pytest.mark.parametrize("N,K,k,M", [(4096, 4096, 2, 32), (1000, 2048, 1, 48), (300, 4096, 4, 33), (4096, 11008, 2, 64),
+                                     (70, 1056, 2, 40)])
+def test_gemv_both_tensor_core_paths(N, K, k, M):
+    """For M >= 32 rb_gemv runs the tcgen05 kernel when given its workspace
+    (K split over clusters of any size up to 16) and the mma.sync kernel
+    without one; both match the oracle."""
+    rng = np.random.default_rng(N + K + M)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=6)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    X = synth.activations(M, K, seed=M + 5)
+    Yr = oracle.apply(planes, g16, h16, N, K, k, X)
+    bound = cases.abs_bound(g16, h16, X)
+    assert rbw.gemv_workspace_bytes(N, K, k, M) > 0
+    Xd = cases.to_dev(X)
+    for ws in (rbw.workspace(rbw.gemv_workspace_bytes(N, K, k, M)), None):
+        st = torch.zeros(4, dtype=torch.int32, device="cuda")
+        Y = rbw.gemv(L, Xd, ws=ws, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st[0].item()) == 0
+        cases.check_y(Y.cpu().numpy().astype(np.float64), Yr, bound, bf16=False, per_elem=per_elem(M, k))
+
+
 def test_gemv_batch_rejects_mixed_shapes():
     a = rbw.PackedLayer(64, 256, 2)
     b = rbw.PackedLayer(64, 512, 2)
