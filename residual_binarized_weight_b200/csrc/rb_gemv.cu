@@ -99,8 +99,8 @@ __host__ __device__ inline int lut_row_bytes(int64_t Nt, int R, int CS)
     return (int)(((CS > 1 ? 2 * rows + CS : rows) + 3) / 4 * 16);
 }
 
-// Byte tables of slice s for all KP planes (256 threads: thread (group gg,
-// part) writes bytes 32*part .. 32*part+31 of group gg).  Plane i's entry
+// Byte tables of slice s for all KP planes (thread (group gg, part) writes
+// the part's 256 / (threads / 32) consecutive bytes of group gg).  Plane i's entry
 // (byte, group) sits at region(i/2) + byte*256 + (i%2)*128 + group*4.
 template <int KP>
 __device__ __forceinline__ void lut_load_h(uint4 (&hr)[KP], const uint16_t* __restrict__ h16, int64_t s, int K)
@@ -143,10 +143,12 @@ __device__ __forceinline__ void lut_build(float* lut, const uint4 (&hrr)[KP], co
             const int q = low == 1 ? 0 : low == 2 ? 1 : low == 4 ? 2 : 3;
             L[n] = L[n & (n - 1)] + 2.0f * v[q];
         }
-        float Hh[2];                              // signed sums of columns 4..7 for this part's high nibbles
+        constexpr int kBPP = 256 / (kLutThreads / 32);          // table bytes per part (thread of a group)
+        constexpr int kHN = kBPP >= 16 ? kBPP / 16 : 1;         // high nibbles per part
+        float Hh[kHN];                            // signed sums of columns 4..7 for this part's high nibbles
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int n = 2 * part + e;
+        for (int e = 0; e < kHN; ++e) {
+            const int n = kHN * part + e;
             float acc = 0.0f;
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc += ((n >> q) & 1) ? v[4 + q] : -v[4 + q];
@@ -154,9 +156,9 @@ __device__ __forceinline__ void lut_build(float* lut, const uint4 (&hrr)[KP], co
         }
         char* base = reinterpret_cast<char*>(lut) + (i >> 1) * 65536 + (i & 1) * 128 + gg * 4;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int b = 32 * part + j;
-            *reinterpret_cast<float*>(base + b * 256) = L[b & 15] + Hh[(b >> 4) & 1];
+        for (int j = 0; j < kBPP; ++j) {
+            const int b = kBPP * part + j;
+            *reinterpret_cast<float*>(base + b * 256) = L[b & 15] + Hh[(b >> 4) - kHN * part];
         }
     }
 }
