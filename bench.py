@@ -485,6 +485,23 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
         t = time_events(torch, f, 2 * LAYERS, stream)
         out["gemv_M%d_plain_launches" % M] = {"us": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
                                "tokens_per_s": M / t}
+    # rb_gemv_batch at M = 4 and 16 (one tensor-core launch over the 96 layers), and
+    # rb_gemv at M = 64 with its workspace (tcgen05 kernel), 96 distinct layers
+    for M in (4, 16):
+        X = torch.from_numpy(synth.activations(M, K_IN, seed=M).view(np.int16)).to(dev)
+        Ys = [torch.empty(M, N_OUT, dtype=torch.float32, device=dev) for _ in range(LAYERS)]
+        t = time_events(torch, lambda: rbw.gemv_batch(layers, [X] * LAYERS, Ys, stream=stream), 5, stream) / LAYERS
+        out["gemv_M%d_batch96" % M] = {"us_per_layer": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
+                                       "TFLOPs": 2.0 * M * N_OUT * K_IN * K_PLANES / t / 1e12}
+    X = torch.from_numpy(synth.activations(64, K_IN, seed=64).view(np.int16)).to(dev)
+    Y = torch.empty(64, N_OUT, dtype=torch.float32, device=dev)
+    ws = rbw.workspace(rbw.gemv_workspace_bytes(N_OUT, K_IN, K_PLANES, 64), dev)
+    it64 = iter(range(10 ** 9))
+    t = time_events(torch, lambda: rbw.gemv(layers[next(it64) % LAYERS], X, Y=Y, ws=ws, stream=stream), 2 * LAYERS,
+                    stream)
+    out["gemv_M64_tcgen05"] = {"us": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
+                               "TFLOPs": 2.0 * 64 * N_OUT * K_IN * K_PLANES / t / 1e12}
+    del layers
     # rb_gemm at M = 2048 on the prefill shape
     try:
         X = torch.from_numpy(synth.activations(2048, K_IN, seed=7).view(np.int16)).to(dev)
@@ -500,6 +517,23 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
                              "flops": fl}
     except rbw.RbError as e:
         out["gemm_M2048"] = {"unavailable": str(e)}
+    # rb_gemm on the prefill workload's up (14336 x 4096) and down (4096 x 14336) layers,
+    # Laplace(0, 0.01) weights, activations with 1% heavy columns, M = 512 and 2048
+    wl5 = synth.workload("prefill_14336x4096_k2")
+    for layer in wl5.layers:
+        N5, K5 = layer.n_out, layer.k_in
+        W5 = torch.from_numpy(synth.weights(layer)).to(dev)
+        g5, h5 = rbw.svid_greedy(W5, K_PLANES, iters=20)
+        L5 = rbw.pack(W5, g5, h5, K_PLANES)
+        del W5
+        for M in (512, 2048):
+            X = torch.from_numpy(synth.activations_for(wl5, M, K5).view(np.int16)).to(dev)
+            Y = torch.empty(M, N5, dtype=torch.float32, device=dev)
+            ws = rbw.workspace(rbw.gemm_workspace_bytes(N5, K5, K_PLANES, M), dev)
+            t = time_events(torch, lambda: rbw.gemm(L5, X, Y=Y, ws=ws, stream=stream), 10, stream)
+            fl = 2.0 * M * N5 * K5 * K_PLANES
+            out["gemm_%s_%dx%d_M%d" % (layer.name, N5, K5, M)] = {
+                "us": t * 1e6, "TFLOPs": fl / t / 1e12, "frac_of_bf16_peak": fl / t / 1e12 / bf16_peak}
     return out
 
 
