@@ -51,6 +51,8 @@ def _load():
         lib.oracle_apply.restype = None
         lib.oracle_svid_greedy.argtypes = [vp, i64, i64, i32, i32, vp, vp]
         lib.oracle_svid_greedy.restype = i32
+        lib.oracle_svid_iterative.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp]
+        lib.oracle_svid_iterative.restype = i32
         lib.oracle_plane_words.argtypes = [i64, i64, i32]
         lib.oracle_plane_words.restype = i64
         lib.oracle_f64_to_f16.argtypes = [dbl]
@@ -149,6 +151,18 @@ def svid_greedy(W, k: int, iters: int = 20):
     st = _load().oracle_svid_greedy(_p(W), N, K, k, iters, _p(g), _p(h))
     if st != 0:
         raise ValueError("oracle_svid_greedy: bad arguments")
+    return g, h
+
+
+def svid_iterative(W, k: int, sweeps: int = 20, iters: int = 20):
+    """Iterative residual SVID (Gauss-Seidel sweeps from the greedy scales), float64."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    g = np.zeros((k, N), np.float32)
+    h = np.zeros((k, K), np.float32)
+    st = _load().oracle_svid_iterative(_p(W), N, K, k, sweeps, iters, _p(g), _p(h))
+    if st != 0:
+        raise ValueError("oracle_svid_iterative: bad arguments")
     return g, h
 
 

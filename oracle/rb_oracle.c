@@ -40,6 +40,14 @@
  *     |R_{i-1}| by power iteration in float64: v0 = 1/sqrt(K), then `iters`
  *     rounds of u = A v / |A v|, v = A^T u / |A^T u|; sigma = u^T A v;
  *     g_i = fp32(sqrt(sigma) u), h_i = fp32(sqrt(sigma) v).
+ *   - the iterative residual SVID (RaBiT, Algorithm 1, without the I/O
+ *     channel preprocessing, i.e. the alpha = 0 form) starts from the greedy
+ *     scales and the signs of the greedy recurrence, then runs `sweeps`
+ *     Gauss-Seidel sweeps: for i = 1..k the target of plane i is
+ *     T_i = W - sum_{j != i} diag(g_j) B_j diag(h_j) with the latest values of
+ *     the other planes, B_i = sign(T_i) and (g_i, h_i) = the rank-1 of |T_i|
+ *     by the same power iteration.  T_i is formed in float64: each term
+ *     g_j[r]*h_j[c] is exact there and is subtracted in plane order j = 1..k.
  *
  * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC (no fast-math);
  * on x86-64 float arithmetic is SSE single precision, so every fp32 step
@@ -353,6 +361,98 @@ int oracle_svid_greedy(const float *W, int64_t N, int64_t K, int k, int iters,
         }
     }
     free(R);
+    free(u);
+    free(v);
+    return 0;
+}
+
+/* Rank-1 of |T| (T float64 [N][K]) by the greedy rule's power iteration,
+ * with the same summation orders; writes g_row[N], h_row[K]. */
+static void rank1_abs_f64(const double *T, int64_t N, int64_t K, int iters, double *u, double *v,
+                          float *g_row, float *h_row)
+{
+    for (int64_t c = 0; c < K; ++c) v[c] = 1.0 / sqrt((double)K);
+    for (int t = 0; t < iters; ++t) {
+        double nu = 0.0, nv = 0.0;
+        #pragma omp parallel for schedule(static)
+        for (int64_t r = 0; r < N; ++r) {          /* u = A v */
+            double acc = 0.0;
+            for (int64_t c = 0; c < K; ++c) acc += fabs(T[r * K + c]) * v[c];
+            u[r] = acc;
+        }
+        for (int64_t r = 0; r < N; ++r) nu += u[r] * u[r];
+        nu = sqrt(nu);
+        for (int64_t r = 0; r < N; ++r) u[r] = nu > 0.0 ? u[r] / nu : 0.0;
+        #pragma omp parallel
+        {                                          /* v = A^T u, rows in order */
+            int nt = omp_get_num_threads(), tid = omp_get_thread_num();
+            int64_t c0 = K * tid / nt, c1 = K * (tid + 1) / nt;
+            for (int64_t c = c0; c < c1; ++c) v[c] = 0.0;
+            for (int64_t r = 0; r < N; ++r) {
+                double ur = u[r];
+                for (int64_t c = c0; c < c1; ++c) v[c] += fabs(T[r * K + c]) * ur;
+            }
+        }
+        for (int64_t c = 0; c < K; ++c) nv += v[c] * v[c];
+        nv = sqrt(nv);
+        for (int64_t c = 0; c < K; ++c) v[c] = nv > 0.0 ? v[c] / nv : 0.0;
+    }
+    double sigma = 0.0;                            /* sigma = u^T A v */
+    for (int64_t r = 0; r < N; ++r) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < K; ++c) acc += fabs(T[r * K + c]) * v[c];
+        sigma += u[r] * acc;
+    }
+    double rs = sigma > 0.0 ? sqrt(sigma) : 0.0;
+    for (int64_t r = 0; r < N; ++r) g_row[r] = (float)(rs * u[r]);
+    for (int64_t c = 0; c < K; ++c) h_row[c] = (float)(rs * v[c]);
+}
+
+int oracle_svid_iterative(const float *W, int64_t N, int64_t K, int k, int sweeps, int iters,
+                          float *g, float *h)
+{
+    if (check_args(N, K, k) || iters < 1 || sweeps < 0) return -1;
+    if (oracle_svid_greedy(W, N, K, k, iters, g, h)) return -1;     /* sweep 0: the greedy pass */
+    if (sweeps == 0) return 0;
+    signed char *B = (signed char *)malloc((size_t)(k * N * K));
+    double *T = (double *)malloc(sizeof(double) * (size_t)(N * K));
+    double *u = (double *)malloc(sizeof(double) * (size_t)N);
+    double *v = (double *)malloc(sizeof(double) * (size_t)K);
+    if (!B || !T || !u || !v) { free(B); free(T); free(u); free(v); return -1; }
+    /* signs of the greedy pass: the fp32 recurrence of the packer */
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < N; ++r) {
+        for (int64_t c = 0; c < K; ++c) {
+            float Rv = W[r * K + c];
+            for (int i = 0; i < k; ++i) {
+                int b = (Rv >= 0.0f);
+                B[((int64_t)i * N + r) * K + c] = (signed char)(b ? 1 : -1);
+                float tt = g[(int64_t)i * N + r] * h[(int64_t)i * K + c];
+                Rv = b ? (Rv - tt) : (Rv + tt);
+            }
+        }
+    }
+    for (int t = 0; t < sweeps; ++t) {
+        for (int i = 0; i < k; ++i) {
+            /* T_i = W - sum_{j != i} g_j B_j h_j (float64, planes in order), B_i = sign(T_i) */
+            #pragma omp parallel for schedule(static)
+            for (int64_t r = 0; r < N; ++r) {
+                for (int64_t c = 0; c < K; ++c) {
+                    double x = (double)W[r * K + c];
+                    for (int j = 0; j < k; ++j) {
+                        if (j == i) continue;
+                        double p = (double)g[(int64_t)j * N + r] * (double)h[(int64_t)j * K + c];
+                        x = B[((int64_t)j * N + r) * K + c] > 0 ? x - p : x + p;
+                    }
+                    T[r * K + c] = x;
+                    B[((int64_t)i * N + r) * K + c] = (signed char)(x >= 0.0 ? 1 : -1);
+                }
+            }
+            rank1_abs_f64(T, N, K, iters, u, v, g + (int64_t)i * N, h + (int64_t)i * K);
+        }
+    }
+    free(B);
+    free(T);
     free(u);
     free(v);
     return 0;
