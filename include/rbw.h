@@ -209,6 +209,26 @@ RB_API rb_status rb_svid_greedy(const float *W, int n_out, int k_in, int k_plane
                          float *g, float *h, void *workspace, size_t workspace_bytes,
                          cudaStream_t stream);
 
+/*
+ * rb_svid_iterative -- iterative residual SVID (RaBiT, Algorithm 1 without
+ * the I/O channel preprocessing): the greedy scales, then `sweeps`
+ * Gauss-Seidel sweeps (the pages run 20).  Sweep t refits plane i = 1..k to
+ * T_i = W - sum_{j != i} diag(g_j) B_j diag(h_j) with the latest scales and
+ * signs of the other planes: B_i = sign(T_i) (sign(0) = +1) and (g_i, h_i) =
+ * the rank-1 of |T_i| by the same float64 power iteration as rb_svid_greedy.
+ * T_i is formed in float64 (each g_j[r] h_j[c] is exact there), planes in
+ * order.  The signs are internal: rb_pack derives the deployed planes from W
+ * and the returned scales by the residual recurrence.
+ *   g, h out [k][N], [k][K] fp32 (also hold the state between sweeps).
+ *   workspace: rb_svid_iterative_workspace_bytes(N, K, k) bytes (scratch of
+ *   the power iteration and the k sign planes); no clearing needed.
+ *   sweeps = 0 gives exactly rb_svid_greedy's scales.
+ */
+RB_API size_t rb_svid_iterative_workspace_bytes(int n_out, int k_in, int k_planes);
+RB_API rb_status rb_svid_iterative(const float *W, int n_out, int k_in, int k_planes, int sweeps, int iters,
+                                   float *g, float *h, void *workspace, size_t workspace_bytes,
+                                   cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,6 +1,10 @@
 // rb_svid.cu -- greedy SVID scales on the device (RaBiT names Greedy SVID as
 // the traditional initialiser it improves on; the greedy form takes, plane by
-// plane, the rank-1 approximation of |R_{i-1}|).
+// plane, the rank-1 approximation of |R_{i-1}|), and the iterative residual
+// SVID of RaBiT's Algorithm 1 without the I/O channel preprocessing
+// (Gauss-Seidel sweeps: plane i is refitted to T_i = W - sum_{j != i}
+// diag(g_j) B_j diag(h_j) with the latest values of the other planes,
+// B_i = sign(T_i), (g_i, h_i) = rank-1 of |T_i|).
 //
 // For plane i the matrix A = |R_{i-1}| is never stored: every pass recomputes
 // R_{i-1} from W and the scales of the earlier planes with the fp32
@@ -40,6 +44,26 @@ SvidWs svid_ws_layout(int N, int K, void* base)
     return w;
 }
 
+// Iterative form: the signs B_j of every plane, [k][N][K/32] words, bit c % 32
+// of word c / 32 set for +1, after the power-iteration scratch.
+size_t svid_sign_bytes(int N, int K, int k) { return ((size_t)k * N * (K / 32) * 4 + 255) / 256 * 256; }
+
+// T_i[r][c] = W - sum_{j != i} g_j[r] h_j[c] B_j[r][c] in float64: each product
+// of two fp32 values is exact, subtracted in plane order.
+__device__ __forceinline__ double target_value(const float* W, const float* g, const float* h, const uint32_t* S,
+                                               int N, int K, int k, int plane, int64_t r, int64_t c)
+{
+    double x = (double)W[r * K + c];
+    const int64_t words = K / 32;
+    for (int j = 0; j < k; ++j) {
+        if (j == plane) continue;
+        const double p = __dmul_rn((double)g[(int64_t)j * N + r], (double)h[(int64_t)j * K + c]);
+        const bool pos = (S[((int64_t)j * N + r) * words + (c >> 5)] >> (c & 31)) & 1u;
+        x = pos ? __dsub_rn(x, p) : __dadd_rn(x, p);
+    }
+    return x;
+}
+
 // |R_{i-1}[r][c]| for plane i (0-based) from W and the scales of planes < i.
 __device__ __forceinline__ double abs_residual(const float* W, const float* g, const float* h,
                                                int N, int K, int plane, int64_t r, int64_t c)
@@ -53,32 +77,43 @@ __device__ __forceinline__ double abs_residual(const float* W, const float* g, c
     return fabs((double)R);
 }
 
+// A[r][c] for plane `plane`: |R_{plane-1}| (greedy) or |T_plane| (iterative, S != nullptr).
+template <bool ITER>
+__device__ __forceinline__ double abs_target(const float* W, const float* g, const float* h, const uint32_t* S,
+                                             int N, int K, int k, int plane, int64_t r, int64_t c)
+{
+    if constexpr (ITER) return fabs(target_value(W, g, h, S, N, K, k, plane, r, c));
+    else return abs_residual(W, g, h, N, K, plane, r, c);
+}
+
 // out[r] = sum_c A[r][c] * x[c]   (one warp per row)
+template <bool ITER>
 __global__ void svid_av_kernel(const float* __restrict__ W, const float* __restrict__ g,
-                               const float* __restrict__ h, int N, int K, int plane,
-                               const double* __restrict__ x, double* __restrict__ out)
+                               const float* __restrict__ h, const uint32_t* __restrict__ S, int N, int K, int k,
+                               int plane, const double* __restrict__ x, double* __restrict__ out)
 {
     const int lane = threadIdx.x & 31;
     const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (r >= N) return;
     double acc = 0.0;
-    for (int64_t c = lane; c < K; c += 32) acc += abs_residual(W, g, h, N, K, plane, r, c) * x[c];
+    for (int64_t c = lane; c < K; c += 32) acc += abs_target<ITER>(W, g, h, S, N, K, k, plane, r, c) * x[c];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) out[r] = acc;
 }
 
 // vpart[chunk][c] = sum_{r in chunk} A[r][c] * u[r]   (rows in order)
+template <bool ITER>
 __global__ void svid_atu_partial_kernel(const float* __restrict__ W, const float* __restrict__ g,
-                                        const float* __restrict__ h, int N, int K, int plane,
-                                        const double* __restrict__ u, double* __restrict__ vpart)
+                                        const float* __restrict__ h, const uint32_t* __restrict__ S, int N, int K,
+                                        int k, int plane, const double* __restrict__ u, double* __restrict__ vpart)
 {
     const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int chunk = blockIdx.y;
     if (c >= K) return;
     const int64_t r0 = (int64_t)N * chunk / kRowChunks, r1 = (int64_t)N * (chunk + 1) / kRowChunks;
     double acc = 0.0;
-    for (int64_t r = r0; r < r1; ++r) acc += abs_residual(W, g, h, N, K, plane, r, c) * u[r];
+    for (int64_t r = r0; r < r1; ++r) acc += abs_target<ITER>(W, g, h, S, N, K, k, plane, r, c) * u[r];
     vpart[(int64_t)chunk * K + c] = acc;
 }
 
@@ -131,6 +166,73 @@ __global__ void svid_finish_kernel(const double* __restrict__ u, const double* _
     for (int64_t c = threadIdx.x; c < K; c += blockDim.x) h[(int64_t)plane * K + c] = (float)(rs * v[c]);
 }
 
+// Signs of the greedy pass (the fp32 recurrence of rb_pack): one warp per
+// (row, word); the ballot of the 32 columns is the word of each plane.
+__global__ void svid_signs_greedy_kernel(const float* __restrict__ W, const float* __restrict__ g,
+                                         const float* __restrict__ h, int N, int K, int k, uint32_t* __restrict__ S)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t words = K / 32, items = (int64_t)N * words;
+    for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items;
+         it += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+        const int64_t r = it / words, w = it % words, c = w * 32 + lane;
+        float R = W[r * K + c];
+        for (int p = 0; p < k; ++p) {
+            const bool b = R >= 0.0f;
+            const uint32_t word = __ballot_sync(0xffffffffu, b);
+            if (lane == 0) S[((int64_t)p * N + r) * words + w] = word;
+            const float tt = __fmul_rn(g[(int64_t)p * N + r], h[(int64_t)p * K + c]);
+            R = b ? __fsub_rn(R, tt) : __fadd_rn(R, tt);
+        }
+    }
+}
+
+// B_plane = sign(T_plane) with the other planes' current scales and signs.
+__global__ void svid_signs_update_kernel(const float* __restrict__ W, const float* __restrict__ g,
+                                         const float* __restrict__ h, uint32_t* __restrict__ S, int N, int K, int k,
+                                         int plane)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t words = K / 32, items = (int64_t)N * words;
+    for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items;
+         it += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+        const int64_t r = it / words, w = it % words, c = w * 32 + lane;
+        const bool b = target_value(W, g, h, S, N, K, k, plane, r, c) >= 0.0;
+        const uint32_t word = __ballot_sync(0xffffffffu, b);
+        if (lane == 0) S[((int64_t)plane * N + r) * words + w] = word;
+    }
+}
+
+// Power iteration on A (greedy or iterative form) for one plane, then
+// (g_plane, h_plane) = fp32(sqrt(sigma) u), fp32(sqrt(sigma) v).
+template <bool ITER>
+rb_status svid_plane(const float* W, float* g, float* h, const uint32_t* S, int N, int K, int k, int plane,
+                     int iters, const SvidWs& ws, cudaStream_t stream)
+{
+    const dim3 av_grid((unsigned)((N + 7) / 8)), av_blk(256);
+    const dim3 atu_grid((unsigned)((K + 255) / 256), kRowChunks), atu_blk(256);
+    const dim3 red_grid((unsigned)((K + 255) / 256)), red_blk(256);
+    rb_status st = launch(svid_init_kernel, dim3(8), dim3(256), 0, stream, false, ws.v, K);
+    for (int it = 0; it < iters && st == RB_OK; ++it) {
+        st = launch(svid_av_kernel<ITER>, av_grid, av_blk, 0, stream, false, W, (const float*)g, (const float*)h, S,
+                    N, K, k, plane, (const double*)ws.v, ws.u);
+        if (st == RB_OK) st = launch(svid_normalize_kernel, dim3(1), dim3(1024), 0, stream, false, ws.u, (int64_t)N);
+        if (st == RB_OK)
+            st = launch(svid_atu_partial_kernel<ITER>, atu_grid, atu_blk, 0, stream, false, W, (const float*)g,
+                        (const float*)h, S, N, K, k, plane, (const double*)ws.u, ws.vpart);
+        if (st == RB_OK) st = launch(svid_atu_reduce_kernel, red_grid, red_blk, 0, stream, false,
+                                     (const double*)ws.vpart, K, ws.v);
+        if (st == RB_OK) st = launch(svid_normalize_kernel, dim3(1), dim3(1024), 0, stream, false, ws.v, (int64_t)K);
+    }
+    if (st == RB_OK)
+        st = launch(svid_av_kernel<ITER>, av_grid, av_blk, 0, stream, false, W, (const float*)g, (const float*)h, S,
+                    N, K, k, plane, (const double*)ws.v, ws.av);
+    if (st == RB_OK)
+        st = launch(svid_finish_kernel, dim3(1), dim3(1024), 0, stream, false, (const double*)ws.u,
+                    (const double*)ws.v, (const double*)ws.av, N, K, plane, g, h);
+    return st;
+}
+
 }  // namespace
 }  // namespace rbw
 
@@ -153,30 +255,47 @@ extern "C" rb_status rb_svid_greedy(const float* W, int n_out, int k_in, int k_p
     SvidWs ws = svid_ws_layout(n_out, k_in, workspace);
     if (workspace_bytes < ws.bytes) return RB_ERR_WORKSPACE;
     if (!device_is_sm100()) return RB_ERR_UNSUPPORTED;
-    const int N = n_out, K = k_in;
-    const dim3 av_grid((unsigned)((N + 7) / 8)), av_blk(256);
-    const dim3 atu_grid((unsigned)((K + 255) / 256), kRowChunks), atu_blk(256);
-    const dim3 red_grid((unsigned)((K + 255) / 256)), red_blk(256);
     for (int i = 0; i < k_planes; ++i) {
-        rb_status st = launch(svid_init_kernel, dim3(8), dim3(256), 0, stream, false, ws.v, K);
-        for (int it = 0; it < iters && st == RB_OK; ++it) {
-            st = launch(svid_av_kernel, av_grid, av_blk, 0, stream, false, W, (const float*)g,
-                        (const float*)h, N, K, i, (const double*)ws.v, ws.u);
-            if (st == RB_OK) st = launch(svid_normalize_kernel, dim3(1), dim3(1024), 0, stream, false, ws.u, (int64_t)N);
-            if (st == RB_OK)
-                st = launch(svid_atu_partial_kernel, atu_grid, atu_blk, 0, stream, false, W, (const float*)g,
-                            (const float*)h, N, K, i, (const double*)ws.u, ws.vpart);
-            if (st == RB_OK) st = launch(svid_atu_reduce_kernel, red_grid, red_blk, 0, stream, false,
-                                         (const double*)ws.vpart, K, ws.v);
-            if (st == RB_OK) st = launch(svid_normalize_kernel, dim3(1), dim3(1024), 0, stream, false, ws.v, (int64_t)K);
-        }
-        if (st == RB_OK)
-            st = launch(svid_av_kernel, av_grid, av_blk, 0, stream, false, W, (const float*)g,
-                        (const float*)h, N, K, i, (const double*)ws.v, ws.av);
-        if (st == RB_OK)
-            st = launch(svid_finish_kernel, dim3(1), dim3(1024), 0, stream, false, (const double*)ws.u,
-                        (const double*)ws.v, (const double*)ws.av, N, K, i, g, h);
+        rb_status st = svid_plane<false>(W, g, h, nullptr, n_out, k_in, k_planes, i, iters, ws, stream);
         if (st != RB_OK) return st;
     }
     return RB_OK;
+}
+
+extern "C" size_t rb_svid_iterative_workspace_bytes(int n_out, int k_in, int k_planes)
+{
+    if (n_out < 1 || k_in < 32 || k_in % 32 != 0 || k_planes < 1 || k_planes > 8) return 0;
+    return svid_ws_layout(n_out, k_in, nullptr).bytes + svid_sign_bytes(n_out, k_in, k_planes);
+}
+
+extern "C" rb_status rb_svid_iterative(const float* W, int n_out, int k_in, int k_planes, int sweeps, int iters,
+                                       float* g, float* h, void* workspace, size_t workspace_bytes,
+                                       cudaStream_t stream)
+{
+    if (!W || !g || !h || !workspace) return RB_ERR_ARG;
+    if (k_planes < 1 || k_planes > 8 || iters < 1 || iters > 10000 || sweeps < 0 || sweeps > 1000) return RB_ERR_ARG;
+    if (n_out < 1 || k_in < 32 || k_in % 32 != 0) return RB_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(g) || !aligned16(h) || !aligned16(workspace)) return RB_ERR_ALIGN;
+    SvidWs ws = svid_ws_layout(n_out, k_in, workspace);
+    if (workspace_bytes < ws.bytes + svid_sign_bytes(n_out, k_in, k_planes)) return RB_ERR_WORKSPACE;
+    if (!device_is_sm100()) return RB_ERR_UNSUPPORTED;
+    uint32_t* S = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + ws.bytes);
+    for (int i = 0; i < k_planes; ++i) {                  // sweep 0: the greedy pass
+        rb_status st = svid_plane<false>(W, g, h, nullptr, n_out, k_in, k_planes, i, iters, ws, stream);
+        if (st != RB_OK) return st;
+    }
+    if (sweeps == 0) return RB_OK;
+    const int64_t items = (int64_t)n_out * (k_in / 32);
+    int64_t ctas = (items + 7) / 8;
+    if (ctas > 16 * num_sms()) ctas = 16 * num_sms();
+    rb_status st = launch(svid_signs_greedy_kernel, dim3((unsigned)ctas), dim3(256), 0, stream, false, W,
+                          (const float*)g, (const float*)h, n_out, k_in, k_planes, S);
+    for (int t = 0; t < sweeps && st == RB_OK; ++t) {
+        for (int i = 0; i < k_planes && st == RB_OK; ++i) {
+            st = launch(svid_signs_update_kernel, dim3((unsigned)ctas), dim3(256), 0, stream, false, W,
+                        (const float*)g, (const float*)h, S, n_out, k_in, k_planes, i);
+            if (st == RB_OK) st = svid_plane<true>(W, g, h, S, n_out, k_in, k_planes, i, iters, ws, stream);
+        }
+    }
+    return st;
 }

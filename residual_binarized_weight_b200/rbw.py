@@ -35,6 +35,8 @@ SIGNATURES = {
     "rb_gemm_noalloc": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _u32, _vp]),
     "rb_svid_workspace_bytes": (_sz, [_i32, _i32]),
     "rb_svid_greedy": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "rb_svid_iterative_workspace_bytes": (_sz, [_i32, _i32, _i32]),
+    "rb_svid_iterative": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
 }
 
 
@@ -193,4 +195,17 @@ def svid_greedy(W, k_planes, iters=20, ws=None, stream=None):
     st = lib().rb_svid_greedy(_ptr(W), N, K, k_planes, iters, _ptr(g), _ptr(h), _ptr(ws),
                               ws.numel(), _stream(stream))
     _check("rb_svid_greedy", st)
+    return g, h
+
+
+def svid_iterative(W, k_planes, sweeps=20, iters=20, ws=None, stream=None):
+    """rb_svid_iterative: greedy scales refined by Gauss-Seidel sweeps; fp32 W [N][K] (CUDA)."""
+    N, K = W.shape
+    g = torch.empty(k_planes, N, dtype=torch.float32, device=W.device)
+    h = torch.empty(k_planes, K, dtype=torch.float32, device=W.device)
+    nbytes = int(lib().rb_svid_iterative_workspace_bytes(N, K, k_planes))
+    ws = ws if ws is not None else workspace(nbytes, W.device)
+    st = lib().rb_svid_iterative(_ptr(W), N, K, k_planes, sweeps, iters, _ptr(g), _ptr(h), _ptr(ws),
+                                 ws.numel(), _stream(stream))
+    _check("rb_svid_iterative", st)
     return g, h
