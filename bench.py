@@ -29,6 +29,7 @@ data-path collective); the step time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import math
 import hashlib
 import json
 import os
@@ -517,6 +518,48 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
                              "flops": fl}
     except rbw.RbError as e:
         out["gemm_M2048"] = {"unavailable": str(e)}
+    # decode on the 7B MLP trio (gate/up 11008 x 4096, down 4096 x 11008, k = 2, M = 1 and 8) and
+    # the 28672 x 8192 layer (k = 1 and 2, M = 1, 16, 64): rb_gemv_batch over copies of each
+    # layer that together exceed 3 x L2, so every application streams its planes from HBM
+    def layer_copies(layer, k, min_bytes=400e6):
+        Wl = torch.from_numpy(synth.weights(layer)).to(dev)
+        gl, hl = rbw.svid_greedy(Wl, k, iters=20)
+        base = rbw.pack(Wl, gl, hl, k)
+        del Wl
+        n = max(2, int(math.ceil(min_bytes / base.packed_bytes())))
+        out_l = [base]
+        for _ in range(n - 1):
+            Lc = rbw.PackedLayer(base.n_out, base.k_in, k, dev)
+            Lc.planes.copy_(base.planes)
+            Lc.g16.copy_(base.g16)
+            Lc.h16.copy_(base.h16)
+            out_l.append(Lc)
+        return out_l
+
+    def batch_time(ls, M, seed):
+        X = torch.from_numpy(synth.activations(M, ls[0].k_in, seed=seed).view(np.int16)).to(dev)
+        Ys = [torch.empty(M, ls[0].n_out, dtype=torch.float32, device=dev) for _ in ls]
+        return time_events(torch, lambda: rbw.gemv_batch(ls, [X] * len(ls), Ys, stream=stream), 5, stream) / len(ls)
+
+    wl3 = synth.workload("mlp_trio_7b_k2")
+    trio = {layer.name: layer_copies(layer, K_PLANES) for layer in wl3.layers}
+    for M in (1, 8):
+        ts = {name: batch_time(ls, M, 250 + M) for name, ls in trio.items()}
+        pb = sum(ls[0].packed_bytes() for ls in trio.values())
+        tt = sum(ts.values())
+        out["mlp_trio_7b_M%d" % M] = {"us_per_trio": tt * 1e6, "trio_tokens_per_s": M / tt,
+                                      "packed_GBps": pb / tt / 1e9,
+                                      "us_per_layer": {n: t * 1e6 for n, t in ts.items()}}
+    del trio
+    wl4 = synth.workload("mlp_28672x8192")
+    for k in (1, 2):
+        ls = layer_copies(wl4.layers[0], k)
+        for M in (1, 16, 64):
+            t = batch_time(ls, M, 350 + M)
+            out["mlp_28672x8192_k%d_M%d" % (k, M)] = {
+                "us_per_layer": t * 1e6, "packed_GBps": ls[0].packed_bytes() / t / 1e9, "tokens_per_s": M / t,
+                "TFLOPs": 2.0 * M * ls[0].n_out * ls[0].k_in * k / t / 1e12}
+        del ls
     # rb_gemm on the prefill workload's up (14336 x 4096) and down (4096 x 14336) layers,
     # Laplace(0, 0.01) weights, activations with 1% heavy columns, M = 512 and 2048
     wl5 = synth.workload("prefill_14336x4096_k2")
