@@ -468,8 +468,11 @@ __device__ __forceinline__ void mma_load_words(uint32_t (&w)[KP][8], const uint3
     }
 }
 
+// Two CTAs per SM where the accumulators allow it (k * NT <= 4: at most 128
+// registers per thread), so each SM has 16 warps to hide the shuffle ->
+// shift -> LOP3 -> HMMA latency chain.
 template <int KP, int NT>
-__global__ void __launch_bounds__(kMmaThreads, 1)
+__global__ void __launch_bounds__(kMmaThreads, (KP * NT <= 4) ? 2 : 1)
 gemv_mma_kernel(const __grid_constant__ LutBatch batch, int N, int K, int M, int CS, int groups, int ydt)
 {
     constexpr int TG = 8 * NT;
