@@ -2,29 +2,37 @@
 // status names, sizes, device queries.
 #include "rbw_internal.cuh"
 
+#include <atomic>
+
 namespace rbw {
 
 int num_sms()
 {
-    static int cache[64] = {};
+    static std::atomic<int> cache[64];         // per device, 0 = not yet queried
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+    if (dev >= 0 && dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c) return c;
+    }
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    if (dev >= 0 && dev < 64) cache[dev] = n;
+    if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 
 bool device_is_sm100()
 {
-    static int cache[64] = {};   // 0 unknown, 1 yes, 2 no
+    static std::atomic<int> cache[64];         // per device: 0 unknown, 1 yes, 2 no
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev] == 1;
+    if (dev >= 0 && dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c) return c == 1;
+    }
     int major = 0;
     const bool ok = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess && major == 10;
-    if (dev >= 0 && dev < 64) cache[dev] = ok ? 1 : 2;
+    if (dev >= 0 && dev < 64) cache[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
     return ok;
 }
 

@@ -589,7 +589,7 @@ rb_status launch_gemm(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs
     int kb_per = (nkb + ks - 1) / ks;
     kb_per = (kb_per + 3) / 4 * 4;                            // whole slices per rank
     ks = (nkb + kb_per - 1) / kb_per;                         // no rank without k-blocks
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64];       // per device; setting the attributes twice is harmless
     int dev = 0;
     cudaGetDevice(&dev);
     constexpr int kMaxSmem = 227 * 1024;
@@ -597,13 +597,13 @@ rb_status launch_gemm(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs
     while (nsx > 2 && gemm_smem_bytes(KP, BT, L->k_in, nsx, ks) > kMaxSmem) --nsx;
     const int smem = gemm_smem_bytes(KP, BT, L->k_in, nsx, ks);
     if (smem > kMaxSmem) return RB_ERR_UNSUPPORTED;          // K too long for the h pairs in shared memory
-    if (dev < 64 && !attr_set[dev]) {
+    if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(gemm_tc_kernel<KP, BT, SA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxSmem) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_tc_kernel<KP, BT, SA>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                 cudaSuccess)
             return RB_ERR_CUDA;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_release);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((L->n_out + kBR - 1) / kBR), (unsigned)((M + BT - 1) / BT), (unsigned)ks);

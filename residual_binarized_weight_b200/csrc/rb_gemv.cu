@@ -23,6 +23,8 @@
 // registers; see gemv_mma_kernel.
 #include "rbw_internal.cuh"
 
+#include <atomic>
+
 #include <mutex>
 
 namespace rbw {
@@ -712,16 +714,16 @@ cudaLaunchConfig_t lut_config(const LutPlan& p, int count, cudaLaunchAttribute* 
 template <int KP>
 bool lut_set_attributes()
 {
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64];       // per device; setting the attributes twice is harmless
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return false;
-    if (!attr_set[dev]) {
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(gemv_lut_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
             return false;
         if (cudaFuncSetAttribute(gemv_lut_kernel<KP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
             return false;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_release);
     }
     return true;
 }
@@ -887,16 +889,16 @@ rb_status launch_lut(const rb_layer_t* const* layers, const uint16_t* const* X, 
 template <int KP, int NT>
 rb_status launch_mma_nt(const LutBatch& b, int n, int N, int K, int M, int ydt, bool pdl, cudaStream_t stream)
 {
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64];       // per device; setting the attributes twice is harmless
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RB_ERR_CUDA;
-    if (!attr_set[dev]) {
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(gemv_mma_kernel<KP, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  227 * 1024) != cudaSuccess ||
             cudaFuncSetAttribute(gemv_mma_kernel<KP, NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                 cudaSuccess)
             return RB_ERR_CUDA;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_release);
     }
     const int64_t S = num_slices(K), Nt = num_row_tiles(N);
     const int groups = (int)((Nt + kMmaWarps - 1) / kMmaWarps);
