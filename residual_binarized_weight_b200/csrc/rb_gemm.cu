@@ -683,9 +683,17 @@ rb_status gemm_with_timeout(const rb_layer_t* layer, const uint16_t* X, int M, v
             default: return launch_gemm_decode<4>(layer, M, Y, ydt, ws, dev_status, stream, timeout_ns);
         }
     }
+    // Wider token tiles amortise each k-block's fixed cost (expansion, barriers)
+    // over more MMA work: 256 tokens for k = 1 and 192 for k = 2 (the widest the
+    // 512 tensor-memory columns hold next to the A stages) once M fills them;
+    // 128 below that, where the padding of a wide last tile would cost more.
     switch (layer->k_planes) {
-        case 1: return launch_gemm<1, gemm_bt(1), gemm_sa(1)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
-        case 2: return launch_gemm<2, gemm_bt(2), gemm_sa(2)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+        case 1:
+            if (M >= 1024) return launch_gemm<1, 256, 4>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+            return launch_gemm<1, gemm_bt(1), gemm_sa(1)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+        case 2:
+            if (M >= 1536) return launch_gemm<2, 192, 2>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+            return launch_gemm<2, gemm_bt(2), gemm_sa(2)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
         case 3: return launch_gemm<3, gemm_bt(3), gemm_sa(3)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
         default: return launch_gemm<4, gemm_bt(4), gemm_sa(4)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
     }
