@@ -684,9 +684,9 @@ rb_status gemm_with_timeout(const rb_layer_t* layer, const uint16_t* X, int M, v
         }
     }
     // Wider token tiles amortise each k-block's fixed cost (expansion, barriers)
-    // over more MMA work: 256 tokens for k = 1 and 192 for k = 2 (the widest the
-    // 512 tensor-memory columns hold next to the A stages) once M fills them;
-    // 128 below that, where the padding of a wide last tile would cost more.
+    // over more MMA work: 256 tokens for k = 1, 192 for k = 2 and 96 for k = 3
+    // (the widest the 512 tensor-memory columns hold next to the A stages) once
+    // M fills them; narrower below that, where a wide last tile pads more.
     switch (layer->k_planes) {
         case 1:
             if (M >= 1024) return launch_gemm<1, 256, 4>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
@@ -694,7 +694,9 @@ rb_status gemm_with_timeout(const rb_layer_t* layer, const uint16_t* X, int M, v
         case 2:
             if (M >= 1536) return launch_gemm<2, 192, 2>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
             return launch_gemm<2, gemm_bt(2), gemm_sa(2)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
-        case 3: return launch_gemm<3, gemm_bt(3), gemm_sa(3)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+        case 3:
+            if (M >= 1024) return launch_gemm<3, 96, 2>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+            return launch_gemm<3, gemm_bt(3), gemm_sa(3)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
         default: return launch_gemm<4, gemm_bt(4), gemm_sa(4)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
     }
 }

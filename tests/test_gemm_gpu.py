@@ -53,7 +53,7 @@ def test_gemm_workloads(wl, li, M, ydt):
 
 @pytest.mark.parametrize("N,K,k,M", [(128, 64, 1, 128), (200, 288, 2, 130), (33, 800, 3, 65), (300, 544, 4, 1),
                                      (4097, 256, 2, 7), (129, 1056, 1, 257), (64, 4096, 2, 300),
-                                     (300, 512, 2, 1700), (257, 800, 1, 1100)])
+                                     (300, 512, 2, 1700), (257, 800, 1, 1100), (130, 544, 3, 1030)])
 def test_gemm_ragged(N, K, k, M):
     rng = np.random.default_rng(N + K + 5 * k + M)
     W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
