@@ -30,8 +30,14 @@
 namespace rbw {
 namespace {
 
-constexpr int kLutThreads = 256;
-constexpr int kLutWarps = kLutThreads / 32;
+// Threads per CTA: 256 (two CTAs per SM) while the tables of a plane pair fit
+// 64 KB; 512 for k >= 3, whose 128 KB of tables leave room for one CTA per SM,
+// so that an SM still runs 16 warps.
+template <int KP> struct LutCfg {
+    static constexpr int threads = KP >= 3 ? 512 : 256;
+    static constexpr int warps = threads / 32;
+    static constexpr int min_blocks = KP >= 3 ? 1 : 2;
+};
 constexpr int kLutPF = 2;              // row tiles per warp held in registers ahead of use
 constexpr int kLutPD = 6;              // row tiles per warp prefetched into L2 ahead of use
 
@@ -145,7 +151,7 @@ __device__ __forceinline__ void lut_build(float* lut, const uint4 (&hrr)[KP], co
             const int q = low == 1 ? 0 : low == 2 ? 1 : low == 4 ? 2 : 3;
             L[n] = L[n & (n - 1)] + 2.0f * v[q];
         }
-        constexpr int kBPP = 256 / (kLutThreads / 32);          // table bytes per part (thread of a group)
+        constexpr int kBPP = 256 / LutCfg<KP>::warps;          // table bytes per part (thread of a group)
         constexpr int kHN = kBPP >= 16 ? kBPP / 16 : 1;         // high nibbles per part
         float Hh[kHN];                            // signed sums of columns 4..7 for this part's high nibbles
 #pragma unroll
@@ -216,7 +222,7 @@ __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_
                                           const uint16_t* __restrict__ g16, int64_t s, int64_t s_next,
                                           int64_t S, int64_t Nt, int N, int tb, int te, int warp, int lane)
 {
-    const int nw = te - tb > warp ? (te - tb - warp + kLutWarps - 1) / kLutWarps : 0;
+    const int nw = te - tb > warp ? (te - tb - warp + LutCfg<KP>::warps - 1) / LutCfg<KP>::warps : 0;
     const int iters = (nw + kLutPF - 1) / kLutPF;
     const bool has_next = s_next < S;
     const uint32_t* cur[KP];
@@ -247,17 +253,17 @@ __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_
 #pragma unroll
             for (int i = 0; i < KP; ++i)
                 pr += __half2float(__ushort_as_half(gv[p][i])) * (acc[p][i][0] + acc[p][i][1]);
-            if (j < nw) red[(j * kLutWarps + warp) * 32 + lane] += pr;
+            if (j < nw) red[(j * LutCfg<KP>::warps + warp) * 32 + lane] += pr;
             const int jp = j + kLutPD;
             const bool pf_here = jp < nw;
             if (pf_lane && (pf_here || (has_next && jp - nw < nw))) {
-                const uint32_t* q = pf_here ? pf_cur + (size_t)(t_w + jp * kLutWarps) * 256
-                                            : pf_nxt + (size_t)(t_w + (jp - nw) * kLutWarps) * 256;
+                const uint32_t* q = pf_here ? pf_cur + (size_t)(t_w + jp * LutCfg<KP>::warps) * 256
+                                            : pf_nxt + (size_t)(t_w + (jp - nw) * LutCfg<KP>::warps) * 256;
                 asm volatile("prefetch.global.L2 [%0];" :: "l"(q));
             }
             if (!last || (has_next && p < nw)) {
                 const int jn = last ? p : min(j + kLutPF, nw - 1);
-                const size_t tn = (size_t)(t_w + jn * kLutWarps);
+                const size_t tn = (size_t)(t_w + jn * LutCfg<KP>::warps);
 #pragma unroll
                 for (int i = 0; i < KP; ++i) {
                     const uint32_t* q = (last ? nxt[i] : cur[i]) + tn * 256;
@@ -289,7 +295,7 @@ struct LutBatch {
 };
 
 template <int KP>
-__global__ void __launch_bounds__(kLutThreads, 2)
+__global__ void __launch_bounds__(LutCfg<KP>::threads, LutCfg<KP>::min_blocks)
 gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, int R, int ydt)
 {
     extern __shared__ __align__(1024) float lut[];
@@ -315,7 +321,7 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
     const int64_t s_first = rank;
 #pragma unroll
     for (int p = 0; p < kLutPF; ++p) {
-        const int64_t t = t_begin + warp + (int64_t)p * kLutWarps;
+        const int64_t t = t_begin + warp + (int64_t)p * LutCfg<KP>::warps;
         if (t < t_end && s_first < S) {
             lut_load_tile<KP>(wd[p], planes, s_first, t, S, Nt, lane);
             lut_load_g<KP>(gv[p], g16, t * 32 + lane, N);
@@ -332,11 +338,11 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
         lut_load_h<KP>(hr, h16, s_first, K);
 #pragma unroll
         for (int p = kLutPF; p < kLutPD; ++p) {
-            const int64_t t = t_begin + warp + (int64_t)p * kLutWarps;
+            const int64_t t = t_begin + warp + (int64_t)p * LutCfg<KP>::warps;
             if (t < t_end) lut_prefetch_tile<KP>(planes, s_first, t, S, Nt, lane);
         }
     }
-    for (int64_t x = threadIdx.x; x < chunk_rows; x += kLutThreads) red[x] = 0.0f;
+    for (int64_t x = threadIdx.x; x < chunk_rows; x += LutCfg<KP>::threads) red[x] = 0.0f;
 
     // Per-lane lookup constants: G[sl] byte b' = group offset ((4 sl + b') ^ lane) * 4;
     // SEL[b'] = PRMT selector giving (word byte (b' ^ lane%4)) << 8 | G byte b', zeros above.
@@ -377,7 +383,7 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
     // ---- cross-slice sum
     if (CS == 1) {
         __syncthreads();
-        for (int64_t x = threadIdx.x; x < chunk_rows; x += kLutThreads) {
+        for (int64_t x = threadIdx.x; x < chunk_rows; x += LutCfg<KP>::threads) {
             const int64_t r = t_begin * 32 + x;
             if (r < N) store_y(Y, ydt, r, red[x]);
         }
@@ -392,7 +398,7 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
     const int rows = (int)chunk_rows;             // <= 32 * Nt, fits 32 bits
     __syncthreads();                              // red[] complete within the CTA
     {                                             // rows [x0(j), x1(j)) go to rank j
-        const int tpo = kLutThreads / CS;         // threads per destination rank
+        const int tpo = LutCfg<KP>::threads / CS;         // threads per destination rank
         const int j = threadIdx.x / tpo;
         if (j < CS) {
             const int jx0 = rows * j / CS, span = rows * (j + 1) / CS - jx0;
@@ -403,7 +409,7 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
     }
     cluster_sync_all();
     const int x0 = rows * rank / CS, my_span = rows * (rank + 1) / CS - x0;
-    for (int xo = threadIdx.x; xo < my_span; xo += kLutThreads) {
+    for (int xo = threadIdx.x; xo < my_span; xo += LutCfg<KP>::threads) {
         float y = 0.0f;
         for (int j = 0; j < CS; ++j) y += recv[j * my_span + xo];
         const int64_t r = t_begin * 32 + x0 + xo;
@@ -686,11 +692,12 @@ struct LutPlan {
     int smem;        // dynamic shared memory bytes
 };
 
-cudaLaunchConfig_t lut_config(const LutPlan& p, int count, cudaLaunchAttribute* attr, bool pdl, cudaStream_t stream)
+cudaLaunchConfig_t lut_config(const LutPlan& p, int count, int threads, cudaLaunchAttribute* attr, bool pdl,
+                              cudaStream_t stream)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(count * p.CS * p.R));
-    cfg.blockDim = dim3(kLutThreads);
+    cfg.blockDim = dim3((unsigned)threads);
     cfg.dynamicSmemBytes = (size_t)p.smem;
     cfg.stream = stream;
     int na = 0;
@@ -735,12 +742,12 @@ int lut_resident(int CS, int smem)
 {
     LutPlan p{CS, 1, smem};
     cudaLaunchAttribute attr[2];
-    cudaLaunchConfig_t cfg = lut_config(p, 1, attr, false, 0);
+    cudaLaunchConfig_t cfg = lut_config(p, 1, LutCfg<KP>::threads, attr, false, 0);
     int n = 0;
     if (CS > 1) {
         if (cudaOccupancyMaxActiveClusters(&n, gemv_lut_kernel<KP>, &cfg) != cudaSuccess) n = 0;
     } else {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_lut_kernel<KP>, kLutThreads, (size_t)smem) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_lut_kernel<KP>, LutCfg<KP>::threads, (size_t)smem) !=
             cudaSuccess)
             n = 0;
         n *= num_sms();
@@ -803,7 +810,7 @@ rb_status lut_plan_uncached(int N, int K, int count, LutPlan* plan)
             const int64_t units = (int64_t)count * R;
             const int64_t waves = (units + resident - 1) / resident;
             const int64_t tiles = (Nt + R - 1) / R;
-            const int64_t per_cta = spc * (kLutBuildTiles + (tiles + kLutWarps - 1) / kLutWarps * kLutWarps);
+            const int64_t per_cta = spc * (kLutBuildTiles + (tiles + LutCfg<KP>::warps - 1) / LutCfg<KP>::warps * LutCfg<KP>::warps);
             double cost = (double)(waves * per_cta);
             if (units < resident) cost *= 1.0 + 0.5 * (double)(resident - units) / (double)resident;
             if (cost < best_cost) {
@@ -875,7 +882,7 @@ rb_status launch_lut(const rb_layer_t* const* layers, const uint16_t* const* X, 
             b.Y[j] = Y[base + j];
         }
         cudaLaunchAttribute attr[2];
-        cudaLaunchConfig_t cfg = lut_config(plan, n, attr, pdl, stream);
+        cudaLaunchConfig_t cfg = lut_config(plan, n, LutCfg<KP>::threads, attr, pdl, stream);
         if (cudaLaunchKernelEx(&cfg, gemv_lut_kernel<KP>, b, (int)L0->n_out, (int)L0->k_in, plan.CS, plan.R, ydt) !=
             cudaSuccess)
             return RB_ERR_CUDA;
