@@ -247,7 +247,8 @@ def run_reference(args, dist: Dist):
     budget = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample(seconds_budget=0.5, max_layers=1)
-    cb, sec_per_layer = oracle_sample(seconds_budget=budget * args.steps, max_layers=max(1, args.steps))
+    # each step: about `budget` seconds of applications (a bounded sample of the step's 3072)
+    cb, sec_per_layer = oracle_sample(seconds_budget=budget * args.steps, max_layers=TOKENS * LAYERS * args.steps)
     line = assemble_line(value=cb["value"], unit="GB/s", n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
                          ms_per_step=sec_per_layer * LAYERS * TOKENS * 1e3,
                          extra={"impl": "reference", "config": config_dict(),
