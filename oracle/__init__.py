@@ -49,6 +49,10 @@ def _load():
         lib.oracle_pack_rows.restype = i32
         lib.oracle_apply.argtypes = [vp, vp, vp, i64, i64, i32, vp, i64, vp, i64, vp, i64, vp]
         lib.oracle_apply.restype = None
+        lib.oracle_transpose_planes.argtypes = [vp, i64, i64, i32, vp]
+        lib.oracle_transpose_planes.restype = None
+        lib.oracle_apply_t.argtypes = [vp, vp, vp, i64, i64, i32, vp, i64, vp]
+        lib.oracle_apply_t.restype = None
         lib.oracle_svid_greedy.argtypes = [vp, i64, i64, i32, i32, vp, vp]
         lib.oracle_svid_greedy.restype = i32
         lib.oracle_svid_iterative.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp]
@@ -140,6 +144,30 @@ def apply(planes, g16, h16, N: int, K: int, k: int, X_bf16, rows=None, toks=None
     _load().oracle_apply(_p(planes), _p(g16), _p(h16), N, K, k, _p(X), M,
                          _p(rows_a), nr, _p(toks_a), nt, _p(Y))
     return Y
+
+
+def transpose_planes(planes, N: int, K: int, k: int):
+    """Sign planes of the transposed (K x N) layer in the same storage layout.
+
+    The transposed layer's scales are the original ones exchanged (g' = h16,
+    h' = g16).  Returns uint32 [plane_words(K, N, k)].
+    """
+    planes = _c(planes, np.uint32)
+    out = np.zeros(max(plane_words(K, N, k), 1), np.uint32)
+    _load().oracle_transpose_planes(_p(planes), N, K, k, _p(out))
+    return out[:plane_words(K, N, k)]
+
+
+def apply_t(planes, g16, h16, N: int, K: int, k: int, dY_bf16):
+    """float64 input gradient dX = dY . What (dY bfloat16 bits [M][N]) -> [M][K]."""
+    planes = _c(planes, np.uint32)
+    g16 = _c(g16, np.uint16)
+    h16 = _c(h16, np.uint16)
+    dY = _c(dY_bf16, np.uint16)
+    M = dY.shape[0]
+    dX = np.zeros((M, K), np.float64)
+    _load().oracle_apply_t(_p(planes), _p(g16), _p(h16), N, K, k, _p(dY), M, _p(dX))
+    return dX
 
 
 def svid_greedy(W, k: int, iters: int = 20):

@@ -299,6 +299,61 @@ void oracle_apply(const uint32_t *planes, const uint16_t *g16, const uint16_t *h
 }
 
 /* ------------------------------------------------------------------ */
+/* Transposed layer and the input gradient (backward data path)          */
+/* ------------------------------------------------------------------ */
+
+/* Sign planes of the transposed layer: bit (i, c, r) of the K x N layer
+ * equals bit (i, r, c) of the N x K layer, written in the same storage
+ * layout (with N and K exchanged).  The scales of the transposed layer are
+ * the original ones exchanged, g' = h and h' = g, since
+ * What^T[c][r] = sum_i h_i[c] * B_i[r][c] * g_i[r].  out must hold
+ * oracle_plane_words(K, N, k) words and is cleared first. */
+void oracle_transpose_planes(const uint32_t *planes, int64_t N, int64_t K, int k, uint32_t *out)
+{
+    int64_t nw = oracle_plane_words(K, N, k);
+    for (int64_t x = 0; x < nw; ++x) out[x] = 0u;
+    for (int i = 0; i < k; ++i)
+        for (int64_t r = 0; r < N; ++r)
+            for (int64_t c = 0; c < K; ++c) {
+                uint32_t bit = (planes[word_index(N, K, i, r, c)] >> (c % 32)) & 1u;
+                out[word_index(K, N, i, c, r)] |= bit << (r % 32);
+            }
+}
+
+/* Input gradient of Y = X What^T (RaBiT, Algorithm 2 backward: the gradient
+ * reaching the layer input): dX[m][c] = sum_n dY[m][n] * What[n][c] in
+ * float64, What dequantised from the stored representation as in
+ * oracle_apply.  dY is [M][N] bfloat16 bit patterns; dX is [M][K]. */
+void oracle_apply_t(const uint32_t *planes, const uint16_t *g16, const uint16_t *h16,
+                    int64_t N, int64_t K, int k,
+                    const uint16_t *dY, int64_t M, double *dX)
+{
+    #pragma omp parallel
+    {
+        double *What = (double *)malloc(sizeof(double) * (size_t)N);
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t c = 0; c < K; ++c) {
+            for (int64_t n = 0; n < N; ++n) What[n] = 0.0;
+            for (int i = 0; i < k; ++i) {
+                double hc = decode_binary16(h16[(int64_t)i * K + c]);
+                for (int64_t n = 0; n < N; ++n) {
+                    uint32_t word = planes[word_index(N, K, i, n, c)];
+                    double s = ((word >> (c % 32)) & 1u) ? 1.0 : -1.0;
+                    What[n] += decode_binary16(g16[(int64_t)i * N + n]) * s * hc;
+                }
+            }
+            for (int64_t m = 0; m < M; ++m) {
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n)
+                    acc += decode_bfloat16(dY[m * N + n]) * What[n];
+                dX[m * K + c] = acc;
+            }
+        }
+        free(What);
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* Greedy SVID scales (rank-1 of |R_{i-1}| per plane, power iteration)   */
 /* ------------------------------------------------------------------ */
 

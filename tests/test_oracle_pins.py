@@ -354,3 +354,63 @@ def test_iterative_svid_matches_exact_svd_restatement(k, sweeps):
     for a, b in ((g, g_ref), (h, h_ref)):
         rel = np.abs(a.astype(np.float64) - b) / np.abs(b).max(axis=1, keepdims=True)
         assert rel.max() < 1e-5, rel.max()
+
+
+# ---------------------------------------------------------------- transposed layer, input gradient
+# shapes: N a multiple of 32 (the transposed layer's input width); N and K not
+# multiples of 256 so both layouts have a ragged last slice and row-tile group.
+_T_SHAPES = [(32, 32, 1), (96, 320, 2), (288, 800, 3), (64, 1056, 4)]
+
+
+@pytest.mark.parametrize("N,K,k", _T_SHAPES)
+def test_transposed_planes_equal_planes_of_transposed_weight(N, K, k):
+    """The recurrence is element-wise and fl(g*h) = fl(h*g), so the planes of
+    (W, g, h) transposed are exactly the planes derived from (W^T, h, g)."""
+    rng = np.random.default_rng(N + K + k)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[rng.random((N, K)) < 0.01] = 0.0                     # sign(0) ties take part too
+    g, h = synth.positive_scales(k, N, K, seed=k)
+    planes, g16, h16, st, _ = oracle.pack(W, g, h, k)
+    planes_t2, g16_t, h16_t, st_t, _ = oracle.pack(np.ascontiguousarray(W.T), h, g, k)
+    assert st == 0 and st_t == 0
+    assert np.array_equal(oracle.transpose_planes(planes, N, K, k), planes_t2)
+    assert np.array_equal(g16_t, h16) and np.array_equal(h16_t, g16)
+
+
+@pytest.mark.parametrize("N,K,k", _T_SHAPES)
+def test_transpose_is_the_bit_matrix_transpose(N, K, k):
+    """Against the numpy layout helpers: unpacking the transposed planes gives
+    the transposed sign matrices, padding stays zero, and a second transpose
+    (allowed when K is a multiple of 32) restores the planes."""
+    rng = np.random.default_rng(3 * N + K)
+    B = rng.random((k, N, K)) < 0.5
+    planes = layout.pack_bits(B)
+    pt = oracle.transpose_planes(planes, N, K, k)
+    assert np.array_equal(layout.unpack_bits(pt, K, N, k), B.transpose(0, 2, 1))
+    assert not layout.padding_words_and_bits(pt, K, N, k).any()
+    assert np.array_equal(oracle.transpose_planes(pt, K, N, k), planes)
+
+
+def test_input_gradient_matches_dense_product_and_adjoint():
+    """dX = dY . What: equal to numpy's product with the dense What built from
+    the layout helpers; equal to the forward oracle on the transposed layer;
+    and <dY, X What^T> = <dY What, X> (the adjoint identity)."""
+    rng = np.random.default_rng(21)
+    N, K, k, M = 96, 320, 2, 3
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    dY = synth.activations(M, N, seed=5)
+    X = synth.activations(M, K, seed=6)
+    dX = oracle.apply_t(planes, g16, h16, N, K, k, dY)
+    B = np.where(layout.unpack_bits(planes, N, K, k), 1.0, -1.0)
+    gq = g16.view(np.float16).astype(np.float64)
+    hq = h16.view(np.float16).astype(np.float64)
+    What = np.einsum("in,inc,ic->nc", gq, B, hq)
+    assert np.allclose(dX, bf16_to_f64(dY) @ What, rtol=1e-12, atol=1e-15)
+    via_t = oracle.apply(oracle.transpose_planes(planes, N, K, k), h16, g16, K, N, k, dY)
+    assert np.allclose(dX, via_t, rtol=1e-12, atol=1e-15)
+    Y = oracle.apply(planes, g16, h16, N, K, k, X)
+    lhs = float(np.sum(bf16_to_f64(dY) * Y))
+    rhs = float(np.sum(dX * bf16_to_f64(X)))
+    assert math.isclose(lhs, rhs, rel_tol=1e-11, abs_tol=1e-14)
