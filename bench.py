@@ -503,7 +503,23 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
                     stream)
     out["gemv_M64_tcgen05"] = {"us": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
                                "TFLOPs": 2.0 * 64 * N_OUT * K_IN * K_PLANES / t / 1e12}
-    del layers
+    # backward data path: rb_transpose_planes over the 96 layers (reads and writes the
+    # planes once), then the input gradient dX = dY . What of one token per layer
+    # through rb_gemv_batch on the transposed layers
+    tlayers = [rbw.transpose(L, stream=stream) for L in layers]
+    itt = iter(range(10 ** 9))
+
+    def tr():
+        j = next(itt) % LAYERS
+        rbw.transpose(layers[j], out=tlayers[j], stream=stream)
+    t = time_events(torch, tr, 2 * LAYERS, stream)
+    out["transpose_planes"] = {"us": t * 1e6, "GBps": 2 * Lp.packed_bytes() / t / 1e9,
+                               "bytes": 2 * Lp.packed_bytes()}
+    dY = torch.from_numpy(synth.activations(1, N_OUT, seed=11).view(np.int16)).to(dev)
+    dXs = [torch.empty(1, K_IN, dtype=torch.float32, device=dev) for _ in range(LAYERS)]
+    t = time_events(torch, lambda: rbw.gemv_batch(tlayers, [dY] * LAYERS, dXs, stream=stream), 5, stream) / LAYERS
+    out["input_grad_M1_batch96"] = {"us_per_layer": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9}
+    del layers, tlayers
     # rb_gemm at M = 2048 on the prefill shape
     try:
         X = torch.from_numpy(synth.activations(2048, K_IN, seed=7).view(np.int16)).to(dev)

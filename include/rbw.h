@@ -195,6 +195,24 @@ RB_API rb_status rb_gemm_noalloc(const rb_layer_t *layer, const uint16_t *X, int
                                  cudaStream_t stream);
 
 /*
+ * rb_transpose_planes -- sign planes of the transposed layer, for the
+ * gradient that reaches the layer input in training (RaBiT, Algorithm 2
+ * backward pass): dX = dY . What.  Since What^T = sum_i diag(h_i) B_i^T
+ * diag(g_i), the K x N layer {n_out = K, k_in = N, k, planes_t, g16 = h16,
+ * h16 = g16} (the same scale arrays, exchanged) is a packed layer whose
+ * forward product is the input gradient: rb_gemv / rb_gemm on it with
+ * X = dY ([M][N] bfloat16) give dX [M][K].
+ *   layer     the forward layer (N x K); N must be a multiple of 32
+ *             (RB_ERR_SHAPE otherwise), as it becomes the input width.
+ *   planes_t  out, rb_packed_words(K, N, k) uint32 words in the storage
+ *             layout of a K x N layer; every word is written.  It must not
+ *             overlap layer->planes (RB_ERR_ARG).
+ * The bits are exactly those rb_pack derives from (W^T, h, g): the
+ * recurrence is element-wise and fl(g h) = fl(h g).
+ */
+RB_API rb_status rb_transpose_planes(const rb_layer_t *layer, uint32_t *planes_t, cudaStream_t stream);
+
+/*
  * rb_svid_greedy -- greedy SVID scales for each plane (RaBiT names Greedy
  * SVID as the traditional initialiser): for i = 1..k, (g_i, h_i) is the
  * rank-1 approximation of |R_{i-1}| by `iters` rounds of power iteration in

@@ -33,6 +33,7 @@ SIGNATURES = {
     "rb_gemm_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
     "rb_gemm": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _u32, _vp]),
     "rb_gemm_noalloc": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _u32, _vp]),
+    "rb_transpose_planes": (_i32, [_vp, _vp, _vp]),
     "rb_svid_workspace_bytes": (_sz, [_i32, _i32]),
     "rb_svid_greedy": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "rb_svid_iterative_workspace_bytes": (_sz, [_i32, _i32, _i32]),
@@ -184,6 +185,26 @@ def gemm_noalloc(layer: PackedLayer, X, Y=None, flags=0, dev_status=None, stream
                                _stream(stream))
     _check("rb_gemm_noalloc", st)
     return Y
+
+
+def transpose(layer: PackedLayer, out: PackedLayer | None = None, stream=None):
+    """rb_transpose_planes: the K x N layer of What^T (new planes, or out's; the
+    scale tensors are shared with `layer`, exchanged).  Its forward product is
+    the input gradient: gemv/gemm(transpose(layer), dY) = dY . What."""
+    if out is None:
+        out = PackedLayer.__new__(PackedLayer)
+        out.n_out, out.k_in, out.k_planes = layer.k_in, layer.n_out, layer.k_planes
+        nw = packed_words(out.n_out, out.k_in, out.k_planes)
+        if nw == 0:
+            raise ValueError("invalid layer shape")
+        out.planes = torch.empty(nw, dtype=torch.int32, device=layer.planes.device)
+    elif (out.n_out, out.k_in, out.k_planes) != (layer.k_in, layer.n_out, layer.k_planes):
+        raise ValueError("out is not shaped as the transposed layer")
+    out.g16, out.h16 = layer.h16, layer.g16
+    L = layer.struct()
+    st = lib().rb_transpose_planes(ctypes.byref(L), _ptr(out.planes), _stream(stream))
+    _check("rb_transpose_planes", st)
+    return out
 
 
 def svid_greedy(W, k_planes, iters=20, ws=None, stream=None):

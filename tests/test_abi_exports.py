@@ -94,6 +94,19 @@ def test_apply_argument_errors_on_host(L):
     assert L.rb_gemv(ctypes.byref(lay), a, 1, a, 0, None, 0, None, 2, None) == rbw.RB_ERR_ARG
 
 
+def test_transpose_argument_errors_on_host(L):
+    lay = rbw.RbLayer(64, 256, 2, 0, 0x10000, 0x10000, 0x10000)
+    dst = _fake(0x100000)
+    assert L.rb_transpose_planes(None, dst, None) == rbw.RB_ERR_ARG
+    assert L.rb_transpose_planes(ctypes.byref(lay), None, None) == rbw.RB_ERR_ARG
+    ragged_n = rbw.RbLayer(48, 256, 2, 0, 0x10000, 0x10000, 0x10000)    # N becomes the input width
+    assert L.rb_transpose_planes(ctypes.byref(ragged_n), dst, None) == rbw.RB_ERR_SHAPE
+    assert L.rb_transpose_planes(ctypes.byref(lay), _fake(0x100008), None) == rbw.RB_ERR_ALIGN
+    # 2 planes x 1 slice x 2 tiles = 4 KB from 0x10000: a destination inside it overlaps
+    assert L.rb_transpose_planes(ctypes.byref(lay), _fake(0x10400), None) == rbw.RB_ERR_ARG
+    assert L.rb_transpose_planes(ctypes.byref(lay), dst, None) == rbw.RB_ERR_UNSUPPORTED
+
+
 def test_svid_argument_errors_on_host(L):
     a = _fake(0x10000)
     assert L.rb_svid_greedy(a, 4, 64, 1, 20, a, a, None, 0, None) == rbw.RB_ERR_ARG
