@@ -948,7 +948,9 @@ template <int KP>
 rb_status launch_mma(const rb_layer_t* const* layers, const uint16_t* const* X, void* const* Y, int count, int M,
                      int ydt, bool pdl, cudaStream_t stream)
 {
-    constexpr int NTMAX = KP <= 2 ? 4 : (KP <= 4 ? 2 : 1);
+    // 16 tokens per CTA at most: at k <= 2 two such CTAs share an SM, which beats one
+    // 32-token CTA per SM (4096 x 4096, k = 2, 96 layers at M = 64: 17.1 vs 24.8 us)
+    constexpr int NTMAX = KP <= 4 ? 2 : 1;
     const rb_layer_t* L0 = layers[0];
     for (int base = 0; base < count; base += kMaxBatch) {
         const int n = count - base < kMaxBatch ? count - base : kMaxBatch;
@@ -962,9 +964,7 @@ rb_status launch_mma(const rb_layer_t* const* layers, const uint16_t* const* X, 
         }
         const int need = (M + 7) / 8;                 // n-tiles for all tokens in one group
         rb_status st;
-        if (need >= 4 && NTMAX >= 4)
-            st = launch_mma_nt<KP, (NTMAX >= 4 ? 4 : 1)>(b, n, L0->n_out, L0->k_in, M, ydt, pdl, stream);
-        else if (need >= 2 && NTMAX >= 2)
+        if (need >= 2 && NTMAX >= 2)
             st = launch_mma_nt<KP, (NTMAX >= 2 ? 2 : 1)>(b, n, L0->n_out, L0->k_in, M, ydt, pdl, stream);
         else
             st = launch_mma_nt<KP, 1>(b, n, L0->n_out, L0->k_in, M, ydt, pdl, stream);
