@@ -91,14 +91,17 @@ def packed_words(n_out, k_in, k_planes):
 class PackedLayer:
     """Device tensors of one packed layer (owns them) plus its rb_layer_t view."""
 
-    def __init__(self, n_out, k_in, k_planes, device="cuda"):
+    def __init__(self, n_out, k_in, k_planes, device="cuda", g16=None, h16=None):
+        """New planes; new scale tensors unless existing ones are passed to share."""
         nw = packed_words(n_out, k_in, k_planes)
         if nw == 0:
             raise ValueError("invalid layer shape")
         self.n_out, self.k_in, self.k_planes = n_out, k_in, k_planes
         self.planes = torch.empty(nw, dtype=torch.int32, device=device)
-        self.g16 = torch.empty(k_planes, n_out, dtype=torch.float16, device=device)
-        self.h16 = torch.empty(k_planes, k_in, dtype=torch.float16, device=device)
+        self.g16 = torch.empty(k_planes, n_out, dtype=torch.float16, device=device) if g16 is None else g16
+        self.h16 = torch.empty(k_planes, k_in, dtype=torch.float16, device=device) if h16 is None else h16
+        if tuple(self.g16.shape) != (k_planes, n_out) or tuple(self.h16.shape) != (k_planes, k_in):
+            raise ValueError("scale tensors do not match the layer shape")
 
     def struct(self):
         return RbLayer(self.n_out, self.k_in, self.k_planes, 0, self.planes.data_ptr(),
@@ -192,15 +195,11 @@ def transpose(layer: PackedLayer, out: PackedLayer | None = None, stream=None):
     scale tensors are shared with `layer`, exchanged).  Its forward product is
     the input gradient: gemv/gemm(transpose(layer), dY) = dY . What."""
     if out is None:
-        out = PackedLayer.__new__(PackedLayer)
-        out.n_out, out.k_in, out.k_planes = layer.k_in, layer.n_out, layer.k_planes
-        nw = packed_words(out.n_out, out.k_in, out.k_planes)
-        if nw == 0:
-            raise ValueError("invalid layer shape")
-        out.planes = torch.empty(nw, dtype=torch.int32, device=layer.planes.device)
+        out = PackedLayer(layer.k_in, layer.n_out, layer.k_planes, layer.planes.device, g16=layer.h16, h16=layer.g16)
     elif (out.n_out, out.k_in, out.k_planes) != (layer.k_in, layer.n_out, layer.k_planes):
         raise ValueError("out is not shaped as the transposed layer")
-    out.g16, out.h16 = layer.h16, layer.g16
+    else:
+        out.g16, out.h16 = layer.h16, layer.g16
     L = layer.struct()
     st = lib().rb_transpose_planes(ctypes.byref(L), _ptr(out.planes), _stream(stream))
     _check("rb_transpose_planes", st)

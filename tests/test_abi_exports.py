@@ -9,8 +9,10 @@
 import ctypes
 import os
 import re
+import types
 
 import pytest
+import torch
 
 import oracle
 from residual_binarized_weight_b200 import build as rbw_build
@@ -125,3 +127,17 @@ def test_product_does_not_import_oracle():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "rb_oracle" not in txt, f
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_binding_fails_loudly_without_a_device():
+    """The binding marshals host tensors' pointers and the library refuses to
+    run without an sm_100 device: no CPU fallback."""
+    L = rbw.PackedLayer(64, 256, 2, "cpu")
+    with pytest.raises(rbw.RbError) as e:
+        rbw.transpose(L, stream=types.SimpleNamespace(cuda_stream=0))
+    assert e.value.status == rbw.RB_ERR_UNSUPPORTED
+    X = torch.zeros(1, 256, dtype=torch.int16)
+    with pytest.raises(rbw.RbError) as e:
+        rbw.gemv(L, X, Y=torch.empty(1, 64), stream=types.SimpleNamespace(cuda_stream=0))
+    assert e.value.status == rbw.RB_ERR_UNSUPPORTED
