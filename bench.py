@@ -459,13 +459,40 @@ def time_events(torch, fn, reps, stream):
     return e0.elapsed_time(e1) / 1e3 / reps
 
 
+def time_graph_calls(torch, fn, reps, stream):
+    """Per-call device time of `fn` with the host out of the way: `reps` calls are
+    captured into one CUDA graph (after an eager call), which is replayed after
+    warm-up between CUDA events on `stream`."""
+    with torch.cuda.stream(stream):
+        fn()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=stream):
+        for _ in range(reps):
+            fn()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(5):
+            gr.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / (5 * reps)
+    del gr
+    return t
+
+
 def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
     """Device timings of the other hot-path steps on the same layer (kernels only)."""
     out = {}
     stream = torch.cuda.Stream(dev)
     # rb_pack: reads W (4NK bytes), writes planes + fp16 scales
     Lp = rbw.PackedLayer(N_OUT, K_IN, K_PLANES, dev)
-    t = time_events(torch, lambda: rbw.pack(W, g, h, K_PLANES, out=Lp, stream=stream), 20, stream)
+    t = time_graph_calls(torch, lambda: rbw.pack(W, g, h, K_PLANES, out=Lp, stream=stream), 20, stream)
     pack_bytes = 4 * N_OUT * K_IN + Lp.packed_bytes() + 2 * K_PLANES * (N_OUT + K_IN)
     out["pack"] = {"us": t * 1e6, "GBps": pack_bytes / t / 1e9, "bytes": pack_bytes}
     # rb_gemv at M = 4 and 16 over 96 distinct layers (L2-defeating), plain launches
@@ -487,20 +514,46 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
         t = time_events(torch, f, 2 * LAYERS, stream)
         out["gemv_M%d_plain_launches" % M] = {"us": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
                                "tokens_per_s": M / t}
+    # isolated single-layer launch at M = 1: a write of 2 x L2 bytes before each launch
+    # evicts the planes, and the launch alone sits between the events (the figures above
+    # are sustained: back-to-back launches over layers that do not fit in L2)
+    try:
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+        X1 = torch.from_numpy(synth.activations(1, K_IN, seed=1).view(np.int16)).to(dev)
+        Y1 = torch.empty(1, N_OUT, dtype=torch.float32, device=dev)
+        ts = []
+        with torch.cuda.stream(stream):
+            for r in range(23):
+                flush.fill_(r & 0xFF)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                rbw.gemv(layers[r % LAYERS], X1, Y=Y1, stream=stream)
+                e1.record(stream)
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3)
+        ts = sorted(ts[3:])
+        med = ts[len(ts) // 2]
+        out["gemv_M1_isolated"] = {"us_median": med, "packed_GBps": Lp.packed_bytes() / med / 1e3,
+                                   "flush_bytes": 2 * l2, "launches": len(ts)}
+        del flush
+    except Exception as e:                       # an informational row: record why it is missing
+        out["gemv_M1_isolated"] = {"unavailable": repr(e)[:200]}
     # rb_gemv_batch at M = 4 and 16 (one tensor-core launch over the 96 layers), and
     # rb_gemv at M = 64 with its workspace (tcgen05 kernel), 96 distinct layers
     for M in (4, 16):
         X = torch.from_numpy(synth.activations(M, K_IN, seed=M).view(np.int16)).to(dev)
         Ys = [torch.empty(M, N_OUT, dtype=torch.float32, device=dev) for _ in range(LAYERS)]
-        t = time_events(torch, lambda: rbw.gemv_batch(layers, [X] * LAYERS, Ys, stream=stream), 5, stream) / LAYERS
+        t = time_graph_calls(torch, lambda: rbw.gemv_batch(layers, [X] * LAYERS, Ys, stream=stream), 5,
+                             stream) / LAYERS
         out["gemv_M%d_batch96" % M] = {"us_per_layer": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
                                        "TFLOPs": 2.0 * M * N_OUT * K_IN * K_PLANES / t / 1e12}
     X = torch.from_numpy(synth.activations(64, K_IN, seed=64).view(np.int16)).to(dev)
     Y = torch.empty(64, N_OUT, dtype=torch.float32, device=dev)
     ws = rbw.workspace(rbw.gemv_workspace_bytes(N_OUT, K_IN, K_PLANES, 64), dev)
     it64 = iter(range(10 ** 9))
-    t = time_events(torch, lambda: rbw.gemv(layers[next(it64) % LAYERS], X, Y=Y, ws=ws, stream=stream), 2 * LAYERS,
-                    stream)
+    t = time_graph_calls(torch, lambda: rbw.gemv(layers[next(it64) % LAYERS], X, Y=Y, ws=ws, stream=stream),
+                         2 * LAYERS, stream)
     out["gemv_M64_tcgen05"] = {"us": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
                                "TFLOPs": 2.0 * 64 * N_OUT * K_IN * K_PLANES / t / 1e12}
     # backward data path: rb_transpose_planes over the 96 layers (reads and writes the
@@ -512,12 +565,13 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
     def tr():
         j = next(itt) % LAYERS
         rbw.transpose(layers[j], out=tlayers[j], stream=stream)
-    t = time_events(torch, tr, 2 * LAYERS, stream)
+    t = time_graph_calls(torch, tr, 2 * LAYERS, stream)
     out["transpose_planes"] = {"us": t * 1e6, "GBps": 2 * Lp.packed_bytes() / t / 1e9,
                                "bytes": 2 * Lp.packed_bytes()}
     dY = torch.from_numpy(synth.activations(1, N_OUT, seed=11).view(np.int16)).to(dev)
     dXs = [torch.empty(1, K_IN, dtype=torch.float32, device=dev) for _ in range(LAYERS)]
-    t = time_events(torch, lambda: rbw.gemv_batch(tlayers, [dY] * LAYERS, dXs, stream=stream), 5, stream) / LAYERS
+    t = time_graph_calls(torch, lambda: rbw.gemv_batch(tlayers, [dY] * LAYERS, dXs, stream=stream), 5,
+                         stream) / LAYERS
     out["input_grad_M1_batch96"] = {"us_per_layer": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9}
     del layers, tlayers
     # rb_gemm at M = 2048 on the prefill shape
@@ -556,7 +610,8 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
     def batch_time(ls, M, seed):
         X = torch.from_numpy(synth.activations(M, ls[0].k_in, seed=seed).view(np.int16)).to(dev)
         Ys = [torch.empty(M, ls[0].n_out, dtype=torch.float32, device=dev) for _ in ls]
-        return time_events(torch, lambda: rbw.gemv_batch(ls, [X] * len(ls), Ys, stream=stream), 5, stream) / len(ls)
+        return time_graph_calls(torch, lambda: rbw.gemv_batch(ls, [X] * len(ls), Ys, stream=stream), 5,
+                                stream) / len(ls)
 
     wl3 = synth.workload("mlp_trio_7b_k2")
     trio = {layer.name: layer_copies(layer, K_PLANES) for layer in wl3.layers}
