@@ -216,6 +216,17 @@ def profiled_traffic(kernel_tag: str):
 
 
 # ---------------------------------------------------------------- CPU oracle legs
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def oracle_sample(seconds_budget=12.0, max_layers=TOKENS * LAYERS):
     """Time the oracle's float64 apply on the workload layer: applications until
     about seconds_budget of CPU work has run, at most one step's worth."""
@@ -235,8 +246,8 @@ def oracle_sample(seconds_budget=12.0, max_layers=TOKENS * LAYERS):
         if time.perf_counter() - t0 > seconds_budget:
             break
     dt = time.perf_counter() - t0
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": plane_bytes * n / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+    return {"value": plane_bytes * n / dt / 1e9, "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
+            "cpu_model": cpu_model(), "nproc": os.cpu_count(),
             "sample": "%d single-token (M=1) applications of one %dx%d k=%d layer, float64 dequantise-then-multiply, %.1f s"
                       % (n, N_OUT, K_IN, K_PLANES, dt)}, dt / n
 

@@ -49,6 +49,8 @@ def _load():
         lib.oracle_pack_rows.restype = i32
         lib.oracle_apply.argtypes = [vp, vp, vp, i64, i64, i32, vp, i64, vp, i64, vp, i64, vp]
         lib.oracle_apply.restype = None
+        lib.oracle_threads.argtypes = []
+        lib.oracle_threads.restype = i32
         lib.oracle_transpose_planes.argtypes = [vp, i64, i64, i32, vp]
         lib.oracle_transpose_planes.restype = None
         lib.oracle_apply_t.argtypes = [vp, vp, vp, i64, i64, i32, vp, i64, vp]
@@ -77,6 +79,11 @@ def _p(a: np.ndarray | None):
 
 def _c(a, dtype):
     return np.ascontiguousarray(a, dtype=dtype)
+
+
+def threads() -> int:
+    """OpenMP threads the oracle's parallel loops use."""
+    return int(_load().oracle_threads())
 
 
 def plane_words(N: int, K: int, k: int) -> int:

@@ -126,6 +126,9 @@ static double decode_bfloat16(uint16_t b)
     return (double)f;
 }
 
+/* OpenMP threads a parallel region of this library runs on (for reporting). */
+int oracle_threads(void) { return omp_get_max_threads(); }
+
 uint16_t oracle_f64_to_f16(double v) { return encode_binary16(v); }
 double oracle_f16_to_f64(uint16_t b) { return decode_binary16(b); }
 uint16_t oracle_f64_to_bf16(double v) { return encode_bfloat16(v); }
