@@ -49,6 +49,8 @@ def _load():
         lib.oracle_pack_rows.restype = i32
         lib.oracle_apply.argtypes = [vp, vp, vp, i64, i64, i32, vp, i64, vp, i64, vp, i64, vp]
         lib.oracle_apply.restype = None
+        lib.oracle_qat_backward.argtypes = [vp, vp, vp, i64, i64, i32, vp, vp, i64, vp, vp, vp, vp]
+        lib.oracle_qat_backward.restype = i32
         lib.oracle_threads.argtypes = []
         lib.oracle_threads.restype = i32
         lib.oracle_transpose_planes.argtypes = [vp, i64, i64, i32, vp]
@@ -175,6 +177,27 @@ def apply_t(planes, g16, h16, N: int, K: int, k: int, dY_bf16):
     dX = np.zeros((M, K), np.float64)
     _load().oracle_apply_t(_p(planes), _p(g16), _p(h16), N, K, k, _p(dY), M, _p(dX))
     return dX
+
+
+def qat_backward(W, g, h, k: int, X_bf16, dY_bf16):
+    """float64 gradients of the coupled-training layer (signs derived from W by
+    the fp32 recurrence and held constant): returns (status, dW [N][K],
+    dg [k][N], dh [k][K], dX [M][K])."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    g = _c(g, np.float32).reshape(k, N)
+    h = _c(h, np.float32).reshape(k, K)
+    X = _c(X_bf16, np.uint16)
+    dY = _c(dY_bf16, np.uint16)
+    M = X.shape[0]
+    assert dY.shape == (M, N)
+    dW = np.zeros((N, K), np.float64)
+    dg = np.zeros((k, N), np.float64)
+    dh = np.zeros((k, K), np.float64)
+    dX = np.zeros((M, K), np.float64)
+    st = _load().oracle_qat_backward(_p(W), _p(g), _p(h), N, K, k, _p(X), _p(dY), M,
+                                     _p(dW), _p(dg), _p(dh), _p(dX))
+    return int(st), dW, dg, dh, dX
 
 
 def svid_greedy(W, k: int, iters: int = 20):

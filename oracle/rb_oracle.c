@@ -357,6 +357,90 @@ void oracle_apply_t(const uint32_t *planes, const uint16_t *g16, const uint16_t 
 }
 
 /* ------------------------------------------------------------------ */
+/* Coupled training: gradients of one layer (Algorithm 2 backward)       */
+/* ------------------------------------------------------------------ */
+
+/* Gradients of a loss L through Y = X What^T with What = sum_i diag(g_i) B_i
+ * diag(h_i) (RaBiT, Algorithm 2: the signs B_i are derived on the fly from W
+ * by the fp32 recurrence of oracle_pack and held constant in the backward
+ * pass; the latent weight takes the effective-weight gradient).  Given
+ * dY = dL/dY, in float64:
+ *   G[n][c]  = sum_m dY[m][n] X[m][c]              (dL/dWhat = dY^T X)
+ *   dW       = G
+ *   dg_i[n]  = sum_c G[n][c] B_i[n][c] h_i[c]
+ *   dh_i[c]  = sum_n G[n][c] g_i[n] B_i[n][c]
+ *   dX[m][c] = sum_n dY[m][n] What[n][c]           (fp32 scales, as trained)
+ * X [M][K] and dY [M][N] are bfloat16 bit patterns; dW [N][K] and dX [M][K]
+ * are nullable; dg [k][N], dh [k][K].  Returns oracle_pack's status codes
+ * (-1 bad arguments, 1 non-finite input; fp16 range is not checked here). */
+int oracle_qat_backward(const float *W, const float *g, const float *h,
+                        int64_t N, int64_t K, int k,
+                        const uint16_t *X, const uint16_t *dY, int64_t M,
+                        double *dW, double *dg, double *dh, double *dX)
+{
+    if (check_args(N, K, k) || M < 1) return -1;
+    int st = scan_inputs(W, g, h, N, K, k, NULL, NULL) == 1 ? 1 : 0;
+    unsigned char *B = (unsigned char *)malloc((size_t)k * (size_t)N * (size_t)K);
+    double *G = (double *)malloc(sizeof(double) * (size_t)(N * K));
+    #pragma omp parallel
+    {
+        float *R = (float *)malloc(sizeof(float) * (size_t)K);
+        unsigned char *bits = (unsigned char *)malloc((size_t)k * (size_t)K);
+        #pragma omp for schedule(static)
+        for (int64_t r = 0; r < N; ++r) {
+            derive_row(W + r * K, g, h, N, K, k, r, R, bits);
+            for (int i = 0; i < k; ++i)
+                memcpy(B + ((int64_t)i * N + r) * K, bits + (int64_t)i * K, (size_t)K);
+            for (int64_t c = 0; c < K; ++c) {
+                double acc = 0.0;
+                for (int64_t m = 0; m < M; ++m)
+                    acc += decode_bfloat16(dY[m * N + r]) * decode_bfloat16(X[m * K + c]);
+                G[r * K + c] = acc;
+            }
+        }
+        free(R);
+        free(bits);
+    }
+    if (dW) memcpy(dW, G, sizeof(double) * (size_t)(N * K));
+    for (int i = 0; i < k; ++i) {
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < K; ++c) {
+                double s = B[((int64_t)i * N + n) * K + c] ? 1.0 : -1.0;
+                acc += G[n * K + c] * s * (double)h[(int64_t)i * K + c];
+            }
+            dg[(int64_t)i * N + n] = acc;
+        }
+        for (int64_t c = 0; c < K; ++c) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                double s = B[((int64_t)i * N + n) * K + c] ? 1.0 : -1.0;
+                acc += G[n * K + c] * (double)g[(int64_t)i * N + n] * s;
+            }
+            dh[(int64_t)i * K + c] = acc;
+        }
+    }
+    if (dX) {
+        for (int64_t m = 0; m < M; ++m)
+            for (int64_t c = 0; c < K; ++c) {
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    double w = 0.0;
+                    for (int i = 0; i < k; ++i) {
+                        double s = B[((int64_t)i * N + n) * K + c] ? 1.0 : -1.0;
+                        w += (double)g[(int64_t)i * N + n] * s * (double)h[(int64_t)i * K + c];
+                    }
+                    acc += decode_bfloat16(dY[m * N + n]) * w;
+                }
+                dX[m * K + c] = acc;
+            }
+    }
+    free(G);
+    free(B);
+    return st;
+}
+
+/* ------------------------------------------------------------------ */
 /* Greedy SVID scales (rank-1 of |R_{i-1}| per plane, power iteration)   */
 /* ------------------------------------------------------------------ */
 

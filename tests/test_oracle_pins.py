@@ -414,3 +414,78 @@ def test_input_gradient_matches_dense_product_and_adjoint():
     lhs = float(np.sum(bf16_to_f64(dY) * Y))
     rhs = float(np.sum(dX * bf16_to_f64(X)))
     assert math.isclose(lhs, rhs, rel_tol=1e-11, abs_tol=1e-14)
+
+
+# ---------------------------------------------------------------- coupled-training gradients
+def _loss_parts(W, g, h, k, X, dY):
+    """Dense float64 pieces of L = <dY, X What^T> with the signs of the fp32
+    recurrence (from oracle.pack through the numpy layout helpers)."""
+    N, K = W.shape
+    planes = oracle.pack(W, g, h, k)[0]
+    S = np.where(layout.unpack_bits(planes, N, K, k), 1.0, -1.0)      # [k][N][K]
+    xf, dyf = bf16_to_f64(X), bf16_to_f64(dY)
+
+    def loss(gg, hh, xx=xf):
+        What = np.einsum("in,inc,ic->nc", gg, S, hh)
+        return float(np.sum(dyf * (xx @ What.T)))
+    return S, xf, dyf, loss
+
+
+def test_qat_gradients_match_central_differences():
+    """L is linear in each g_i[n], each h_i[c], in What and in X, so central
+    differences with a large step are exact up to rounding: they pin dg, dh,
+    dW (= dL/dWhat, passed to the latent weight) and dX."""
+    rng = np.random.default_rng(31)
+    N, K, k, M = 12, 96, 3, 4
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=10)
+    X = synth.activations(M, K, seed=2)
+    dY = synth.activations(M, N, seed=3)
+    st, dW, dg, dh, dX = oracle.qat_backward(W, g, h, k, X, dY)
+    assert st == 0
+    S, xf, dyf, loss = _loss_parts(W, g, h, k, X, dY)
+    g64, h64 = g.astype(np.float64), h.astype(np.float64)
+    scale = abs(loss(g64, h64)) + float(np.abs(dyf).sum() * np.abs(xf).max())
+    d = 0.5
+    for i, n in [(0, 0), (1, 5), (2, N - 1)]:
+        e = np.zeros_like(g64)
+        e[i, n] = d
+        fd = (loss(g64 + e, h64) - loss(g64 - e, h64)) / (2 * d)
+        assert math.isclose(dg[i, n], fd, rel_tol=1e-9, abs_tol=1e-12 * scale)
+    for i, c in [(0, 0), (1, 40), (2, K - 1)]:
+        e = np.zeros_like(h64)
+        e[i, c] = d
+        fd = (loss(g64, h64 + e) - loss(g64, h64 - e)) / (2 * d)
+        assert math.isclose(dh[i, c], fd, rel_tol=1e-9, abs_tol=1e-12 * scale)
+    What = np.einsum("in,inc,ic->nc", g64, S, h64)
+    V = rng.standard_normal((N, K))
+    fd = (np.sum(dyf * (xf @ (What + d * V).T)) - np.sum(dyf * (xf @ (What - d * V).T))) / (2 * d)
+    assert math.isclose(float(np.sum(dW * V)), float(fd), rel_tol=1e-9, abs_tol=1e-12 * scale)
+    U = rng.standard_normal((M, K))
+    fd = (loss(g64, h64, xf + d * U) - loss(g64, h64, xf - d * U)) / (2 * d)
+    assert math.isclose(float(np.sum(dX * U)), float(fd), rel_tol=1e-9, abs_tol=1e-12 * scale)
+
+
+def test_qat_gradients_agree_with_the_deployment_oracle():
+    """With scales exactly representable in fp16 the training-time gradients
+    reach the same numbers through the stored representation: dX equals
+    oracle.apply_t, and dg_i[n] = sum_m dY[m][n] * (B_i (h_i . x_m))[n], the
+    latter from oracle.apply on plane i alone with unit g."""
+    rng = np.random.default_rng(32)
+    N, K, k, M = 32, 320, 2, 3
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=10)
+    g = g.astype(np.float16).astype(np.float32)
+    h = h.astype(np.float16).astype(np.float32)
+    X = synth.activations(M, K, seed=4)
+    dY = synth.activations(M, N, seed=5)
+    st, _, dg, _, dX = oracle.qat_backward(W, g, h, k, X, dY)
+    planes, g16, h16, st2, _ = oracle.pack(W, g, h, k)
+    assert st == 0 and st2 == 0
+    assert np.allclose(dX, oracle.apply_t(planes, g16, h16, N, K, k, dY), rtol=1e-12, atol=1e-15)
+    per_plane = oracle.plane_words(N, K, 1)
+    ones = np.full((1, N), oracle.f64_to_f16_bits(1.0), np.uint16)
+    for i in range(k):
+        Yi = oracle.apply(planes[i * per_plane:(i + 1) * per_plane], ones, h16[i:i + 1], N, K, 1, X)
+        want = np.sum(bf16_to_f64(dY) * Yi, axis=0)
+        assert np.allclose(dg[i], want, rtol=1e-12, atol=1e-15)
