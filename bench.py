@@ -121,6 +121,19 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
 REJECT_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
 
 
+def clocks_rejected(clocks) -> bool:
+    """A timed region that saw thermal or hardware slowdown, or whose median SM
+    clock sat well below the maximum with no power cap to explain it (a clock
+    lock left behind), is taken again."""
+    if not clocks:
+        return False
+    reasons = set(clocks.get("reasons") or [])
+    if reasons & REJECT_REASONS:
+        return True
+    sm, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    return bool(sm and mx and sm < 0.8 * mx and "sw_power_cap" not in reasons)
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clock and throttle reasons during the timed region.
 
@@ -398,7 +411,7 @@ def run_rbw(args, dist: Dist):
         sampler.start()
         t_local = time_graph(graph, args.steps, sampler=sampler)
         clocks = sampler.stop()
-        if not (clocks and set(clocks["reasons"]) & REJECT_REASONS):
+        if not clocks_rejected(clocks):
             break
         if clocks:
             clocks["retaken"] = True

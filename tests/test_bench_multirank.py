@@ -62,3 +62,40 @@ def test_json_line_carries_the_contract_keys():
         assert k in line
     assert line["scaling"] == "weak" and line["higher_is_better"] is True
     assert line["config"]["workload"] == bench.WORKLOAD
+
+
+def test_clock_rejection_rule():
+    ok = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped = {"sm_mhz": 1300.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    thermal = {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_thermal_slowdown"]}
+    locked = {"sm_mhz": 1100.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert not bench.clocks_rejected(ok) and not bench.clocks_rejected(capped)
+    assert bench.clocks_rejected(thermal) and bench.clocks_rejected(locked)
+    assert not bench.clocks_rejected(None)
+
+
+def test_clock_sampler_keeps_samples_inside_the_timed_region(tmp_path, monkeypatch):
+    """nvidia-smi is replaced by a script: samples before begin() report a
+    thermal slowdown, samples after it a power cap only."""
+    flag = tmp_path / "timed"
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text("#!/bin/sh\nwhile true; do\n"
+                    "  if [ -e %s ]; then echo '1950, 1965, 100, 900.0, 0x0000000000000004';\n"
+                    "  else echo '1200, 1965, 100, 900.0, 0x0000000000000020'; fi\n"
+                    "  sleep 0.02\ndone\n" % flag)
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", str(tmp_path) + os.pathsep + os.environ["PATH"])
+    s = bench.ClockSampler(None, interval_ms=20)
+    s.start()
+    import time
+    time.sleep(0.2)
+    flag.write_text("")
+    time.sleep(0.1)
+    s.begin()
+    time.sleep(0.4)
+    s.end()
+    c = s.stop()
+    assert c["samples_in_timed_region"] >= 5
+    assert c["sm_mhz"] == 1950.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"]
+    assert not bench.clocks_rejected(c)
