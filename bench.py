@@ -240,10 +240,18 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def oracle_sample(seconds_budget=12.0, max_layers=TOKENS * LAYERS):
+def oracle_sample(seconds_budget=12.0, max_layers=TOKENS * LAYERS, threads=None):
     """Time the oracle's float64 apply on the workload layer: applications until
-    about seconds_budget of CPU work has run, at most one step's worth."""
+    about seconds_budget of CPU work has run, at most one step's worth (on
+    `threads` OpenMP threads if given, else all)."""
     import oracle
+    if threads is not None:
+        all_threads = oracle.threads()
+        oracle.set_threads(threads)
+        try:
+            return oracle_sample(seconds_budget, max_layers)
+        finally:
+            oracle.set_threads(all_threads)
     from residual_binarized_weight_b200 import synth
     wl = synth.workload(WORKLOAD)
     W = synth.weights(wl.layers[0])
@@ -448,6 +456,9 @@ def run_rbw(args, dist: Dist):
         cb = None
         if dist.world == 1 and not args.no_cpu_baseline:
             cb, _ = oracle_sample(seconds_budget=args.cpu_seconds)
+            one, _ = oracle_sample(seconds_budget=3.0, threads=1)
+            cb["single_thread"] = {"value": one["value"], "unit": one["unit"], "cores": one["cores"],
+                                   "sample": one["sample"]}
         line = assemble_line(
             value=value, unit="GB/s", n_gpus=dist.world, steps=args.steps, warmup=args.warmup,
             ms_per_step=t_max / args.steps * 1e3,

@@ -51,6 +51,8 @@ def _load():
         lib.oracle_apply.restype = None
         lib.oracle_qat_backward.argtypes = [vp, vp, vp, i64, i64, i32, vp, vp, i64, vp, vp, vp, vp]
         lib.oracle_qat_backward.restype = i32
+        lib.oracle_set_threads.argtypes = [i32]
+        lib.oracle_set_threads.restype = None
         lib.oracle_threads.argtypes = []
         lib.oracle_threads.restype = i32
         lib.oracle_transpose_planes.argtypes = [vp, i64, i64, i32, vp]
@@ -86,6 +88,11 @@ def _c(a, dtype):
 def threads() -> int:
     """OpenMP threads the oracle's parallel loops use."""
     return int(_load().oracle_threads())
+
+
+def set_threads(n: int) -> None:
+    """Thread count of the oracle's later parallel loops (from this thread)."""
+    _load().oracle_set_threads(int(n))
 
 
 def plane_words(N: int, K: int, k: int) -> int:

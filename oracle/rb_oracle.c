@@ -129,6 +129,9 @@ static double decode_bfloat16(uint16_t b)
 /* OpenMP threads a parallel region of this library runs on (for reporting). */
 int oracle_threads(void) { return omp_get_max_threads(); }
 
+/* Thread count of later parallel regions started from the calling thread. */
+void oracle_set_threads(int n) { if (n > 0) omp_set_num_threads(n); }
+
 uint16_t oracle_f64_to_f16(double v) { return encode_binary16(v); }
 double oracle_f16_to_f64(uint16_t b) { return decode_binary16(b); }
 uint16_t oracle_f64_to_bf16(double v) { return encode_bfloat16(v); }
