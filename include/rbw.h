@@ -69,7 +69,10 @@ typedef enum {
 
 /* Bits OR-ed into *dev_status by the kernels. */
 #define RB_DEV_NONFINITE 0x1  /* W, g or h held a NaN or infinity            */
-#define RB_DEV_RANGE 0x2      /* |g| or |h| rounds to infinity in fp16       */
+#define RB_DEV_RANGE 0x2      /* a value rounds to infinity in fp16: a scale
+                                 g or h (rb_pack), or an activation x on a
+                                 tensor-core path (rb_gemm; rb_gemv and
+                                 rb_gemv_batch for M >= 2 or k > 4)          */
 #define RB_DEV_TIMEOUT 0x4    /* a bounded device-side wait expired          */
 
 typedef enum { RB_F32 = 0, RB_BF16 = 1 } rb_dtype;
@@ -97,6 +100,27 @@ RB_API const char *rb_status_string(int status);
  * (layout above): k * ceil(K/256) * ceil(N/32) * 256.  Returns 0 for invalid
  * sizes. */
 RB_API size_t rb_packed_words(int n_out, int k_in, int k_planes);
+
+/*
+ * Plain row-major packing <-> storage layout.  RaBiT's kernel paragraph
+ * ("Technical novelty": 32 columns packed into one uint32_t) fixes only the
+ * word contents; the plain form of it is words [k][N][K/32]: row r, column c
+ * at bit c % 32 of word c / 32 (LSB first), bit = 1 meaning B = +1 -- e.g.
+ * numpy's packbits(B >= 0, bitorder="little") viewed as little-endian uint32.
+ * These calls permute whole words between that form and the storage layout
+ * above, so planes packed elsewhere can be applied here and planes derived
+ * here can be exported.
+ *   rowmajor   rb_rowmajor_words(N, K, k) = k * N * K/32 uint32 words.
+ *   planes     rb_packed_words(N, K, k) words in the storage layout; from the
+ *              plain form every word is written (padding words zero).
+ * The two buffers must not overlap (RB_ERR_ARG).  Asynchronous on `stream`;
+ * HBM-bound (one read and one write of k N K / 8 bytes).
+ */
+RB_API size_t rb_rowmajor_words(int n_out, int k_in, int k_planes);
+RB_API rb_status rb_planes_from_rowmajor(const uint32_t *rowmajor, int n_out, int k_in, int k_planes,
+                                         uint32_t *planes, cudaStream_t stream);
+RB_API rb_status rb_planes_to_rowmajor(const uint32_t *planes, int n_out, int k_in, int k_planes,
+                                       uint32_t *rowmajor, cudaStream_t stream);
 
 /*
  * rb_pack -- derive and bit-pack the residual sign planes (RaBiT, Algorithm 2
@@ -132,9 +156,10 @@ RB_API rb_status rb_pack(const float *W, const float *g, const float *h,
  * Otherwise (no workspace, or k > 4): mma.sync kernel.  Both tensor-core paths
  * use fp16 operands with fp32 accumulation: the +-h_i operands are exact in
  * fp16 and X is converted to fp16 (exact for bf16 values of magnitude
- * 2^-14 .. 65504; smaller ones lose low bits, larger ones overflow; the
- * tcgen05 path flags |x| >= 65520 with RB_DEV_RANGE), so every product is
- * exact and only the accumulation rounds.
+ * 2^-14 .. 65504; smaller ones lose low bits; |x| >= 65520 overflows and
+ * both paths raise RB_DEV_RANGE in *dev_status), so every product is exact
+ * and only the accumulation rounds.  The byte-table path forms h*x in fp32
+ * and raises nothing.
  */
 RB_API size_t rb_gemv_workspace_bytes(int n_out, int k_in, int k_planes, int M);
 RB_API rb_status rb_gemv(const rb_layer_t *layer, const uint16_t *X, int M,
@@ -152,7 +177,8 @@ RB_API rb_status rb_gemv(const rb_layer_t *layer, const uint16_t *X, int M,
  * busy and each CTA's table builds are spread over many rows.  The per-slice
  * sums are therefore associated differently than in rb_gemv for the same layer,
  * so results may differ from rb_gemv's in the last bits; both are
- * deterministic for a given count.  Needs no workspace.
+ * deterministic for a given count.  Needs no workspace.  dev_status
+ * (nullable, 16-byte aligned) gets RB_DEV_RANGE as for rb_gemv.
  */
 RB_API rb_status rb_gemv_batch(const rb_layer_t *const *layers, const uint16_t *const *X, void *const *Y,
                                int count, int M, rb_dtype y_dtype, int32_t *dev_status, unsigned flags,
@@ -160,7 +186,11 @@ RB_API rb_status rb_gemv_batch(const rb_layer_t *const *layers, const uint16_t *
 
 /*
  * rb_gemm -- batched (prefill) Y = X . What^T for any M >= 1 (tuned for
- * M >= 64) on the tcgen05 tensor cores: sign tiles are expanded to +-h_i
+ * M >= 64) on the tcgen05 tensor cores.  It computes the same product as
+ * rb_gemv (RaBiT, "Residual binarization": Y = sum_i g_i .* (B_i (h_i .* X)),
+ * the k paths side by side) from the bit-packed planes of RaBiT's kernel
+ * paragraph ("Technical novelty": 32 columns per uint32_t), organised as a
+ * dense contraction: sign tiles are expanded to +-h_i
  * (fp16, exact) and multiplied with X converted to fp16 (exact in the normal
  * range), fp32 accumulation in tensor memory, one accumulator per plane,
  * epilogue Y = sum_i g_i . acc_i.
@@ -170,6 +200,26 @@ RB_API size_t rb_gemm_workspace_bytes(int n_out, int k_in, int k_planes, int M);
 RB_API rb_status rb_gemm(const rb_layer_t *layer, const uint16_t *X, int M,
                   void *Y, rb_dtype y_dtype, void *workspace, size_t workspace_bytes,
                   int32_t *dev_status, unsigned flags, cudaStream_t stream);
+
+/*
+ * rb_gemm_wait_limit -- rb_gemm with a caller-chosen bound on every
+ * device-side pipeline wait (rb_gemm uses 1 s), for callers that run their
+ * own watchdog and want the kernel to give up sooner, and for tests of the
+ * error path.  The pages have no counterpart.  When a wait expires the
+ * kernel stops issuing work, lets the copies
+ * and MMAs it already issued finish, frees its tensor memory, raises
+ * RB_DEV_TIMEOUT in *dev_status and returns; Y is then undefined, and the
+ * stream and context stay usable.
+ *   wait_limit_ns  0 .. 1e9.  0 waits not at all: any pipeline stage that is
+ *                  not ready at its first probe ends the call with
+ *                  RB_DEV_TIMEOUT (useful only to exercise the error path).
+ *                  Larger values return RB_ERR_ARG.
+ * Other arguments as rb_gemm.
+ */
+RB_API rb_status rb_gemm_wait_limit(const rb_layer_t *layer, const uint16_t *X, int M,
+                                    void *Y, rb_dtype y_dtype, void *workspace, size_t workspace_bytes,
+                                    int32_t *dev_status, unsigned flags, uint64_t wait_limit_ns,
+                                    cudaStream_t stream);
 
 /*
  * rb_gemm_noalloc -- rb_gemm for callers that must not allocate device memory.

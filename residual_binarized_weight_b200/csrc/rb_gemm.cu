@@ -37,6 +37,11 @@ constexpr int kBK = 64;           // K per pipeline stage (one 128-byte swizzle 
 constexpr int kSX = 8;            // X stages (at most; fewer when h pairs of a long K need the room)
 constexpr int kThreads = 192;
 constexpr uint64_t kTimeoutNs = 1000000000ull;   // 1 s per wait
+// Cap on the waits that only drain work already issued (TMA loads, MMAs): such
+// work always completes, so these waits end long before the cap; it only keeps
+// a broken device from holding the thread for ever.  Independent of the
+// caller's limit, which may be tiny.
+constexpr uint64_t kDrainCapNs = 2000000000ull;  // 2 s
 
 // ---------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -47,6 +52,14 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.b32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
@@ -63,9 +76,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 // Bounded wait: gives up after timeout_ns, or as soon as another thread of the
 // CTA (abort_flag) or another CTA (RB_DEV_TIMEOUT in dev_status) has given up.
-// A thread that times out raises both flags.
+// A thread that times out raises both flags.  timeout_ns = 0 waits not at all:
+// a phase that is not complete at the first (non-blocking) probe gives up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           int32_t* dev_status, uint64_t timeout_ns) {
+    if (timeout_ns == 0) {
+        if (mbar_test_wait(bar, parity)) return true;
+        *abort_flag = 1;
+        set_dev_status(dev_status, RB_DEV_TIMEOUT);
+        return false;
+    }
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
@@ -83,6 +103,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             }
         }
     }
+}
+// Wait for a phase that is certain to complete (work this CTA already issued),
+// capped by kDrainCapNs only.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, uint64_t t0) {
+    while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kDrainCapNs) {}
 }
 // Warp-uniform form for code that continues with .sync.aligned instructions.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -306,12 +331,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
                 ++issued;
                 if (++s == nsx) { s = 0; ++j; }
             }
-            if (*abort_flag) {                    // drain the loads this thread issued (bounded)
+            if (*abort_flag) {                    // drain the loads this thread issued: they always land
                 const uint64_t t0 = globaltimer_ns();
                 for (int kb = issued - nsx < 0 ? 0 : issued - nsx; kb < issued; ++kb)
-                    while (!mbar_try_wait(full_x(kb % nsx), (kb / nsx) & 1) && globaltimer_ns() - t0 < timeout_ns) {}
-                if constexpr (gemm_hp_in_smem(KP))
-                    while (!mbar_try_wait(hp_full, 0) && globaltimer_ns() - t0 < timeout_ns) {}
+                    mbar_drain(full_x(kb % nsx), (kb / nsx) & 1, t0);
+                if constexpr (gemm_hp_in_smem(KP)) mbar_drain(hp_full, 0, t0);
             }
         }
     } else if (warp == 1) {
@@ -523,10 +547,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
     }
 
     // ---- teardown: every MMA has completed (acc_full) or the CTA gave up
-    if (warp == 1 && lane == 0 && *abort_flag) {    // no MMA may still run when TMEM is freed
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(acc_full, 0) && globaltimer_ns() - t0 < timeout_ns) {}
-    }
+    if (warp == 1 && lane == 0 && *abort_flag)      // no MMA may still run when TMEM is freed:
+        mbar_drain(acc_full, 0, globaltimer_ns());  // acc_full is committed after the last MMA, always
     tc_fence_before();
     __syncthreads();
     if (*abort_flag && threadIdx.x == 0) set_dev_status(dev_status, RB_DEV_TIMEOUT);
@@ -540,13 +562,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
 {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    // Looked up once per process; host threads may race here, and every racer
+    // stores the same driver address.
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> cache{nullptr};
+    PFN_cuTensorMapEncodeTiled_v12000 fn = cache.load(std::memory_order_acquire);
     if (!fn) {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
+            q == cudaDriverEntryPointSuccess) {
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+            cache.store(fn, std::memory_order_release);
+        }
     }
     return fn;
 }
@@ -719,6 +746,16 @@ extern "C" rb_status rb_gemm(const rb_layer_t* layer, const uint16_t* X, int M, 
 {
     return gemm_with_timeout(layer, X, M, Y, y_dtype, workspace, workspace_bytes, dev_status, flags,
                              stream, kTimeoutNs, false);
+}
+
+extern "C" rb_status rb_gemm_wait_limit(const rb_layer_t* layer, const uint16_t* X, int M, void* Y,
+                                        rb_dtype y_dtype, void* workspace, size_t workspace_bytes,
+                                        int32_t* dev_status, unsigned flags, uint64_t wait_limit_ns,
+                                        cudaStream_t stream)
+{
+    if (wait_limit_ns > kTimeoutNs) return RB_ERR_ARG;
+    return gemm_with_timeout(layer, X, M, Y, y_dtype, workspace, workspace_bytes, dev_status, flags,
+                             stream, wait_limit_ns, false);
 }
 
 // ---------------------------------------------------------------------------

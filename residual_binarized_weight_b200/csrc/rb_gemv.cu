@@ -481,7 +481,8 @@ __device__ __forceinline__ void mma_load_words(uint32_t (&w)[KP][8], const uint3
 // shift -> LOP3 -> HMMA latency chain.
 template <int KP, int NT>
 __global__ void __launch_bounds__(kMmaThreads, (KP * NT <= 4) ? 2 : 1)
-gemv_mma_kernel(const __grid_constant__ LutBatch batch, int N, int K, int M, int CS, int groups, int ydt)
+gemv_mma_kernel(const __grid_constant__ LutBatch batch, int N, int K, int M, int CS, int groups, int ydt,
+                int32_t* dev_status)
 {
     constexpr int TG = 8 * NT;
     extern __shared__ __align__(16) uint8_t msm[];
@@ -540,7 +541,9 @@ gemv_mma_kernel(const __grid_constant__ LutBatch batch, int N, int K, int M, int
     pdl_launch_dependents();
     pdl_wait();
     // ---- activations of the CTA's columns, fp16, pair order (j, j+16) per word;
-    // one item = token m, word wl, half q: pairs j = 8q .. 8q+7 from two 16 B loads
+    // one item = token m, word wl, half q: pairs j = 8q .. 8q+7 from two 16 B loads.
+    // A value that is infinite in fp16 (|x| >= 65520, or x infinite) raises RB_DEV_RANGE.
+    int x_range = 0;
     for (int idx = threadIdx.x; idx < TG * nsl * 16; idx += kMmaThreads) {
         const int m = idx / (nsl * 16), rem = idx % (nsl * 16), wl = rem >> 1, q = rem & 1;
         const int64_t c0 = s0 * 256 + 32 * wl + 8 * q;
@@ -557,13 +560,14 @@ gemv_mma_kernel(const __grid_constant__ LutBatch batch, int N, int K, int M, int
             const uint32_t a = (e & 1) ? (lw[e >> 1] & 0xffff0000u) : (lw[e >> 1] << 16);
             const uint32_t b = (e & 1) ? (hw[e >> 1] & 0xffff0000u) : (hw[e >> 1] << 16);
             const __half2 h2 = __floats2half2_rn(__uint_as_float(a), __uint_as_float(b));
+            x_range |= __hisinf(__low2half(h2)) | __hisinf(__high2half(h2));
             pr[e] = *reinterpret_cast<const uint32_t*>(&h2);
         }
         uint4* dst = reinterpret_cast<uint4*>(xs + m * XS + 32 * wl + 16 * q);
         dst[0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
         dst[1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
     }
-    __syncthreads();
+    if (__syncthreads_or(x_range) && threadIdx.x == 0) set_dev_status(dev_status, RB_DEV_RANGE);
 
     float acc[KP][2][NT][4];
 #pragma unroll
@@ -894,7 +898,8 @@ rb_status launch_lut(const rb_layer_t* const* layers, const uint16_t* const* X, 
 // registers); CS = the smallest power of two that fits the staged activations
 // (at most 96 KB) and gives about two CTAs per SM, at most min(16, S).
 template <int KP, int NT>
-rb_status launch_mma_nt(const LutBatch& b, int n, int N, int K, int M, int ydt, bool pdl, cudaStream_t stream)
+rb_status launch_mma_nt(const LutBatch& b, int n, int N, int K, int M, int ydt, int32_t* dev_status, bool pdl,
+                        cudaStream_t stream)
 {
     static std::atomic<bool> attr_set[64];       // per device; setting the attributes twice is harmless
     int dev = 0;
@@ -939,14 +944,14 @@ rb_status launch_mma_nt(const LutBatch& b, int n, int N, int K, int M, int ydt, 
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    if (cudaLaunchKernelEx(&cfg, gemv_mma_kernel<KP, NT>, b, N, K, M, CS, groups, ydt) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, gemv_mma_kernel<KP, NT>, b, N, K, M, CS, groups, ydt, dev_status) != cudaSuccess)
         return RB_ERR_CUDA;
     return RB_OK;
 }
 
 template <int KP>
 rb_status launch_mma(const rb_layer_t* const* layers, const uint16_t* const* X, void* const* Y, int count, int M,
-                     int ydt, bool pdl, cudaStream_t stream)
+                     int ydt, int32_t* dev_status, bool pdl, cudaStream_t stream)
 {
     // 16 tokens per CTA at most: at k <= 2 two such CTAs share an SM, which beats one
     // 32-token CTA per SM (4096 x 4096, k = 2, 96 layers at M = 64: 17.1 vs 24.8 us)
@@ -965,9 +970,9 @@ rb_status launch_mma(const rb_layer_t* const* layers, const uint16_t* const* X, 
         const int need = (M + 7) / 8;                 // n-tiles for all tokens in one group
         rb_status st;
         if (need >= 2 && NTMAX >= 2)
-            st = launch_mma_nt<KP, (NTMAX >= 2 ? 2 : 1)>(b, n, L0->n_out, L0->k_in, M, ydt, pdl, stream);
+            st = launch_mma_nt<KP, (NTMAX >= 2 ? 2 : 1)>(b, n, L0->n_out, L0->k_in, M, ydt, dev_status, pdl, stream);
         else
-            st = launch_mma_nt<KP, 1>(b, n, L0->n_out, L0->k_in, M, ydt, pdl, stream);
+            st = launch_mma_nt<KP, 1>(b, n, L0->n_out, L0->k_in, M, ydt, dev_status, pdl, stream);
         if (st != RB_OK) return st;
     }
     return RB_OK;
@@ -991,7 +996,8 @@ extern "C" size_t rb_gemv_workspace_bytes(int n_out, int k_in, int k_planes, int
 }
 
 static rb_status gemv_dispatch(const rb_layer_t* const* layers, const uint16_t* const* X, void* const* Y,
-                               int count, int M, rb_dtype y_dtype, unsigned flags, cudaStream_t stream)
+                               int count, int M, rb_dtype y_dtype, int32_t* dev_status, unsigned flags,
+                               cudaStream_t stream)
 {
     const rb_layer_t* L0 = layers[0];
     for (int j = 0; j < count; ++j) {
@@ -1001,6 +1007,7 @@ static rb_status gemv_dispatch(const rb_layer_t* const* layers, const uint16_t* 
             return RB_ERR_SHAPE;
     }
     if (M > 64) return RB_ERR_SHAPE;
+    if (dev_status && !aligned16(dev_status)) return RB_ERR_ALIGN;
     if (!device_is_sm100()) return RB_ERR_UNSUPPORTED;
     const bool pdl = (flags & RB_LAUNCH_PDL) != 0;
     const int ydt = (int)y_dtype;
@@ -1013,14 +1020,14 @@ static rb_status gemv_dispatch(const rb_layer_t* const* layers, const uint16_t* 
         }
     }
     switch (L0->k_planes) {
-        case 1: return launch_mma<1>(layers, X, Y, count, M, ydt, pdl, stream);
-        case 2: return launch_mma<2>(layers, X, Y, count, M, ydt, pdl, stream);
-        case 3: return launch_mma<3>(layers, X, Y, count, M, ydt, pdl, stream);
-        case 4: return launch_mma<4>(layers, X, Y, count, M, ydt, pdl, stream);
-        case 5: return launch_mma<5>(layers, X, Y, count, M, ydt, pdl, stream);
-        case 6: return launch_mma<6>(layers, X, Y, count, M, ydt, pdl, stream);
-        case 7: return launch_mma<7>(layers, X, Y, count, M, ydt, pdl, stream);
-        default: return launch_mma<8>(layers, X, Y, count, M, ydt, pdl, stream);
+        case 1: return launch_mma<1>(layers, X, Y, count, M, ydt, dev_status, pdl, stream);
+        case 2: return launch_mma<2>(layers, X, Y, count, M, ydt, dev_status, pdl, stream);
+        case 3: return launch_mma<3>(layers, X, Y, count, M, ydt, dev_status, pdl, stream);
+        case 4: return launch_mma<4>(layers, X, Y, count, M, ydt, dev_status, pdl, stream);
+        case 5: return launch_mma<5>(layers, X, Y, count, M, ydt, dev_status, pdl, stream);
+        case 6: return launch_mma<6>(layers, X, Y, count, M, ydt, dev_status, pdl, stream);
+        case 7: return launch_mma<7>(layers, X, Y, count, M, ydt, dev_status, pdl, stream);
+        default: return launch_mma<8>(layers, X, Y, count, M, ydt, dev_status, pdl, stream);
     }
 }
 
@@ -1033,16 +1040,15 @@ extern "C" rb_status rb_gemv(const rb_layer_t* layer, const uint16_t* X, int M, 
         workspace_bytes >= rb_gemv_workspace_bytes(layer->n_out, layer->k_in, layer->k_planes, M))
         return gemm_with_timeout(layer, X, M, Y, y_dtype, workspace, workspace_bytes, dev_status, flags, stream,
                                  kWaitTimeoutNs, true);
-    return gemv_dispatch(&layer, &X, &Y, 1, M, y_dtype, flags, stream);
+    return gemv_dispatch(&layer, &X, &Y, 1, M, y_dtype, dev_status, flags, stream);
 }
 
 extern "C" rb_status rb_gemv_batch(const rb_layer_t* const* layers, const uint16_t* const* X, void* const* Y,
                                    int count, int M, rb_dtype y_dtype, int32_t* dev_status, unsigned flags,
                                    cudaStream_t stream)
 {
-    (void)dev_status;
     if (!layers || !X || !Y || count < 1) return RB_ERR_ARG;
     for (int j = 0; j < count; ++j)
         if (!layers[j]) return RB_ERR_ARG;
-    return gemv_dispatch(layers, X, Y, count, M, y_dtype, flags, stream);
+    return gemv_dispatch(layers, X, Y, count, M, y_dtype, dev_status, flags, stream);
 }

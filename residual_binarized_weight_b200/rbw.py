@@ -32,8 +32,12 @@ SIGNATURES = {
     "rb_gemv_batch": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _u32, _vp]),
     "rb_gemm_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
     "rb_gemm": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _u32, _vp]),
+    "rb_gemm_wait_limit": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _u32, ctypes.c_uint64, _vp]),
     "rb_gemm_noalloc": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _u32, _vp]),
     "rb_transpose_planes": (_i32, [_vp, _vp, _vp]),
+    "rb_rowmajor_words": (_sz, [_i32, _i32, _i32]),
+    "rb_planes_from_rowmajor": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
+    "rb_planes_to_rowmajor": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "rb_svid_workspace_bytes": (_sz, [_i32, _i32]),
     "rb_svid_greedy": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "rb_svid_iterative_workspace_bytes": (_sz, [_i32, _i32, _i32]),
@@ -178,6 +182,20 @@ def gemm(layer: PackedLayer, X, Y=None, ws=None, flags=0, dev_status=None, strea
     return _apply("rb_gemm", layer, X, Y, ws, flags, dev_status, stream)
 
 
+def gemm_wait_limit(layer: PackedLayer, X, wait_limit_ns, Y=None, ws=None, flags=0, dev_status=None, stream=None,
+                    y_dtype=torch.float32):
+    """rb_gemm_wait_limit: rb_gemm with a caller-chosen bound (ns) on every device-side wait."""
+    if Y is None:
+        Y = torch.empty(X.shape[0], layer.n_out, dtype=y_dtype, device=X.device)
+    L = layer.struct()
+    ydt = RB_BF16 if Y.dtype == torch.bfloat16 else RB_F32
+    wsp, wsb = (None, 0) if ws is None else (_ptr(ws), ws.numel() * ws.element_size())
+    st = lib().rb_gemm_wait_limit(ctypes.byref(L), _ptr(X), X.shape[0], _ptr(Y), ydt, wsp, wsb, _ptr(dev_status),
+                                  flags, int(wait_limit_ns), _stream(stream))
+    _check("rb_gemm_wait_limit", st)
+    return Y
+
+
 def gemm_noalloc(layer: PackedLayer, X, Y=None, flags=0, dev_status=None, stream=None, y_dtype=torch.float32):
     """rb_gemm_noalloc: rb_gemm without a workspace (fixed 32 MiB library scratch; see include/rbw.h)."""
     if Y is None:
@@ -203,6 +221,29 @@ def transpose(layer: PackedLayer, out: PackedLayer | None = None, stream=None):
     L = layer.struct()
     st = lib().rb_transpose_planes(ctypes.byref(L), _ptr(out.planes), _stream(stream))
     _check("rb_transpose_planes", st)
+    return out
+
+
+def rowmajor_words(n_out, k_in, k_planes):
+    return int(lib().rb_rowmajor_words(n_out, k_in, k_planes))
+
+
+def planes_from_rowmajor(rowmajor, n_out, k_in, k_planes, out: PackedLayer | None = None, stream=None):
+    """rb_planes_from_rowmajor: plain [k][N][K/32] LSB-first words (int32 CUDA tensor)
+    -> a PackedLayer whose planes hold them in the storage layout (scales left to the caller)."""
+    out = out or PackedLayer(n_out, k_in, k_planes, rowmajor.device)
+    st = lib().rb_planes_from_rowmajor(_ptr(rowmajor), n_out, k_in, k_planes, _ptr(out.planes), _stream(stream))
+    _check("rb_planes_from_rowmajor", st)
+    return out
+
+
+def planes_to_rowmajor(layer: PackedLayer, out=None, stream=None):
+    """rb_planes_to_rowmajor: the layer's planes as plain [k][N][K/32] LSB-first words (int32)."""
+    n = rowmajor_words(layer.n_out, layer.k_in, layer.k_planes)
+    out = out if out is not None else torch.empty(n, dtype=torch.int32, device=layer.planes.device)
+    st = lib().rb_planes_to_rowmajor(_ptr(layer.planes), layer.n_out, layer.k_in, layer.k_planes, _ptr(out),
+                                     _stream(stream))
+    _check("rb_planes_to_rowmajor", st)
     return out
 
 

@@ -43,6 +43,46 @@ def test_two_gloo_ranks_take_the_max_time(tmp_path):
     assert r["value"] == pytest.approx(1e9 * 2 * 10 / 1.5 / 1e9)
 
 
+def _retake_main(rank, world, port, out_path):
+    """Rank 1's first clock record shows a thermal slowdown, rank 0's is clean:
+    both ranks must take the timed region again, in lock step."""
+    os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    d = bench.Dist()
+    d.init("gloo")
+    calls = []
+
+    def sample_and_time():
+        d.barrier()                               # the real timed region brackets itself with barriers
+        calls.append(len(calls))
+        bad = rank == 1 and len(calls) == 1
+        return 1.0 + len(calls), {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0,
+                                  "reasons": ["sw_thermal_slowdown"] if bad else []}
+    t, clocks = bench.timed_with_retake(d, sample_and_time)
+    t_max = d.max(t)                              # the next collective must pair up across ranks
+    with open(out_path + ".%d" % rank, "w") as f:
+        json.dump({"calls": len(calls), "t": t, "t_max": t_max, "retaken": clocks.get("retaken", False)}, f)
+    d.close()
+
+
+def test_retake_is_collective_when_one_rank_rejects(tmp_path):
+    out = str(tmp_path / "retake")
+    mp.start_processes(_retake_main, args=(2, _free_port(), out), nprocs=2, join=True, start_method="spawn")
+    r = [json.load(open(out + ".%d" % j)) for j in range(2)]
+    for x in r:
+        assert x["calls"] == 2 and x["retaken"] is True
+        assert x["t"] == pytest.approx(3.0) and x["t_max"] == pytest.approx(3.0)
+
+
+def test_no_retake_when_clean():
+    d = _FakeDist(0, 1)
+    d.max = lambda x, device=None: x
+    n = []
+    t, c = bench.timed_with_retake(d, lambda: (n.append(1) or 2.0, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0,
+                                                                   "reasons": []}))
+    assert len(n) == 1 and t == 2.0 and "retaken" not in c
+
+
 class _FakeDist:
     def __init__(self, rank, world):
         self.rank, self.world, self.pg = rank, world, False

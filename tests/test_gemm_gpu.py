@@ -87,3 +87,40 @@ def test_gemm_k_above_4_unsupported():
     with pytest.raises(rbw.RbError) as e:
         rbw.gemm(L, torch.zeros(8, K, dtype=torch.int16, device="cuda"), ws=rbw.workspace(1 << 20))
     assert e.value.status == rbw.RB_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("N,K,k,M", [(512, 1024, 2, 256), (300, 800, 3, 130)])
+def test_gemm_wait_limit_expiry_reports_timeout_and_context_survives(N, K, k, M):
+    """Bounded device waits (failure handling without a GPU fault): with a wait
+    limit of 0 every pipeline stage that is not ready at its first probe ends
+    the call; the kernel drains what it issued, frees its tensor memory and
+    reports RB_DEV_TIMEOUT.  The next calls on the same stream (rb_gemm, and
+    rb_gemm_wait_limit with a generous limit) then match the oracle."""
+    rng = np.random.default_rng(N + K + M)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=6)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    X = synth.activations(M, K, seed=M)
+    Xd = cases.to_dev(X)
+    ws = rbw.workspace(rbw.gemm_workspace_bytes(N, K, k, M))
+    Yr = oracle.apply(planes, g16, h16, N, K, k, X)
+    bound = cases.abs_bound(g16, h16, X)
+    for _ in range(2):
+        st = torch.zeros(4, dtype=torch.int32, device="cuda")
+        rbw.gemm_wait_limit(L, Xd, 0, ws=ws, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st[0].item()) & rbw.RB_DEV_TIMEOUT
+        st = torch.zeros(4, dtype=torch.int32, device="cuda")
+        Y = rbw.gemm(L, Xd, ws=ws, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st[0].item()) == 0
+        cases.check_y(Y.cpu().numpy().astype(np.float64), Yr, bound, bf16=False, per_elem=1e-4)
+    st = torch.zeros(4, dtype=torch.int32, device="cuda")
+    Y = rbw.gemm_wait_limit(L, Xd, 500_000_000, ws=ws, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st[0].item()) == 0
+    cases.check_y(Y.cpu().numpy().astype(np.float64), Yr, bound, bf16=False, per_elem=1e-4)
+    with pytest.raises(rbw.RbError) as e:
+        rbw.gemm_wait_limit(L, Xd, 2_000_000_000, ws=ws)
+    assert e.value.status == rbw.RB_ERR_ARG

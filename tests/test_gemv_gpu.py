@@ -153,6 +153,38 @@ def test_gemv_batch_matches_oracle_and_is_deterministic(N, K, k, count):
             cases.check_y(single.cpu().numpy().astype(np.float64), Yr, bound, bf16=False)
 
 
+def test_gemv_batch_timed_launch_matches_oracle():
+    """The benchmark's timed launch exactly: rb_gemv_batch over 96 distinct
+    buffers of the 4096 x 4096 q_proj workload layer (k = 2, M = 1, fp32 out,
+    programmatic dependent launch), one distinct activation row per
+    application.  The batch plan picks the launch shape from the count, so this
+    is the only way to check the association of per-slice sums that the bench
+    times.  Every application is compared with the float64 oracle."""
+    count, k = 96, 2
+    W, g, h = cases.layer_case(1, 0, k)
+    N, K = W.shape
+    planes, g16, h16 = cases.packed_case(1, 0, k)
+    base = cases.upload_layer(planes, g16, h16, N, K, k)
+    layers = []
+    for _ in range(count):
+        L = rbw.PackedLayer(N, K, k)
+        L.planes.copy_(base.planes)
+        L.g16.copy_(base.g16)
+        L.h16.copy_(base.h16)
+        layers.append(L)
+    X = synth.activations_for(synth.workload(1), count, K)          # one row per application
+    Xd = cases.to_dev(X)
+    Ys = [torch.empty(1, N, dtype=torch.float32, device="cuda") for _ in range(count)]
+    st = torch.zeros(4, dtype=torch.int32, device="cuda")
+    rbw.gemv_batch(layers, [Xd[j:j + 1] for j in range(count)], Ys, flags=rbw.RB_LAUNCH_PDL, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st[0].item()) == 0
+    Yr = oracle.apply(planes, g16, h16, N, K, k, X)
+    bound = cases.abs_bound(g16, h16, X)
+    for j in range(count):
+        cases.check_y(Ys[j].cpu().numpy().astype(np.float64), Yr[j:j + 1], bound[j:j + 1], bf16=False)
+
+
 @pytest.mark.parametrize("N,K,k,M,count", [(4096, 4096, 2, 4, 6), (4096, 4096, 2, 16, 3), (11008, 4096, 2, 8, 2),
                                            (300, 800, 3, 5, 7)])
 def test_gemv_batch_multi_token(N, K, k, M, count):
@@ -213,3 +245,32 @@ def test_gemv_batch_rejects_mixed_shapes():
     with pytest.raises(rbw.RbError) as e:
         rbw.gemv_batch([a, b], X, Y)
     assert e.value.status == rbw.RB_ERR_SHAPE
+
+
+def test_activation_overflow_is_reported_on_tensor_core_paths():
+    """An activation that overflows the fp16 operand (|x| >= 65520) raises
+    RB_DEV_RANGE on the mma.sync path (rb_gemv and rb_gemv_batch at M >= 2) and
+    on the tcgen05 path; the byte-table path (M = 1) forms h*x in fp32 and
+    raises nothing."""
+    N, K, k = 256, 512, 2
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=6)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    big = np.uint16(0x4789)                        # bf16 70144: finite, above fp16's range
+    for M, ws in ((1, None), (4, None), (40, None), (40, "ws")):
+        X = synth.activations(M, K, seed=M)
+        X[M - 1, 100] = big
+        Xd = cases.to_dev(X)
+        st = torch.zeros(4, dtype=torch.int32, device="cuda")
+        w = rbw.workspace(rbw.gemv_workspace_bytes(N, K, k, M)) if ws else None
+        rbw.gemv(L, Xd, ws=w, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st[0].item()) == (0 if M == 1 else rbw.RB_DEV_RANGE), (M, ws)
+        if M > 1:
+            st = torch.zeros(4, dtype=torch.int32, device="cuda")
+            Ys = [torch.empty(M, N, device="cuda") for _ in range(2)]
+            rbw.gemv_batch([L, L], [cases.to_dev(synth.activations(M, K, seed=9)), Xd], Ys, dev_status=st)
+            torch.cuda.synchronize()
+            assert int(st[0].item()) == rbw.RB_DEV_RANGE

@@ -202,6 +202,27 @@ def test_svid_plane1_is_top_singular_pair_of_abs_w():
     assert np.all(g >= 0) and np.all(h >= 0)
 
 
+@pytest.mark.parametrize("wl_index,shape", [(0, None), (1, (512, 1024))])
+def test_svid_later_planes_are_top_singular_pair_of_abs_residual(wl_index, shape):
+    """Greedy SVID (RaBiT, Technical novelty: the traditional greedy initialiser):
+    plane i's scales reproduce the top singular triple of |R_{i-1}| (numpy SVD),
+    with R_{i-1} the fp32 residual of the recurrence after the first i-1 planes
+    (RaBiT Algorithm 2 forward).  Pins planes 2..4 directly: feeding plane i
+    the wrong residual, or W itself, moves g_i h_i^T far from this triple."""
+    W = synth.weights(synth.workload(wl_index).layers[0], *(shape or (None, None)))
+    k = 4
+    g, h = oracle.svid_greedy(W, k, iters=20)
+    for i in range(2, k + 1):
+        _, _, _, st, R = oracle.pack(W, g[:i - 1], h[:i - 1], i - 1, want_residual=True)
+        assert st == 0
+        U, s, Vt = np.linalg.svd(np.abs(R.astype(np.float64)), full_matrices=False)
+        ref = s[0] * np.outer(U[:, 0], Vt[0])
+        ref *= np.sign(ref.sum())
+        got = np.outer(g[i - 1], h[i - 1]).astype(np.float64)
+        assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 1e-4, "plane %d" % i
+        assert np.all(g[i - 1] >= 0) and np.all(h[i - 1] >= 0)
+
+
 def test_zero_weight_degenerate():
     """W = 0: every plane is all +1 (sign(0) = +1), greedy scales are 0, R stays 0."""
     N, K = 8, 64
