@@ -193,7 +193,12 @@ RB_API rb_status rb_gemv_batch(const rb_layer_t *const *layers, const uint16_t *
  * dense contraction: sign tiles are expanded to +-h_i
  * (fp16, exact) and multiplied with X converted to fp16 (exact in the normal
  * range), fp32 accumulation in tensor memory, one accumulator per plane,
- * epilogue Y = sum_i g_i . acc_i.
+ * epilogue Y = sum_i g_i . acc_i.  Every k = 1..8 is served: the k
+ * accumulators and the sign-expansion stages share the 512 tensor-memory
+ * columns, so the token tile narrows from 192-256 (k <= 2) to 16-32 (k >= 5).
+ * For k >= 3 the h pairs of the whole layer sit in shared memory, which
+ * bounds k * K (k = 4: K <= 26848; k = 8: K <= 13920); beyond that
+ * RB_ERR_UNSUPPORTED.
  *   workspace: rb_gemm_workspace_bytes(N, K, k, M) bytes (holds X in fp16).
  */
 RB_API size_t rb_gemm_workspace_bytes(int n_out, int k_in, int k_planes, int M);
@@ -232,8 +237,8 @@ RB_API rb_status rb_gemm_wait_limit(const rb_layer_t *layer, const uint16_t *X, 
  * 32 MiB array compiled into the library instead (every GPU that loads the
  * library holds it until the process exits).  It allocates nothing.
  *   - Sizes whose rb_gemm_workspace_bytes(N, K, k, M) exceeds 32 MiB (about
- *     M*K <= 16.7 million) return RB_ERR_WORKSPACE; k > 4 returns
- *     RB_ERR_UNSUPPORTED, as for rb_gemm.
+ *     M*K <= 16.7 million) return RB_ERR_WORKSPACE; other limits as for
+ *     rb_gemm.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
  *   - All calls share the array.  Each call rewrites what it uses before
@@ -261,6 +266,34 @@ RB_API rb_status rb_gemm_noalloc(const rb_layer_t *layer, const uint16_t *X, int
  * recurrence is element-wise and fl(g h) = fl(h g).
  */
 RB_API rb_status rb_transpose_planes(const rb_layer_t *layer, uint32_t *planes_t, cudaStream_t stream);
+
+/*
+ * rb_qat_backward -- gradients of one coupled-training layer (RaBiT,
+ * Algorithm 2 backward pass: the signs derived on the fly from the latent
+ * weight W are held constant, W takes the gradient of the effective weight,
+ * the scales follow by the chain rule).  With G = dY^T X:
+ *   dW[n][c] = G[n][c]
+ *   dg_i[n]  = sum_c G[n][c] B_i[n][c] h_i[c]
+ *   dh_i[c]  = sum_n G[n][c] g_i[n] B_i[n][c]
+ * (the input gradient dX = dY What comes from rb_transpose_planes + rb_gemm).
+ *   planes   the signs of W: rb_pack(W, g, h) output, storage layout above.
+ *   g, h     [k][N], [k][K] fp32 trainable scales (the same ones rb_pack used).
+ *   X, dY    [M][K], [M][N] bfloat16 bit patterns (layer input, output gradient).
+ *   dW       out, [N][K] fp32: G, on the tcgen05 tensor cores (bf16 products are
+ *            exact, accumulation in fp32 over the M tokens).
+ *   dg, dh   out, [k][N], [k][K] fp32: one pass over G and the planes, partial
+ *            sums added in a fixed order (deterministic).
+ *   workspace  rb_qat_backward_workspace_bytes(N, K, k) bytes (partial sums).
+ * N must be a multiple of 32 (RB_ERR_SHAPE otherwise): dY rows are read by TMA.
+ * dev_status gets RB_DEV_TIMEOUT if a bounded pipeline wait expires.
+ */
+RB_API size_t rb_qat_backward_workspace_bytes(int n_out, int k_in, int k_planes);
+RB_API rb_status rb_qat_backward(const uint32_t *planes, const float *g, const float *h,
+                                 int n_out, int k_in, int k_planes,
+                                 const uint16_t *X, const uint16_t *dY, int M,
+                                 float *dW, float *dg, float *dh,
+                                 void *workspace, size_t workspace_bytes,
+                                 int32_t *dev_status, cudaStream_t stream);
 
 /*
  * rb_svid_greedy -- greedy SVID scales for each plane (RaBiT names Greedy

@@ -28,6 +28,7 @@
 #include <cudaTypedefs.h>
 
 #include "rbw_internal.cuh"
+#include "rb_tcgen05.cuh"
 
 namespace rbw {
 namespace {
@@ -36,147 +37,6 @@ constexpr int kBR = 128;          // output rows per CTA (MMA M, TMEM lanes)
 constexpr int kBK = 64;           // K per pipeline stage (one 128-byte swizzle row of fp16)
 constexpr int kSX = 8;            // X stages (at most; fewer when h pairs of a long K need the room)
 constexpr int kThreads = 192;
-constexpr uint64_t kTimeoutNs = 1000000000ull;   // 1 s per wait
-// Cap on the waits that only drain work already issued (TMA loads, MMAs): such
-// work always completes, so these waits end long before the cap; it only keeps
-// a broken device from holding the thread for ever.  Independent of the
-// caller's limit, which may be tiny.
-constexpr uint64_t kDrainCapNs = 2000000000ull;  // 2 s
-
-// ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.b32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.b32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-// Bounded wait: gives up after timeout_ns, or as soon as another thread of the
-// CTA (abort_flag) or another CTA (RB_DEV_TIMEOUT in dev_status) has given up.
-// A thread that times out raises both flags.  timeout_ns = 0 waits not at all:
-// a phase that is not complete at the first (non-blocking) probe gives up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* dev_status, uint64_t timeout_ns) {
-    if (timeout_ns == 0) {
-        if (mbar_test_wait(bar, parity)) return true;
-        *abort_flag = 1;
-        set_dev_status(dev_status, RB_DEV_TIMEOUT);
-        return false;
-    }
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 1023u) == 0u) {
-            if (*abort_flag) return false;
-            if (dev_status && (*reinterpret_cast<volatile int32_t*>(dev_status) & RB_DEV_TIMEOUT)) {
-                *abort_flag = 1;
-                return false;
-            }
-            if (globaltimer_ns() - t0 > timeout_ns) {
-                *abort_flag = 1;
-                set_dev_status(dev_status, RB_DEV_TIMEOUT);
-                return false;
-            }
-        }
-    }
-}
-// Wait for a phase that is certain to complete (work this CTA already issued),
-// capped by kDrainCapNs only.
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, uint64_t t0) {
-    while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kDrainCapNs) {}
-}
-// Warp-uniform form for code that continues with .sync.aligned instructions.
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                               int32_t* dev_status, uint64_t timeout_ns) {
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, dev_status, timeout_ns) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
-    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-                 :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                              uint32_t accumulate) {
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "setp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-                 :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
-}
-__device__ __forceinline__ void tc_st_32x32b_x32(uint32_t taddr, const uint32_t (&v)[32]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-                 "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-                 "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
-                 :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
-                    "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
-                    "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]),
-                    "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
-                    "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-                 : "memory");
-}
-__device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-                   "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
-                   "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
-                   "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-                 : "r"(taddr) : "memory");
-}
-__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-                   "=r"(v[14]), "=r"(v[15])
-                 : "r"(taddr));
-}
-__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ uint32_t lop3_sign(uint32_t shifted, uint32_t hpair) {
-    // (~shifted & 0x80008000) ^ hpair : a clear sign bit flips +h to -h
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xA6;" : "=r"(d) : "r"(shifted), "r"(0x80008000u), "r"(hpair));
-    return d;
-}
-
-// UMMA shared-memory descriptor: K-major operand, 128-byte swizzle, 8-row
-// groups 1024 bytes apart (SBO), sm100 descriptor version 1.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
-           ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
-}
 
 // Instruction descriptor, kind::f16: fp32 D, fp16 A and B, both K-major, N = bt, M = 128.
 __host__ __device__ constexpr uint32_t idesc_f16(int bt) {
@@ -197,10 +57,6 @@ __host__ __device__ inline int gemm_hp_bytes(int kp, int K) {
 // ks > 1 adds the receive area of the cluster reduction (128 rows x bt tokens fp32).
 __host__ __device__ inline int gemm_smem_bytes(int kp, int bt, int K, int nsx, int ks) {
     return nsx * bt * 128 + gemm_hp_bytes(kp, K) + 1024 + 256 + (ks > 1 ? ks * ((kBR + ks - 1) / ks) * bt * 4 : 0);
-}
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
 // ---------------------------------------------------------------- pre-pass
@@ -496,22 +352,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
             for (int i = 0; i < KP; ++i)
                 gi[i] = n < N ? __half2float(__ushort_as_half(g16[(int64_t)i * N + n])) : 0.0f;
             constexpr int CW = BT < 32 ? BT : 32;            // tokens per TMEM load
+            constexpr int PB = KP <= 4 ? KP : 2;             // planes per batch of TMEM loads (registers)
 #pragma unroll 1
             for (int c = 0; c < BT / CW; ++c) {
                 float y[CW];
 #pragma unroll
                 for (int j = 0; j < CW; ++j) y[j] = 0.0f;
-                uint32_t v[KP][CW];
 #pragma unroll
-                for (int i = 0; i < KP; ++i) {
-                    if constexpr (CW == 32) tc_ld_32x32b_x32(tmem + lane_base + (uint32_t)(i * BT + c * CW), v[i]);
-                    else tc_ld_32x32b_x16(tmem + lane_base + (uint32_t)(i * BT + c * CW), v[i]);
+                for (int i0 = 0; i0 < KP; i0 += PB) {
+                    uint32_t v[PB][CW];
+#pragma unroll
+                    for (int ii = 0; ii < PB; ++ii) {
+                        if (i0 + ii >= KP) break;
+                        const uint32_t col = (uint32_t)((i0 + ii) * BT + c * CW);
+                        if constexpr (CW == 32) tc_ld_32x32b_x32(tmem + lane_base + col, v[ii]);
+                        else tc_ld_32x32b_x16(tmem + lane_base + col, v[ii]);
+                    }
+                    tc_wait_ld();
+#pragma unroll
+                    for (int ii = 0; ii < PB; ++ii) {
+                        if (i0 + ii >= KP) break;
+#pragma unroll
+                        for (int j = 0; j < CW; ++j) y[j] = fmaf(gi[i0 + ii], __uint_as_float(v[ii][j]), y[j]);
+                    }
                 }
-                tc_wait_ld();
-#pragma unroll
-                for (int i = 0; i < KP; ++i)
-#pragma unroll
-                    for (int j = 0; j < CW; ++j) y[j] = fmaf(gi[i], __uint_as_float(v[i][j]), y[j]);
                 if (ks == 1) {
                     if (n < N) {
 #pragma unroll
@@ -686,8 +550,7 @@ rb_status gemm_with_timeout(const rb_layer_t* layer, const uint16_t* X, int M, v
 {
     rb_status st = check_apply_args(layer, X, M, Y, y_dtype, flags);
     if (st != RB_OK) return st;
-    if (layer->k_planes > 4) return RB_ERR_UNSUPPORTED;
-    if (decode && M > 64) return RB_ERR_SHAPE;
+    if (decode && (M > 64 || layer->k_planes > 4)) return RB_ERR_UNSUPPORTED;
     if (dev_status && !aligned16(dev_status)) return RB_ERR_ALIGN;
     GemmWs ws = gemm_ws_layout(layer->k_in, layer->k_planes, M, workspace);
     if (!workspace || workspace_bytes < ws.bytes) return RB_ERR_WORKSPACE;
@@ -724,7 +587,14 @@ rb_status gemm_with_timeout(const rb_layer_t* layer, const uint16_t* X, int M, v
         case 3:
             if (M >= 1024) return launch_gemm<3, 96, 2>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
             return launch_gemm<3, gemm_bt(3), gemm_sa(3)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
-        default: return launch_gemm<4, gemm_bt(4), gemm_sa(4)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+        case 4: return launch_gemm<4, gemm_bt(4), gemm_sa(4)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+        // k = 5..8: the accumulators (k x BT columns) and the A stages (SA x k x 32)
+        // share the 512 tensor-memory columns, so the tiles narrow and the
+        // pipeline shortens as k grows.
+        case 5: return launch_gemm<5, 32, 2>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+        case 6: return launch_gemm<6, 16, 2>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+        case 7: return launch_gemm<7, 32, 1>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
+        default: return launch_gemm<8, 32, 1>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1);
     }
 }
 
@@ -736,7 +606,7 @@ using namespace rbw;
 
 extern "C" size_t rb_gemm_workspace_bytes(int n_out, int k_in, int k_planes, int M)
 {
-    if (n_out < 1 || k_in < 32 || k_in % 32 != 0 || k_planes < 1 || k_planes > 4 || M < 1) return 0;
+    if (n_out < 1 || k_in < 32 || k_in % 32 != 0 || k_planes < 1 || k_planes > 8 || M < 1) return 0;
     return gemm_ws_layout(k_in, k_planes, M, nullptr).bytes;
 }
 
@@ -801,7 +671,6 @@ extern "C" rb_status rb_gemm_noalloc(const rb_layer_t* layer, const uint16_t* X,
 {
     rb_status st = rbw::check_apply_args(layer, X, M, Y, y_dtype, flags);
     if (st != RB_OK) return st;
-    if (layer->k_planes > 4) return RB_ERR_UNSUPPORTED;
     if (rb_gemm_workspace_bytes(layer->n_out, layer->k_in, layer->k_planes, M) > kNoAllocScratchBytes)
         return RB_ERR_WORKSPACE;                 // problem larger than the fixed scratch array
     if (!rbw::device_is_sm100()) return RB_ERR_UNSUPPORTED;

@@ -38,6 +38,8 @@ SIGNATURES = {
     "rb_rowmajor_words": (_sz, [_i32, _i32, _i32]),
     "rb_planes_from_rowmajor": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "rb_planes_to_rowmajor": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
+    "rb_qat_backward_workspace_bytes": (_sz, [_i32, _i32, _i32]),
+    "rb_qat_backward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
     "rb_svid_workspace_bytes": (_sz, [_i32, _i32]),
     "rb_svid_greedy": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "rb_svid_iterative_workspace_bytes": (_sz, [_i32, _i32, _i32]),
@@ -245,6 +247,23 @@ def planes_to_rowmajor(layer: PackedLayer, out=None, stream=None):
                                      _stream(stream))
     _check("rb_planes_to_rowmajor", st)
     return out
+
+
+def qat_backward(layer: PackedLayer, g, h, X, dY, dW=None, dg=None, dh=None, ws=None, dev_status=None,
+                 stream=None):
+    """rb_qat_backward: (dW [N][K], dg [k][N], dh [k][K]) fp32 from the layer's planes, fp32 scales
+    g [k][N], h [k][K], X bf16 [M][K] and dY bf16 [M][N] (CUDA tensors)."""
+    N, K, k = layer.n_out, layer.k_in, layer.k_planes
+    dev = layer.planes.device
+    dW = dW if dW is not None else torch.empty(N, K, dtype=torch.float32, device=dev)
+    dg = dg if dg is not None else torch.empty(k, N, dtype=torch.float32, device=dev)
+    dh = dh if dh is not None else torch.empty(k, K, dtype=torch.float32, device=dev)
+    nb = int(lib().rb_qat_backward_workspace_bytes(N, K, k))
+    ws = ws if ws is not None else workspace(nb, dev)
+    st = lib().rb_qat_backward(_ptr(layer.planes), _ptr(g), _ptr(h), N, K, k, _ptr(X), _ptr(dY), X.shape[0],
+                               _ptr(dW), _ptr(dg), _ptr(dh), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream))
+    _check("rb_qat_backward", st)
+    return dW, dg, dh
 
 
 def svid_greedy(W, k_planes, iters=20, ws=None, stream=None):

@@ -59,7 +59,11 @@ def test_size_helpers_reject_bad_shapes(L):
     assert L.rb_packed_words(4, 64, 9) == 0
     assert L.rb_gemv_workspace_bytes(4096, 4096, 2, 1) == 0   # partial sums stay on chip
     assert L.rb_gemm_workspace_bytes(4096, 4096, 2, 64) >= 64 * 4096 * 2
-    assert L.rb_gemm_workspace_bytes(4096, 4096, 5, 64) == 0  # the tensor-core path serves k <= 4
+    assert L.rb_gemm_workspace_bytes(4096, 4096, 8, 64) > 0   # the tensor-core path serves k <= 8
+    assert L.rb_gemm_workspace_bytes(4096, 4096, 9, 64) == 0
+    assert L.rb_qat_backward_workspace_bytes(100, 512, 2) == 0  # N must be a multiple of 32
+    assert L.rb_qat_backward_workspace_bytes(4096, 4096, 2) > 0
+    assert L.rb_rowmajor_words(4096, 4096, 2) == 2 * 4096 * 128
     assert L.rb_svid_workspace_bytes(4096, 4096) > 0
 
 

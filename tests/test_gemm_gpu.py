@@ -81,11 +81,32 @@ def test_gemm_matches_gemv_small_m():
     assert np.linalg.norm(Yg - Yv) / np.linalg.norm(Yv) < 1e-5
 
 
-def test_gemm_k_above_4_unsupported():
-    N, K, k = 64, 256, 5
+@pytest.mark.parametrize("N,K,k,M", [(200, 544, 5, 77), (130, 1056, 6, 300), (64, 4096, 7, 33), (257, 800, 8, 129),
+                                     (128, 13920, 8, 40), (300, 2080, 5, 1)])
+def test_gemm_k5_to_8_matches_oracle(N, K, k, M):
+    """k = 5..8 planes on the tensor cores (narrower token tiles, shorter
+    pipeline; the k accumulators share tensor memory with the expansion
+    stages), including the longest K whose h pairs fit shared memory at k = 8."""
+    rng = np.random.default_rng(N + K + 7 * k + M)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=6)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    X = synth.activations(M, K, seed=N + M + k)
+    Yr = oracle.apply(planes, g16, h16, N, K, k, X)
+    for ydt in (torch.float32, torch.bfloat16):
+        st = torch.zeros(4, dtype=torch.int32, device="cuda")
+        Yg = run_gemm(L, X, ydt, dev_status=st)
+        assert int(st[0].item()) == 0
+        cases.check_y(Yg, Yr, cases.abs_bound(g16, h16, X), bf16=ydt == torch.bfloat16, per_elem=1e-4)
+
+
+def test_gemm_k8_beyond_shared_memory_unsupported():
+    N, K, k = 64, 14080, 8
     L = rbw.PackedLayer(N, K, k)
     with pytest.raises(rbw.RbError) as e:
-        rbw.gemm(L, torch.zeros(8, K, dtype=torch.int16, device="cuda"), ws=rbw.workspace(1 << 20))
+        rbw.gemm(L, torch.zeros(8, K, dtype=torch.int16, device="cuda"),
+                 ws=rbw.workspace(rbw.gemm_workspace_bytes(N, K, k, 8)))
     assert e.value.status == rbw.RB_ERR_UNSUPPORTED
 
 
