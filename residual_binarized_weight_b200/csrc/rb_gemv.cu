@@ -76,26 +76,17 @@ __device__ __forceinline__ void lut_load_g(uint16_t (&gv)[KP], const uint16_t* _
     for (int i = 0; i < KP; ++i) gv[i] = r < N ? g16[(int64_t)i * N + r] : (uint16_t)0;
 }
 
-// Shared-window address of dynamic shared memory in a kernel without static
-// shared memory on sm_100 (the driver reserves the first 1 KB per block).  The
-// byte tables start there, so a lookup is one LDS with the PRMT result as
-// register and the table base folded into the immediate.  The kernels are
-// compiled both ways (FAST: base folded; otherwise a register add per lookup)
-// and the host picks FAST when the device reports exactly 1 KB reserved.
-constexpr uint32_t kDynSmemBase = 1024;
+// The byte tables start at the dynamic shared memory base.  That base is the
+// same for every thread of a CTA, so the compiler keeps it in a uniform
+// register and folds it, with the plane's constant offset, into the LDS
+// address: a lookup stays PRMT + LDS + FADD.  (The base is not a compile-time
+// constant: in a cluster launch the shared window of CTA rank r starts at
+// r << 24.)
 
-template <uint32_t IMM>
-__device__ __forceinline__ float lds_imm(uint32_t off) {
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(off), "n"(IMM));
-    return v;
-}
-
-template <bool FAST, int I>
+template <int I>
 __device__ __forceinline__ float lut_entry(uint32_t tbase, uint32_t off) {
     constexpr uint32_t C = (uint32_t)((I >> 1) * 65536 + (I & 1) * 128);
-    if constexpr (FAST) return lds_imm<kDynSmemBase + C>(off);
-    else return lds_f32(tbase + C + off);
+    return lds_f32(tbase + C + off);
 }
 
 
@@ -176,7 +167,7 @@ __device__ __forceinline__ void lut_build(float* lut, const uint4 (&hrr)[KP], co
 // offsets of 4 bytes x kLutPF tiles x KP planes are formed first, then all the
 // LDS are issued, then the FADDs, so each warp keeps 4*kLutPF*KP independent
 // table reads in flight.
-template <int KP, bool FAST>
+template <int KP>
 __device__ __forceinline__ void lut_lookups(float (&acc)[kLutPF][KP][2], const uint32_t (&wd)[kLutPF][KP][8],
                                             const uint32_t (&G)[8], const uint32_t (&SEL)[4], uint32_t tbase)
 {
@@ -194,10 +185,10 @@ __device__ __forceinline__ void lut_lookups(float (&acc)[kLutPF][KP][2], const u
         for (int b = 0; b < 4; ++b)
 #pragma unroll
             for (int p = 0; p < kLutPF; ++p) {
-                e[b][p][0] = lut_entry<FAST, 0>(tbase, off[b][p][0]);
-                if constexpr (KP > 1) e[b][p][1] = lut_entry<FAST, 1>(tbase, off[b][p][1]);
-                if constexpr (KP > 2) e[b][p][2] = lut_entry<FAST, 2>(tbase, off[b][p][2]);
-                if constexpr (KP > 3) e[b][p][3] = lut_entry<FAST, 3>(tbase, off[b][p][3]);
+                e[b][p][0] = lut_entry<0>(tbase, off[b][p][0]);
+                if constexpr (KP > 1) e[b][p][1] = lut_entry<1>(tbase, off[b][p][1]);
+                if constexpr (KP > 2) e[b][p][2] = lut_entry<2>(tbase, off[b][p][2]);
+                if constexpr (KP > 3) e[b][p][3] = lut_entry<3>(tbase, off[b][p][3]);
             }
 #pragma unroll
         for (int b = 0; b < 4; ++b)
@@ -216,7 +207,7 @@ __device__ __forceinline__ void lut_lookups(float (&acc)[kLutPF][KP][2], const u
 // L2 prefetches run kLutPD tiles ahead in the same sequence, on into the next
 // slice.  Tile validity only gates the red[] update, so no load is guarded by
 // a branch.
-template <int KP, bool FAST>
+template <int KP>
 __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_t (&gv)[kLutPF][KP],
                                           const uint32_t (&G)[8], const uint32_t (&SEL)[4], uint32_t tbase,
                                           float* red, const uint32_t* __restrict__ planes,
@@ -245,7 +236,7 @@ __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_
         for (int p = 0; p < kLutPF; ++p)
 #pragma unroll
             for (int i = 0; i < KP; ++i) acc[p][i][0] = acc[p][i][1] = 0.0f;
-        lut_lookups<KP, FAST>(acc, wd, G, SEL, tbase);
+        lut_lookups<KP>(acc, wd, G, SEL, tbase);
         const bool last = it + 1 == iters;
 #pragma unroll
         for (int p = 0; p < kLutPF; ++p) {
@@ -295,7 +286,7 @@ struct LutBatch {
     void* Y[kMaxBatch];
 };
 
-template <int KP, bool FAST>
+template <int KP>
 __global__ void __launch_bounds__(LutCfg<KP>::threads, LutCfg<KP>::min_blocks)
 gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, int R, int ydt)
 {
@@ -372,7 +363,7 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
         lut_build<KP>(lut, hr, X, s, K);
         __syncthreads();
 
-        lut_tiles<KP, FAST>(wd, gv, G, SEL, tbase, red, planes, g16, s, s + CS, S, Nt, N, (int)t_begin,
+        lut_tiles<KP>(wd, gv, G, SEL, tbase, red, planes, g16, s, s + CS, S, Nt, N, (int)t_begin,
                             (int)t_end, warp, lane);
     }
 
@@ -410,408 +401,6 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
         for (int j = 0; j < CS; ++j) y += recv[j * my_span + xo];
         const int64_t r = t_begin * 32 + x0 + xo;
         if (r < N) store_y(Y, ydt, r, y);
-    }
-}
-
-// ---------------------------------------------------------------- persistent batched byte-table kernel
-// A batch of `count` layers as one stream of count * Nt row tiles (layer-major).
-// The grid is the resident set of clusters (CS CTAs each, one CTA per slice
-// group); cluster c owns the contiguous tiles [U c / C, U (c+1) / C) of the
-// stream, so every cluster gets the same amount of work whatever count is, and
-// its CTAs stay resident for the whole launch (no waves, no per-CTA start-up).
-// The range is cut into segments (at layer boundaries and every `segmax`
-// tiles); a CTA walks its runs, one per (segment, slice), building the tables
-// of the run's (layer, slice) and streaming the run's tiles through them.  At
-// the end of a segment the per-row sums go over DSMEM to the CTA that owns the
-// row and the cluster barrier is only arrived at; its wait, and the owner's
-// rank-order sum and store of Y, come at the end of the next segment, so a
-// slow CTA costs the others nothing until a whole segment later.  The receive
-// areas alternate between two buffers by segment parity.  Order at the end of
-// segment g: wait (barrier phase g; phase 0 is an arrival at start-up),
-// sum segment g-1, push segment g, arrive (phase g+1).  A CTA pushes segment
-// g into a buffer after its wait on phase g, which needs the owner's arrival
-// at phase g, which the owner makes only after summing segment g-2 from that
-// same buffer.
-struct LutRun {
-    int layer;       // layer of the batch
-    int s;           // slice
-    int t0;          // first row tile of the run's segment
-    int ntiles;      // row tiles of the segment
-};
-constexpr int kMaxRuns = 256;
-
-template <int KP>
-__device__ __forceinline__ int lut_run_nw(const LutRun& r, int warp)
-{
-    constexpr int NW = LutCfg<KP>::warps;
-    return r.ntiles > warp ? (r.ntiles - warp + NW - 1) / NW : 0;
-}
-
-// One register slot: the sign words and g values of one row tile of one slice,
-// plus the row's index in the segment's per-row sums (-1: nothing loaded).
-template <int KP> struct LutSlot {
-    uint32_t wd[KP][8];
-    uint32_t gp[(KP + 1) / 2];   // g of the row, fp16 pairs (plane 2q in the low half)
-    int ridx;
-};
-// Register slots per warp: with three, a tile's words are loaded two tiles of
-// lookups before their use; k >= 3 keeps two (registers).
-template <int KP> constexpr int lut_slots() { return KP <= 2 ? 3 : 2; }
-constexpr bool kLutPackedAdd = true;
-
-// Position of a warp in its sequence of (run, tile) elements.
-template <int KP> struct LutCursor {
-    int r, j, nw;
-    const uint32_t* p;     // plane 0 words of the element's tile, this lane's column
-    int64_t row;           // row of this lane
-};
-
-template <int KP>
-__device__ __forceinline__ void lut_cursor_set(LutCursor<KP>& c, const LutRun* runs, int nruns,
-                                               const LutBatch& b, int64_t S, int64_t Nt, int warp, int lane)
-{
-    while (c.r < nruns && (c.nw = lut_run_nw<KP>(runs[c.r], warp)) == 0) ++c.r;
-    c.j = 0;
-    if (c.r < nruns) {
-        const LutRun& R = runs[c.r];
-        const int64_t t = R.t0 + warp;
-        c.p = b.planes[R.layer] + block_index(0, R.s, t, S, Nt) * 256 + lane;
-        c.row = t * 32 + lane;
-    }
-}
-
-template <int KP>
-__device__ __forceinline__ void lut_cursor_next(LutCursor<KP>& c, const LutRun* runs, int nruns,
-                                                const LutBatch& b, int64_t S, int64_t Nt, int warp, int lane)
-{
-    constexpr int NW = LutCfg<KP>::warps;
-    if (++c.j < c.nw) {
-        c.p += NW * 256;
-        c.row += NW * 32;
-    } else {
-        ++c.r;
-        lut_cursor_set<KP>(c, runs, nruns, b, S, Nt, warp, lane);
-    }
-}
-
-template <int KP>
-__device__ __forceinline__ void lut_slot_load(LutSlot<KP>& q, const LutCursor<KP>& c, int nruns, const LutRun* runs,
-                                              const LutBatch& b, int64_t S, int64_t Nt, int N, int warp)
-{
-    constexpr int NW = LutCfg<KP>::warps;
-    if (c.r < nruns) {
-        const int64_t plane_words = S * Nt * 256;
-#pragma unroll
-        for (int i = 0; i < KP; ++i)
-#pragma unroll
-            for (int sl = 0; sl < 8; ++sl) q.wd[i][sl] = __ldcs(c.p + i * plane_words + sl * 32);
-        const uint16_t* g = b.g16[runs[c.r].layer];
-        const int64_t r = c.row < N ? c.row : N - 1;
-#pragma unroll
-        for (int i = 0; i < KP; i += 2) {
-            const uint32_t lo = g[(int64_t)i * N + r];
-            const uint32_t hi = i + 1 < KP ? (uint32_t)g[(int64_t)(i + 1) * N + r] : 0u;
-            q.gp[i / 2] = lo | (hi << 16);
-        }
-        q.ridx = (c.j * NW + warp) * 32 + (int)(c.row & 31);
-    } else {
-#pragma unroll
-        for (int i = 0; i < KP; ++i)
-#pragma unroll
-            for (int sl = 0; sl < 8; ++sl) q.wd[i][sl] = 0u;
-#pragma unroll
-        for (int i = 0; i < (KP + 1) / 2; ++i) q.gp[i] = 0u;
-        q.ridx = -1;
-    }
-}
-
-// Lookups of one tile: per word slot, the PRMT offsets of 4 bytes x KP planes,
-// then the LDS, then packed fp32x2 adds into two partial sums per plane.
-template <int KP, bool FAST>
-__device__ __forceinline__ float lut_tile_sum(const LutSlot<KP>& q, const uint32_t (&G)[8], const uint32_t (&SEL)[4],
-                                              uint32_t tbase)
-{
-    float2 acc[KP];
-#pragma unroll
-    for (int i = 0; i < KP; ++i) acc[i] = make_float2(0.0f, 0.0f);
-#pragma unroll
-    for (int sl = 0; sl < 8; ++sl) {
-        uint32_t off[4][KP];
-        float e[4][KP];
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb)
-#pragma unroll
-            for (int i = 0; i < KP; ++i) off[bb][i] = prmt(q.wd[i][sl], G[sl], SEL[bb]);
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-            e[bb][0] = lut_entry<FAST, 0>(tbase, off[bb][0]);
-            if constexpr (KP > 1) e[bb][1] = lut_entry<FAST, 1>(tbase, off[bb][1]);
-            if constexpr (KP > 2) e[bb][2] = lut_entry<FAST, 2>(tbase, off[bb][2]);
-            if constexpr (KP > 3) e[bb][3] = lut_entry<FAST, 3>(tbase, off[bb][3]);
-        }
-#pragma unroll
-        for (int i = 0; i < KP; ++i) {
-            if constexpr (kLutPackedAdd) {
-                acc[i] = __fadd2_rn(acc[i], make_float2(e[0][i], e[1][i]));
-                acc[i] = __fadd2_rn(acc[i], make_float2(e[2][i], e[3][i]));
-            } else {
-                acc[i].x += e[0][i];
-                acc[i].y += e[1][i];
-                acc[i].x += e[2][i];
-                acc[i].y += e[3][i];
-            }
-        }
-    }
-    float pr = 0.0f;
-#pragma unroll
-    for (int i = 0; i < KP; ++i) {
-        const uint32_t gb = (i & 1) ? (q.gp[i / 2] >> 16) : (q.gp[i / 2] & 0xffffu);
-        pr += __half2float(__ushort_as_half((unsigned short)gb)) * (acc[i].x + acc[i].y);
-    }
-    return pr;
-}
-
-// Table build from the staged h and x of the run (shared memory, see
-// lut_stage_hx); the same tables as lut_build.
-template <int KP>
-__device__ __forceinline__ void lut_build_staged(float* lut, const uint16_t* stage)
-{
-    const int gg = threadIdx.x & 31, part = threadIdx.x >> 5;
-    float xv[8];
-    const uint4 xr = *reinterpret_cast<const uint4*>(stage + KP * 256 + gg * 8);
-    const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        xv[2 * q] = bf16_bits_to_f32(xw[q] & 0xffffu);
-        xv[2 * q + 1] = bf16_bits_to_f32(xw[q] >> 16);
-    }
-#pragma unroll
-    for (int i = 0; i < KP; ++i) {
-        const uint4 hq = *reinterpret_cast<const uint4*>(stage + i * 256 + gg * 8);
-        const uint32_t hw[4] = {hq.x, hq.y, hq.z, hq.w};
-        float v[8];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            v[2 * q] = __half2float(__ushort_as_half((unsigned short)(hw[q] & 0xffffu))) * xv[2 * q];
-            v[2 * q + 1] = __half2float(__ushort_as_half((unsigned short)(hw[q] >> 16))) * xv[2 * q + 1];
-        }
-        float L[16];
-        L[0] = -((v[0] + v[1]) + (v[2] + v[3]));
-#pragma unroll
-        for (int n = 1; n < 16; ++n) {
-            const int low = n & -n;
-            const int q = low == 1 ? 0 : low == 2 ? 1 : low == 4 ? 2 : 3;
-            L[n] = L[n & (n - 1)] + 2.0f * v[q];
-        }
-        constexpr int kBPP = 256 / LutCfg<KP>::warps;
-        constexpr int kHN = kBPP >= 16 ? kBPP / 16 : 1;
-        float Hh[kHN];
-#pragma unroll
-        for (int e = 0; e < kHN; ++e) {
-            const int n = kHN * part + e;
-            float acc = 0.0f;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc += ((n >> q) & 1) ? v[4 + q] : -v[4 + q];
-            Hh[e] = acc;
-        }
-        char* base = reinterpret_cast<char*>(lut) + (i >> 1) * 65536 + (i & 1) * 128 + gg * 4;
-#pragma unroll
-        for (int j = 0; j < kBPP; ++j) {
-            const int bt = kBPP * part + j;
-            *reinterpret_cast<float*>(base + bt * 256) = L[bt & 15] + Hh[(bt >> 4) - kHN * part];
-        }
-    }
-}
-
-// Asynchronous copy (cp.async, 16 B per thread) of the run's h (KP x 256
-// columns) and x (256 columns) into a staging buffer; columns past K read as
-// zeros.  The caller waits (cp.async.wait_all) and synchronises before use.
-template <int KP>
-__device__ __forceinline__ void lut_stage_hx(uint16_t* stage, const LutBatch& b, const LutRun& R, int K)
-{
-    const int t = threadIdx.x;
-    if (t < (KP + 1) * 32) {
-        const int v = t >> 5, gg = t & 31;
-        const int64_t c0 = (int64_t)R.s * 256 + gg * 8;
-        uint16_t* dst = stage + v * 256 + gg * 8;
-        if (c0 < K) {
-            const uint16_t* src = v < KP ? b.h16[R.layer] + (int64_t)v * K + c0 : b.X[R.layer] + c0;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(smem_u32(dst)), "l"(src) : "memory");
-        } else {
-            *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-        }
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-__host__ __device__ inline int lut_persist_recv_floats(int segmax, int CS)
-{
-    return ((segmax * 32 + CS - 1) / CS) * CS;            // CS slots of at most ceil(rows / CS) rows
-}
-__host__ __device__ inline int lut_persist_smem(int kp, int segmax, int CS)
-{
-    return lut_table_bytes(kp) + segmax * 32 * 4 + 2 * lut_persist_recv_floats(segmax, CS) * 4 +
-           kMaxRuns * (int)sizeof(LutRun) + 16 + 2 * (kp + 1) * 512;
-}
-
-// Rank-order sum of a finished segment's rows that this rank owns, store Y.
-__device__ __forceinline__ void lut_persist_finish(const LutRun& P, const float* rv, const LutBatch& batch, int rank,
-                                                   int CS, int N, int ydt)
-{
-    const int prow = P.ntiles * 32;
-    const int x0 = prow * rank / CS, my = prow * (rank + 1) / CS - x0;
-    for (int xo = threadIdx.x; xo < my; xo += blockDim.x) {
-        float y = 0.0f;
-        for (int jj = 0; jj < CS; ++jj) y += rv[jj * my + xo];
-        const int64_t row = (int64_t)P.t0 * 32 + x0 + xo;
-        if (row < N) store_y(batch.Y[P.layer], ydt, row, y);
-    }
-}
-
-template <int KP, bool FAST>
-__global__ void __launch_bounds__(LutCfg<KP>::threads, LutCfg<KP>::min_blocks)
-gemv_lut_persist_kernel(const __grid_constant__ LutBatch batch, int count, int N, int K, int CS, int segmax, int ydt)
-{
-    constexpr int NT = LutCfg<KP>::threads;
-    extern __shared__ __align__(1024) float lut[];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t S = num_slices(K), Nt = num_row_tiles(N);
-    const int rank = CS > 1 ? (int)cluster_rank() : 0;
-    const int C = (int)(gridDim.x / CS), c = (int)(blockIdx.x / CS);
-    const int64_t U = (int64_t)count * Nt;
-    const int64_t u0 = U * c / C, u1 = U * (c + 1) / C;
-    float* red = lut + lut_table_bytes(KP) / 4;                 // [segmax*32] per-row sums of this CTA's slices
-    float* recv = red + segmax * 32;                           // [2][CS slots] received partial sums
-    const int recv_floats = lut_persist_recv_floats(segmax, CS);
-    LutRun* runs = reinterpret_cast<LutRun*>(recv + 2 * recv_floats);
-    int* s_nruns = reinterpret_cast<int*>(runs + kMaxRuns);     // (no static shared memory: see kDynSmemBase)
-    uint16_t* stage = reinterpret_cast<uint16_t*>(s_nruns + 4);  // [2][KP + 1][256] h and x of a run
-
-    // ---- the run list: segments of [u0, u1) in order, this CTA's slices in each
-    if (threadIdx.x == 0) {
-        int n = 0;
-        for (int64_t u = u0; u < u1;) {
-            const int layer = (int)(u / Nt);
-            const int64_t t0 = u - (int64_t)layer * Nt;
-            int64_t nt = Nt - t0;
-            if (nt > segmax) nt = segmax;
-            if (nt > u1 - u) nt = u1 - u;
-            for (int64_t s = rank; s < S && n < kMaxRuns; s += CS) runs[n++] = LutRun{layer, (int)s, (int)t0, (int)nt};
-            u += nt;
-        }
-        *s_nruns = n;
-    }
-    for (int x = threadIdx.x; x < segmax * 32; x += NT) red[x] = 0.0f;
-    __syncthreads();
-    const int nruns = *s_nruns;
-    const int spc = (int)((S - rank + CS - 1) / CS);              // runs per segment (slices of this CTA)
-
-    // ---- before the dependency wait: the first kLutSlots tiles, the L2 prefetch cursor, h of run 0
-    constexpr int kLutSlots = lut_slots<KP>();
-    LutSlot<KP> qs[kLutSlots];
-    LutCursor<KP> ld;
-    ld.r = 0;
-    lut_cursor_set<KP>(ld, runs, nruns, batch, S, Nt, warp, lane);
-#pragma unroll
-    for (int q = 0; q < kLutSlots; ++q) {
-        lut_slot_load<KP>(qs[q], ld, nruns, runs, batch, S, Nt, N, warp);
-        if (ld.r < nruns) lut_cursor_next<KP>(ld, runs, nruns, batch, S, Nt, warp, lane);
-    }
-    // L2 prefetch: kLutPD elements ahead; lane l < 8 KP touches line l % 8 of plane l / 8
-    LutCursor<KP> pf;
-    pf.r = 0;
-    lut_cursor_set<KP>(pf, runs, nruns, batch, S, Nt, warp, lane);
-    const bool pf_lane = lane < 8 * KP;
-    const int64_t pf_off = (int64_t)(lane >> 3) * S * Nt * 256 + (lane & 7) * 32 - lane;
-    for (int e = 0; e < kLutPD && pf.r < nruns; ++e) {
-        if (pf_lane) asm volatile("prefetch.global.L2 [%0];" :: "l"(pf.p + pf_off));
-        lut_cursor_next<KP>(pf, runs, nruns, batch, S, Nt, warp, lane);
-    }
-
-    uint32_t G[8], SEL[4];
-#pragma unroll
-    for (int sl = 0; sl < 8; ++sl) {
-        uint32_t gw = 0;
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) gw |= (uint32_t)((((4 * sl + bb) ^ lane) * 4) & 0xff) << (8 * bb);
-        G[sl] = gw;
-    }
-#pragma unroll
-    for (int bb = 0; bb < 4; ++bb)
-        SEL[bb] = (uint32_t)(4 + bb) | ((uint32_t)(bb ^ (lane & 3)) << 4) | ((uint32_t)(12 + bb) << 8) |
-                  ((uint32_t)(12 + bb) << 12);
-    const uint32_t tbase = smem_u32(lut);
-    pdl_launch_dependents();
-    pdl_wait();
-    if (nruns > 0) lut_stage_hx<KP>(stage, batch, runs[0], K);
-
-    // Phase 0 of the cluster barrier: every CTA of the cluster has started (its
-    // shared memory exists) before anyone pushes into it at the first segment end.
-    if (CS > 1) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-    int par = 0;                    // which slot holds this warp's next element
-    int seg = 0;                    // segment index of the current run
-    for (int r = 0; r < nruns; ++r) {
-        const LutRun R = runs[r];
-        cp_async_wait_all();                                  // this run's h and x have landed
-        __syncthreads();                                      // (for all threads); the previous run is done with the tables
-        lut_build_staged<KP>(lut, stage + (r & 1) * (KP + 1) * 256);
-        if (r + 1 < nruns) lut_stage_hx<KP>(stage + ((r + 1) & 1) * (KP + 1) * 256, batch, runs[r + 1], K);
-        __syncthreads();
-        const int nw = lut_run_nw<KP>(R, warp);
-        for (int j = 0; j < nw; ++j) {
-            // use the slot holding element e, refill it with element e + kLutSlots,
-            // prefetch element e + kLutPD into L2 (slot indices stay compile-time)
-#pragma unroll
-            for (int q = 0; q < kLutSlots; ++q) {
-                if (par == q) {
-                    const float pr = lut_tile_sum<KP, FAST>(qs[q], G, SEL, tbase);
-                    red[qs[q].ridx] += pr;
-                    lut_slot_load<KP>(qs[q], ld, nruns, runs, batch, S, Nt, N, warp);
-                }
-            }
-            par = par + 1 == kLutSlots ? 0 : par + 1;
-            if (ld.r < nruns) lut_cursor_next<KP>(ld, runs, nruns, batch, S, Nt, warp, lane);
-            if (pf.r < nruns) {
-                if (pf_lane) asm volatile("prefetch.global.L2 [%0];" :: "l"(pf.p + pf_off));
-                lut_cursor_next<KP>(pf, runs, nruns, batch, S, Nt, warp, lane);
-            }
-        }
-        const bool seg_end = (r + 1) % spc == 0 || r + 1 == nruns;
-        if (!seg_end) continue;
-
-        // ---- end of segment `seg`: finish the previous segment (wait, rank-order
-        // sum, store Y), push this segment's per-row sums to their owners, arrive.
-        const int rows = R.ntiles * 32;
-        const int p = seg & 1;
-        __syncthreads();                                      // red[] complete
-        if (CS == 1) {
-            for (int x = threadIdx.x; x < rows; x += NT) {
-                const int64_t row = (int64_t)R.t0 * 32 + x;
-                if (row < N) store_y(batch.Y[R.layer], ydt, row, red[x]);
-                red[x] = 0.0f;
-            }
-        } else {
-            asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-            if (seg > 0) lut_persist_finish(runs[r - spc], recv + (p ^ 1) * recv_floats, batch, rank, CS, N, ydt);
-            const int tpo = NT / CS;
-            const int jd = threadIdx.x / tpo;
-            if (jd < CS) {
-                const int jx0 = rows * jd / CS, span = rows * (jd + 1) / CS - jx0;
-                const uint32_t dst = smem_u32(recv + p * recv_floats) + (uint32_t)(rank * span) * 4u;
-                for (int xo = threadIdx.x - jd * tpo; xo < span; xo += tpo) {
-                    st_dsmem_f32(dst + (uint32_t)xo * 4u, (uint32_t)jd, red[jx0 + xo]);
-                    red[jx0 + xo] = 0.0f;
-                }
-            }
-            asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-        }
-        ++seg;
-    }
-    if (CS > 1) {                                             // the last segment
-        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-        if (seg > 0) lut_persist_finish(runs[nruns - 1], recv + ((seg - 1) & 1) * recv_floats, batch, rank, CS, N, ydt);
     }
 }
 
@@ -1120,25 +709,6 @@ cudaLaunchConfig_t lut_config(const LutPlan& p, int count, int threads, cudaLaun
     return cfg;
 }
 
-// Dynamic shared memory of the byte-table kernels (no static shared memory)
-// starts right after the per-block reservation: the FAST kernels fold that
-// address (kDynSmemBase) into their lookups, so they run only where the device
-// reserves exactly that much.
-bool lut_fast_base()
-{
-    static std::atomic<int> cache[64];           // per device: 0 unknown, 1 yes, 2 no
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-    int c = cache[dev].load(std::memory_order_relaxed);
-    if (!c) {
-        int reserved = -1;
-        c = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) == cudaSuccess &&
-                    reserved == (int)kDynSmemBase ? 1 : 2;
-        cache[dev].store(c, std::memory_order_relaxed);
-    }
-    return c == 1;
-}
-
 template <int KP>
 bool lut_set_attributes()
 {
@@ -1147,12 +717,10 @@ bool lut_set_attributes()
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return false;
     if (!attr_set[dev].load(std::memory_order_acquire)) {
-        for (auto kern : {gemv_lut_kernel<KP, true>, gemv_lut_kernel<KP, false>}) {
-            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
-                return false;
-            if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-                return false;
-        }
+        if (cudaFuncSetAttribute(gemv_lut_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+            return false;
+        if (cudaFuncSetAttribute(gemv_lut_kernel<KP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+            return false;
         attr_set[dev].store(true, std::memory_order_release);
     }
     return true;
@@ -1168,9 +736,9 @@ int lut_resident(int CS, int smem)
     cudaLaunchConfig_t cfg = lut_config(p, 1, LutCfg<KP>::threads, attr, false, 0);
     int n = 0;
     if (CS > 1) {
-        if (cudaOccupancyMaxActiveClusters(&n, gemv_lut_kernel<KP, true>, &cfg) != cudaSuccess) n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemv_lut_kernel<KP>, &cfg) != cudaSuccess) n = 0;
     } else {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_lut_kernel<KP, true>, LutCfg<KP>::threads, (size_t)smem) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_lut_kernel<KP>, LutCfg<KP>::threads, (size_t)smem) !=
             cudaSuccess)
             n = 0;
         n *= num_sms();
@@ -1286,154 +854,6 @@ rb_status lut_plan(int N, int K, int count, LutPlan* plan)
     return RB_OK;
 }
 
-// ---- persistent batched kernel: plan and launch
-struct PersistPlan {
-    int CS;          // CTAs per cluster (slice groups)
-    int C;           // resident clusters = grid / CS
-    int segmax;      // row tiles per segment at most
-    int smem;        // dynamic shared memory bytes
-};
-
-template <int KP>
-bool persist_set_attributes()
-{
-    static std::atomic<bool> attr_set[64];       // per device; setting the attributes twice is harmless
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-    if (!attr_set[dev].load(std::memory_order_acquire)) {
-        for (auto kern : {gemv_lut_persist_kernel<KP, true>, gemv_lut_persist_kernel<KP, false>})
-            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
-                cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-                return false;
-        attr_set[dev].store(true, std::memory_order_release);
-    }
-    return true;
-}
-
-cudaLaunchConfig_t persist_config(int CS, int C, int smem, int threads, cudaLaunchAttribute* attr, bool pdl,
-                                  cudaStream_t stream)
-{
-    LutPlan p{CS, C, smem};
-    return lut_config(p, 1, threads, attr, pdl, stream);
-}
-
-template <int KP>
-int persist_resident(int CS, int smem)
-{
-    cudaLaunchAttribute attr[2];
-    cudaLaunchConfig_t cfg = persist_config(CS, 1, smem, LutCfg<KP>::threads, attr, false, 0);
-    int n = 0;
-    if (CS > 1) {
-        if (cudaOccupancyMaxActiveClusters(&n, gemv_lut_persist_kernel<KP, true>, &cfg) != cudaSuccess) n = 0;
-    } else {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_lut_persist_kernel<KP, true>, LutCfg<KP>::threads,
-                                                          (size_t)smem) != cudaSuccess)
-            n = 0;
-        n *= num_sms();
-    }
-    return n;
-}
-
-// Segments of the cluster with the most of them (segments end at layer
-// boundaries and every segmax tiles).
-inline int64_t persist_max_segments(int64_t U, int64_t Nt, int C, int segmax)
-{
-    int64_t best = 0;
-    for (int c = 0; c < C; ++c) {
-        int64_t n = 0;
-        for (int64_t u = U * c / C, u1 = U * (c + 1) / C; u < u1; ++n) {
-            int64_t nt = Nt - u % Nt;
-            if (nt > segmax) nt = segmax;
-            if (nt > u1 - u) nt = u1 - u;
-            u += nt;
-        }
-        if (n > best) best = n;
-    }
-    return best;
-}
-
-// CS (a power of two <= 16, <= S) and segmax: the largest segment that fits
-// two CTAs per SM (one for k >= 3), then the CS whose CTAs carry the least
-// modelled work: ceil(U / C) tiles per slice over ceil(S / CS) slices, plus a
-// table build (kLutBuildTiles tile-units) per run.
-template <int KP>
-rb_status persist_plan_uncached(int N, int K, int count, PersistPlan* plan)
-{
-    const int64_t S = num_slices(K), Nt = num_row_tiles(N), U = (int64_t)count * Nt;
-    const int cap = lut_table_bytes(KP) < 96 * 1024 ? 105 * 1024 : 227 * 1024;
-    PersistPlan best{0, 0, 0, 0};
-    double best_cost = 1e300;
-    for (int CS = 1; CS <= 16 && CS <= S; CS *= 2) {
-        int segmax = 128;
-        while (segmax > 8 && lut_persist_smem(KP, segmax, CS) > cap) segmax -= 8;
-        const int smem = lut_persist_smem(KP, segmax, CS);
-        if (smem > cap) continue;
-        int C = persist_resident<KP>(CS, smem);
-        if (C <= 0) continue;
-        if (C > U) C = (int)U;
-        const int64_t spc = (S + CS - 1) / CS;
-        const int64_t segs = persist_max_segments(U, Nt, C, segmax);
-        if (segs * spc > kMaxRuns) continue;
-        const double cost = (double)((U + C - 1) / C) * (double)spc + (double)(segs * spc * kLutBuildTiles);
-        if (cost < best_cost) {
-            best_cost = cost;
-            best = PersistPlan{CS, C, segmax, smem};
-        }
-    }
-    if (best.CS == 0) return RB_ERR_UNSUPPORTED;
-    *plan = best;
-    return RB_OK;
-}
-
-struct PersistKey {
-    int dev, kp, N, K, count;
-    bool operator==(const PersistKey& o) const {
-        return dev == o.dev && kp == o.kp && N == o.N && K == o.K && count == o.count;
-    }
-};
-std::mutex g_persist_mu;
-PersistKey g_persist_keys[kPlanCache];
-PersistPlan g_persist_vals[kPlanCache];
-int g_persist_n = 0;
-
-template <int KP>
-rb_status persist_plan(int N, int K, int count, PersistPlan* plan)
-{
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return RB_ERR_CUDA;
-    if (!persist_set_attributes<KP>()) return RB_ERR_CUDA;
-    const PersistKey key{dev, KP, N, K, count};
-    {
-        std::lock_guard<std::mutex> lk(g_persist_mu);
-        for (int j = 0; j < g_persist_n; ++j)
-            if (g_persist_keys[j] == key) {
-                *plan = g_persist_vals[j];
-                return RB_OK;
-            }
-    }
-    rb_status st = persist_plan_uncached<KP>(N, K, count, plan);
-    if (st != RB_OK) return st;
-    std::lock_guard<std::mutex> lk(g_persist_mu);
-    const int j = g_persist_n < kPlanCache ? g_persist_n++ : (int)((unsigned)(N ^ K ^ count) % kPlanCache);
-    g_persist_keys[j] = key;
-    g_persist_vals[j] = *plan;
-    return RB_OK;
-}
-
-template <int KP>
-rb_status launch_lut_persist(const LutBatch& b, int n, int N, int K, int ydt, bool pdl, cudaStream_t stream)
-{
-    PersistPlan plan;
-    rb_status st = persist_plan<KP>(N, K, n, &plan);
-    if (st != RB_OK) return st;
-    cudaLaunchAttribute attr[2];
-    cudaLaunchConfig_t cfg = persist_config(plan.CS, plan.C, plan.smem, LutCfg<KP>::threads, attr, pdl, stream);
-    if (cudaLaunchKernelEx(&cfg, lut_fast_base() ? gemv_lut_persist_kernel<KP, true> : gemv_lut_persist_kernel<KP, false>,
-                           b, n, N, K, plan.CS, plan.segmax, ydt) != cudaSuccess)
-        return RB_ERR_CUDA;
-    return RB_OK;
-}
-
 template <int KP>
 rb_status launch_lut(const rb_layer_t* const* layers, const uint16_t* const* X, void* const* Y, int count,
                      int ydt, bool pdl, cudaStream_t stream)
@@ -1449,18 +869,12 @@ rb_status launch_lut(const rb_layer_t* const* layers, const uint16_t* const* X, 
             b.X[j] = X[base + j];
             b.Y[j] = Y[base + j];
         }
-        if (n > 1) {                              // many layers: the persistent kernel
-            rb_status st = launch_lut_persist<KP>(b, n, L0->n_out, L0->k_in, ydt, pdl, stream);
-            if (st != RB_OK) return st;
-            continue;
-        }
         LutPlan plan;
         rb_status st = lut_plan<KP>(L0->n_out, L0->k_in, n, &plan);
         if (st != RB_OK) return st;
         cudaLaunchAttribute attr[2];
         cudaLaunchConfig_t cfg = lut_config(plan, n, LutCfg<KP>::threads, attr, pdl, stream);
-        if (cudaLaunchKernelEx(&cfg, lut_fast_base() ? gemv_lut_kernel<KP, true> : gemv_lut_kernel<KP, false>, b,
-                               (int)L0->n_out, (int)L0->k_in, plan.CS, plan.R, ydt) !=
+        if (cudaLaunchKernelEx(&cfg, gemv_lut_kernel<KP>, b, (int)L0->n_out, (int)L0->k_in, plan.CS, plan.R, ydt) !=
             cudaSuccess)
             return RB_ERR_CUDA;
     }
