@@ -330,6 +330,24 @@ RB_API rb_status rb_svid_iterative(const float *W, int n_out, int k_in, int k_pl
                                    float *g, float *h, void *workspace, size_t workspace_bytes,
                                    cudaStream_t stream);
 
+/*
+ * rb_svid_pack -- the deployment path of a trained latent weight in one call,
+ * on the device with no host round trip: scales by iterative residual SVID
+ * (RaBiT, Algorithm 1 without the I/O preprocessing; `sweeps` = 0 gives the
+ * greedy SVID), then the residual sign planes and fp16 scales by rb_pack
+ * (Algorithm 2 forward; deployment freezes the planes).  The result equals
+ * rb_svid_iterative followed by rb_pack on the same stream.
+ *   g, h                out, [k][N], [k][K] fp32 scales (also returned).
+ *   planes, g16, h16    out, as rb_pack.
+ *   workspace           rb_svid_pack_workspace_bytes(N, K, k) bytes.
+ * dev_status gets rb_pack's RB_DEV_* bits.
+ */
+RB_API size_t rb_svid_pack_workspace_bytes(int n_out, int k_in, int k_planes);
+RB_API rb_status rb_svid_pack(const float *W, int n_out, int k_in, int k_planes, int sweeps, int iters,
+                              float *g, float *h, uint32_t *planes, uint16_t *g16, uint16_t *h16,
+                              void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                              cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -10,7 +10,12 @@
 // R_{i-1} from W and the scales of the earlier planes with the fp32
 // recurrence of rb_pack (t = fl(g*h); R = fl(R -/+ t)).  Power iteration runs
 // in float64 with fixed summation orders (warp tree per row, row chunks in
-// order per column), so the result is deterministic.
+// order per column), so the result is deterministic.  One iteration is three
+// launches (A v, A^T u in row chunks, the chunk sum).  The vectors stay
+// unnormalised: the kernel that produces one also produces 1 / its norm --
+// every CTA writes the sum of squares of its part, the last CTA to finish
+// (a counter, no waiting) adds the parts in index order -- and the consumer
+// scales on the fly, so no single-CTA normalisation pass sits between them.
 #include <math.h>
 
 #include "rbw_internal.cuh"
@@ -25,9 +30,12 @@ struct SvidWs {
     double* v;        // [K]
     double* av;       // [N]
     double* vpart;    // [kRowChunks][K]
-    double* scal;     // [8]
+    double* scal;     // [8]: 1/|u|, 1/|v|
+    double* part;     // per-CTA sums of squares of the vector being produced
+    unsigned* cnt;    // finished-CTA counters (zeroed by svid_init_kernel, reset by their last CTA)
     size_t bytes;
 };
+constexpr int kAvRows = 8;           // rows per CTA of svid_av_kernel (one warp each)
 
 SvidWs svid_ws_layout(int N, int K, void* base)
 {
@@ -40,6 +48,10 @@ SvidWs svid_ws_layout(int N, int K, void* base)
     w.av = reinterpret_cast<double*>(p + off);    off += up((size_t)N * 8);
     w.vpart = reinterpret_cast<double*>(p + off); off += up((size_t)kRowChunks * K * 8);
     w.scal = reinterpret_cast<double*>(p + off);  off += 256;
+    const size_t nparts = (size_t)((N + kAvRows - 1) / kAvRows) > (size_t)((K + 255) / 256)
+                        ? (size_t)((N + kAvRows - 1) / kAvRows) : (size_t)((K + 255) / 256);
+    w.part = reinterpret_cast<double*>(p + off);  off += up(nparts * 8);
+    w.cnt = reinterpret_cast<unsigned*>(p + off); off += 256;
     w.bytes = off;
     return w;
 }
@@ -86,44 +98,93 @@ __device__ __forceinline__ double abs_target(const float* W, const float* g, con
     else return abs_residual(W, g, h, N, K, plane, r, c);
 }
 
-// out[r] = sum_c A[r][c] * x[c]   (one warp per row)
-template <bool ITER>
-__global__ void svid_av_kernel(const float* __restrict__ W, const float* __restrict__ g,
-                               const float* __restrict__ h, const uint32_t* __restrict__ S, int N, int K, int k,
-                               int plane, const double* __restrict__ x, double* __restrict__ out)
+// Called by every thread of every CTA after the CTA's sum of squares `mine`
+// (valid in thread 0) is final: stores it as part[blockIdx.x]; the last CTA
+// to arrive adds all parts in index order and writes 1 / sqrt(sum) (0 for a
+// zero vector) to *inv, then re-arms the counter.
+__device__ void finish_norm(double mine, double* part, unsigned* cnt, double* inv)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (r >= N) return;
-    double acc = 0.0;
-    for (int64_t c = lane; c < K; c += 32) acc += abs_target<ITER>(W, g, h, S, N, K, k, plane, r, c) * x[c];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) out[r] = acc;
+    __shared__ bool last;
+    if (threadIdx.x == 0) {
+        part[blockIdx.x] = mine;
+        __threadfence();
+        last = atomicAdd(cnt, 1u) == gridDim.x * gridDim.y - 1;
+    }
+    __syncthreads();
+    if (last && threadIdx.x == 0) {
+        __threadfence();
+        double sum = 0.0;
+        for (unsigned b = 0; b < gridDim.x * gridDim.y; ++b) sum += reinterpret_cast<volatile double*>(part)[b];
+        *inv = sum > 0.0 ? 1.0 / sqrt(sum) : 0.0;
+        *cnt = 0u;
+    }
 }
 
-// vpart[chunk][c] = sum_{r in chunk} A[r][c] * u[r]   (rows in order)
+// out[r] = sum_c A[r][c] * (x[c] * sx)   (one warp per row; sx = 1/|x|, x unnormalised);
+// with inv_out, also 1 / |out|.
+template <bool ITER>
+__global__ void __launch_bounds__(kAvRows * 32)
+svid_av_kernel(const float* __restrict__ W, const float* __restrict__ g,
+               const float* __restrict__ h, const uint32_t* __restrict__ S, int N, int K, int k,
+               int plane, const double* __restrict__ x, const double* __restrict__ sxp, double* __restrict__ out,
+               double* part, unsigned* cnt, double* inv_out)
+{
+    __shared__ double sq[kAvRows];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const double sx = *sxp;
+    const int64_t r = (int64_t)blockIdx.x * kAvRows + warp;
+    double acc = 0.0;
+    if (r < N) {
+        for (int64_t c = lane; c < K; c += 32) acc += abs_target<ITER>(W, g, h, S, N, K, k, plane, r, c) * (x[c] * sx);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) out[r] = acc;
+    }
+    if (!inv_out) return;
+    if (lane == 0) sq[warp] = acc * acc;              // 0 for rows past N
+    __syncthreads();
+    double mine = 0.0;
+    if (threadIdx.x == 0)
+        for (int w = 0; w < kAvRows; ++w) mine += sq[w];
+    finish_norm(mine, part, cnt, inv_out);
+}
+
+// vpart[chunk][c] = sum_{r in chunk} A[r][c] * (u[r] * su)   (rows in order; su = 1/|u|)
 template <bool ITER>
 __global__ void svid_atu_partial_kernel(const float* __restrict__ W, const float* __restrict__ g,
                                         const float* __restrict__ h, const uint32_t* __restrict__ S, int N, int K,
-                                        int k, int plane, const double* __restrict__ u, double* __restrict__ vpart)
+                                        int k, int plane, const double* __restrict__ u, const double* __restrict__ sup,
+                                        double* __restrict__ vpart)
 {
+    const double su = *sup;
     const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int chunk = blockIdx.y;
     if (c >= K) return;
     const int64_t r0 = (int64_t)N * chunk / kRowChunks, r1 = (int64_t)N * (chunk + 1) / kRowChunks;
     double acc = 0.0;
-    for (int64_t r = r0; r < r1; ++r) acc += abs_target<ITER>(W, g, h, S, N, K, k, plane, r, c) * u[r];
+    for (int64_t r = r0; r < r1; ++r) acc += abs_target<ITER>(W, g, h, S, N, K, k, plane, r, c) * (u[r] * su);
     vpart[(int64_t)chunk * K + c] = acc;
 }
 
-__global__ void svid_atu_reduce_kernel(const double* __restrict__ vpart, int K, double* __restrict__ v)
+// v[c] = sum of the chunks in order; 1 / |v| through the CTAs' sums of squares.
+__global__ void __launch_bounds__(256)
+svid_atu_reduce_kernel(const double* __restrict__ vpart, int K, double* __restrict__ v, double* part,
+                       unsigned* cnt, double* inv_v)
 {
+    __shared__ double sq[256];
     const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= K) return;
     double acc = 0.0;
-    for (int ch = 0; ch < kRowChunks; ++ch) acc += vpart[(int64_t)ch * K + c];
-    v[c] = acc;
+    if (c < K) {
+        for (int ch = 0; ch < kRowChunks; ++ch) acc += vpart[(int64_t)ch * K + c];
+        v[c] = acc;
+    }
+    sq[threadIdx.x] = acc * acc;
+    __syncthreads();
+    for (int st = 128; st > 0; st >>= 1) {
+        if ((int)threadIdx.x < st) sq[threadIdx.x] += sq[threadIdx.x + st];
+        __syncthreads();
+    }
+    finish_norm(sq[0], part, cnt, inv_v);
 }
 
 // Fixed-order block reduction of sum(a[j] * b[j]) by one CTA of 1024 threads.
@@ -143,27 +204,28 @@ __device__ double block_dot(const double* a, const double* b, int64_t n)
     return r;
 }
 
-__global__ void svid_normalize_kernel(double* __restrict__ x, int64_t n)
-{
-    const double nrm = sqrt(block_dot(x, x, n));
-    for (int64_t j = threadIdx.x; j < n; j += blockDim.x) x[j] = nrm > 0.0 ? x[j] / nrm : 0.0;
-}
-
-__global__ void svid_init_kernel(double* __restrict__ v, int K)
+// v0 = 1/sqrt(K) (already unit: 1/|v0| = 1); counters armed.
+__global__ void svid_init_kernel(double* __restrict__ v, int K, double* scal, unsigned* cnt)
 {
     for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < K; j += (int64_t)gridDim.x * blockDim.x)
         v[j] = 1.0 / sqrt((double)K);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        scal[1] = 1.0;
+        cnt[0] = 0u;
+    }
 }
 
-// sigma = u^T (A v); g_i = fp32(sqrt(sigma) u); h_i = fp32(sqrt(sigma) v)
+// With u = u_raw * su, v = v_raw * sv and av = A v:
+// sigma = u^T av; g_i = fp32(sqrt(sigma) u); h_i = fp32(sqrt(sigma) v)
 __global__ void svid_finish_kernel(const double* __restrict__ u, const double* __restrict__ v,
-                                   const double* __restrict__ av, int N, int K, int plane,
-                                   float* __restrict__ g, float* __restrict__ h)
+                                   const double* __restrict__ av, const double* __restrict__ scal, int N, int K,
+                                   int plane, float* __restrict__ g, float* __restrict__ h)
 {
-    const double sigma = block_dot(u, av, N);
+    const double su = scal[0], sv = scal[1];
+    const double sigma = block_dot(u, av, N) * su;
     const double rs = sigma > 0.0 ? sqrt(sigma) : 0.0;
-    for (int64_t r = threadIdx.x; r < N; r += blockDim.x) g[(int64_t)plane * N + r] = (float)(rs * u[r]);
-    for (int64_t c = threadIdx.x; c < K; c += blockDim.x) h[(int64_t)plane * K + c] = (float)(rs * v[c]);
+    for (int64_t r = threadIdx.x; r < N; r += blockDim.x) g[(int64_t)plane * N + r] = (float)(rs * (u[r] * su));
+    for (int64_t c = threadIdx.x; c < K; c += blockDim.x) h[(int64_t)plane * K + c] = (float)(rs * (v[c] * sv));
 }
 
 // Signs of the greedy pass (the fp32 recurrence of rb_pack): one warp per
@@ -209,27 +271,28 @@ template <bool ITER>
 rb_status svid_plane(const float* W, float* g, float* h, const uint32_t* S, int N, int K, int k, int plane,
                      int iters, const SvidWs& ws, cudaStream_t stream)
 {
-    const dim3 av_grid((unsigned)((N + 7) / 8)), av_blk(256);
+    const dim3 av_grid((unsigned)((N + kAvRows - 1) / kAvRows)), av_blk(kAvRows * 32);
     const dim3 atu_grid((unsigned)((K + 255) / 256), kRowChunks), atu_blk(256);
     const dim3 red_grid((unsigned)((K + 255) / 256)), red_blk(256);
-    rb_status st = launch(svid_init_kernel, dim3(8), dim3(256), 0, stream, false, ws.v, K);
+    double* inv_u = ws.scal;
+    double* inv_v = ws.scal + 1;
+    rb_status st = launch(svid_init_kernel, dim3(8), dim3(256), 0, stream, false, ws.v, K, ws.scal, ws.cnt);
     for (int it = 0; it < iters && st == RB_OK; ++it) {
         st = launch(svid_av_kernel<ITER>, av_grid, av_blk, 0, stream, false, W, (const float*)g, (const float*)h, S,
-                    N, K, k, plane, (const double*)ws.v, ws.u);
-        if (st == RB_OK) st = launch(svid_normalize_kernel, dim3(1), dim3(1024), 0, stream, false, ws.u, (int64_t)N);
+                    N, K, k, plane, (const double*)ws.v, (const double*)inv_v, ws.u, ws.part, ws.cnt, inv_u);
         if (st == RB_OK)
             st = launch(svid_atu_partial_kernel<ITER>, atu_grid, atu_blk, 0, stream, false, W, (const float*)g,
-                        (const float*)h, S, N, K, k, plane, (const double*)ws.u, ws.vpart);
+                        (const float*)h, S, N, K, k, plane, (const double*)ws.u, (const double*)inv_u, ws.vpart);
         if (st == RB_OK) st = launch(svid_atu_reduce_kernel, red_grid, red_blk, 0, stream, false,
-                                     (const double*)ws.vpart, K, ws.v);
-        if (st == RB_OK) st = launch(svid_normalize_kernel, dim3(1), dim3(1024), 0, stream, false, ws.v, (int64_t)K);
+                                     (const double*)ws.vpart, K, ws.v, ws.part, ws.cnt, inv_v);
     }
-    if (st == RB_OK)
+    if (st == RB_OK)                              // A v with the final v, no norm needed
         st = launch(svid_av_kernel<ITER>, av_grid, av_blk, 0, stream, false, W, (const float*)g, (const float*)h, S,
-                    N, K, k, plane, (const double*)ws.v, ws.av);
+                    N, K, k, plane, (const double*)ws.v, (const double*)inv_v, ws.av, ws.part, ws.cnt,
+                    (double*)nullptr);
     if (st == RB_OK)
         st = launch(svid_finish_kernel, dim3(1), dim3(1024), 0, stream, false, (const double*)ws.u,
-                    (const double*)ws.v, (const double*)ws.av, N, K, plane, g, h);
+                    (const double*)ws.v, (const double*)ws.av, (const double*)ws.scal, N, K, plane, g, h);
     return st;
 }
 
@@ -298,4 +361,21 @@ extern "C" rb_status rb_svid_iterative(const float* W, int n_out, int k_in, int 
         }
     }
     return st;
+}
+
+extern "C" size_t rb_svid_pack_workspace_bytes(int n_out, int k_in, int k_planes)
+{
+    return rb_svid_iterative_workspace_bytes(n_out, k_in, k_planes);
+}
+
+extern "C" rb_status rb_svid_pack(const float* W, int n_out, int k_in, int k_planes, int sweeps, int iters,
+                                  float* g, float* h, uint32_t* planes, uint16_t* g16, uint16_t* h16,
+                                  void* workspace, size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream)
+{
+    if (!planes || !g16 || !h16) return RB_ERR_ARG;
+    if (!aligned16(planes) || !aligned16(g16) || !aligned16(h16) || (dev_status && !aligned16(dev_status)))
+        return RB_ERR_ALIGN;
+    rb_status st = rb_svid_iterative(W, n_out, k_in, k_planes, sweeps, iters, g, h, workspace, workspace_bytes, stream);
+    if (st != RB_OK) return st;
+    return rb_pack(W, g, h, n_out, k_in, k_planes, planes, g16, h16, dev_status, stream);
 }

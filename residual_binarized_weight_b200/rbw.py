@@ -44,6 +44,8 @@ SIGNATURES = {
     "rb_svid_greedy": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "rb_svid_iterative_workspace_bytes": (_sz, [_i32, _i32, _i32]),
     "rb_svid_iterative": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "rb_svid_pack_workspace_bytes": (_sz, [_i32, _i32, _i32]),
+    "rb_svid_pack": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
 }
 
 
@@ -289,3 +291,19 @@ def svid_iterative(W, k_planes, sweeps=20, iters=20, ws=None, stream=None):
                                  ws.numel(), _stream(stream))
     _check("rb_svid_iterative", st)
     return g, h
+
+
+def svid_pack(W, k_planes, sweeps=0, iters=20, out: PackedLayer | None = None, ws=None, dev_status=None,
+              stream=None):
+    """rb_svid_pack: fp32 W [N][K] (CUDA) -> (PackedLayer, g, h): SVID scales (greedy when sweeps = 0,
+    else iterative) and the packed planes, in one device-side call."""
+    N, K = W.shape
+    out = out or PackedLayer(N, K, k_planes, W.device)
+    g = torch.empty(k_planes, N, dtype=torch.float32, device=W.device)
+    h = torch.empty(k_planes, K, dtype=torch.float32, device=W.device)
+    nbytes = int(lib().rb_svid_pack_workspace_bytes(N, K, k_planes))
+    ws = ws if ws is not None else workspace(nbytes, W.device)
+    st = lib().rb_svid_pack(_ptr(W), N, K, k_planes, sweeps, iters, _ptr(g), _ptr(h), _ptr(out.planes),
+                            _ptr(out.g16), _ptr(out.h16), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream))
+    _check("rb_svid_pack", st)
+    return out, g, h

@@ -67,6 +67,27 @@ def test_gemm_ragged(N, K, k, M):
         cases.check_y(Yg, Yr, cases.abs_bound(g16, h16, X), bf16=ydt == torch.bfloat16, per_elem=1e-4)
 
 
+@pytest.mark.parametrize("N,K,k,M", [(4097, 800, 2, 1000), (4000, 1056, 1, 2000), (2100, 544, 3, 1500),
+                                     (1000, 4096, 4, 1300), (4096, 4096, 2, 2048), (300, 14336, 2, 9000)])
+def test_gemm_many_tiles_match_oracle(N, K, k, M):
+    """Grids of several waves (ragged rows, tokens and K; k = 1..4; a long K
+    with a large M): sampled rows and tokens against the oracle."""
+    rng = np.random.default_rng(N + K + 3 * k + M)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=4)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    X = synth.activations(M, K, seed=N + M + k)
+    st = torch.zeros(4, dtype=torch.int32, device="cuda")
+    for ydt in (torch.float32, torch.bfloat16):
+        Yg = run_gemm(L, X, ydt, dev_status=st)
+        assert int(st[0].item()) == 0
+        rows, toks = sample(N, 200, 3), sample(M, 80, 4)
+        Yr = oracle.apply(planes, g16, h16, N, K, k, X, rows=rows, toks=toks)
+        cases.check_y(Yg[np.ix_(toks, rows)], Yr, cases.abs_bound(g16, h16, X[toks], rows),
+                      bf16=ydt == torch.bfloat16, per_elem=1e-4)
+
+
 def test_gemm_matches_gemv_small_m():
     """For M <= 64 both entry points compute the same product (to fp32 rounding)."""
     W, g, h = cases.layer_case(1, 0, 2)
@@ -145,3 +166,33 @@ def test_gemm_wait_limit_expiry_reports_timeout_and_context_survives(N, K, k, M)
     with pytest.raises(rbw.RbError) as e:
         rbw.gemm_wait_limit(L, Xd, 2_000_000_000, ws=ws)
     assert e.value.status == rbw.RB_ERR_ARG
+
+
+def test_gemm_wait_limit_expiry_many_ctas_then_correct():
+    """The bounded-wait error path on a grid of several waves (4096 x 1024,
+    M = 2048): limit 0 ends the call with RB_DEV_TIMEOUT after every CTA drains
+    its loads and MMAs; the next rb_gemm on the stream matches the oracle on
+    sampled outputs."""
+    N, K, k, M = 4096, 1024, 2, 2048
+    rng = np.random.default_rng(11)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=4)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    X = synth.activations(M, K, seed=5)
+    Xd = cases.to_dev(X)
+    ws = rbw.workspace(rbw.gemm_workspace_bytes(N, K, k, M))
+    rows, toks = sample(N, 200, 5), sample(M, 60, 6)
+    Yr = oracle.apply(planes, g16, h16, N, K, k, X, rows=rows, toks=toks)
+    bound = cases.abs_bound(g16, h16, X[toks], rows)
+    for _ in range(2):
+        st = torch.zeros(4, dtype=torch.int32, device="cuda")
+        rbw.gemm_wait_limit(L, Xd, 0, ws=ws, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st[0].item()) & rbw.RB_DEV_TIMEOUT
+        st = torch.zeros(4, dtype=torch.int32, device="cuda")
+        Y = rbw.gemm(L, Xd, ws=ws, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st[0].item()) == 0
+        Yg = Y.cpu().numpy().astype(np.float64)
+        cases.check_y(Yg[np.ix_(toks, rows)], Yr, bound, bf16=False, per_elem=1e-4)

@@ -69,3 +69,31 @@ def test_svid_iterative_lowers_the_packed_error():
         What = oracle.apply(planes, g16, h16, 512, 1024, 2, synth.to_bf16_bits(eye))   # rows of What^T
         errs.append(np.linalg.norm(W.astype(np.float64) - What.T))
     assert errs[1] <= errs[0] * 1.001, errs
+
+
+@pytest.mark.parametrize("wl,k,sweeps,shape", [(1, 2, 0, (512, 1024)), (1, 2, 3, (256, 512)), (4, 3, 0, (300, 544)),
+                                               (2, 2, 0, None)])
+def test_svid_pack_one_call(wl, k, sweeps, shape):
+    """rb_svid_pack (SVID scales then the residual sign planes, one device-side
+    call): the scales agree with the oracle's SVID, and the planes and fp16
+    scales are bit-exact with the oracle's packer run on those scales."""
+    layer = synth.workload(wl).layers[0]
+    W = synth.weights(layer, *(shape or (None, None)))
+    N, K = W.shape
+    if sweeps:
+        g_ref, h_ref = oracle.svid_iterative(W, k, sweeps=sweeps, iters=20)
+    else:
+        g_ref, h_ref = oracle.svid_greedy(W, k, iters=20)
+    st = torch.zeros(4, dtype=torch.int32, device="cuda")
+    L, g, h = rbw.svid_pack(cases.to_dev(W), k, sweeps=sweeps, iters=20, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st[0].item()) == 0
+    g, h = g.cpu().numpy(), h.cpu().numpy()
+    for a, b in ((g, g_ref), (h, h_ref)):
+        err = np.abs(a.astype(np.float64) - b) / np.maximum(np.abs(b).max(axis=1, keepdims=True), 1e-30)
+        assert err.max() < 1e-5, err.max()
+    planes, g16, h16, st2, _ = oracle.pack(W, g, h, k)
+    assert st2 == 0
+    assert np.array_equal(cases.to_host(L.planes, np.uint32), planes)
+    assert np.array_equal(cases.to_host(L.g16, np.uint16).reshape(k, N), g16)
+    assert np.array_equal(cases.to_host(L.h16, np.uint16).reshape(k, K), h16)
