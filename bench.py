@@ -88,6 +88,24 @@ class Dist:
             dist.destroy_process_group()
 
 
+def rowsplit_gather(dist, y_local, n_out, shard_bounds):
+    """Row-parallel split: every rank holds Y[:, row0_r:row1_r] ([M][rows_r], a
+    torch tensor); returns the full [M][n_out] on every rank.  Shards are padded
+    to the largest one for one all_gather, then cut and concatenated along N."""
+    import torch
+    if not dist.pg:
+        return y_local
+    import torch.distributed as td
+    bounds = [shard_bounds(n_out, dist.world, r) for r in range(dist.world)]
+    width = max(b1 - b0 for b0, b1 in bounds)
+    M = y_local.shape[0]
+    pad = torch.zeros(M, width, dtype=y_local.dtype, device=y_local.device)
+    pad[:, :y_local.shape[1]] = y_local
+    parts = [torch.empty_like(pad) for _ in range(dist.world)]
+    td.all_gather(parts, pad)
+    return torch.cat([p[:, :b1 - b0] for p, (b0, b1) in zip(parts, bounds)], dim=1)
+
+
 def assemble_line(*, value, unit, n_gpus, steps, warmup, ms_per_step, extra) -> dict:
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": n_gpus, "steps": steps,
             "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -652,6 +670,38 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
                          stream) / LAYERS
     out["input_grad_M1_batch96"] = {"us_per_layer": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9}
     del layers, tlayers
+    # device scale derivation: greedy SVID (20 power iterations per plane) and the
+    # one-call deployment path rb_svid_pack (SVID scales, then planes + fp16 scales)
+    t = time_events(torch, lambda: rbw.svid_greedy(W, K_PLANES, iters=20, stream=stream), 3, stream)
+    out["svid_greedy"] = {"us": t * 1e6, "iters": 20, "planes": K_PLANES,
+                          "W_passes": K_PLANES * (2 * 20 + 1), "W_bytes": 4 * N_OUT * K_IN}
+    Ls = rbw.PackedLayer(N_OUT, K_IN, K_PLANES, dev)
+    t = time_events(torch, lambda: rbw.svid_pack(W, K_PLANES, sweeps=0, iters=20, out=Ls, stream=stream), 3, stream)
+    out["svid_pack_greedy"] = {"us": t * 1e6}
+    t = time_events(torch, lambda: rbw.svid_pack(W, K_PLANES, sweeps=2, iters=20, out=Ls, stream=stream), 1, stream)
+    out["svid_pack_2_sweeps"] = {"us": t * 1e6}
+    # plain row-major words <-> storage layout (one read and one write of the planes)
+    rm = rbw.planes_to_rowmajor(Lp, stream=stream)
+    t = time_graph_calls(torch, lambda: rbw.planes_from_rowmajor(rm, N_OUT, K_IN, K_PLANES, out=Ls, stream=stream),
+                         20, stream)
+    out["planes_from_rowmajor"] = {"us": t * 1e6, "GBps": 2 * Lp.packed_bytes() / t / 1e9}
+    # coupled-training gradients of one layer at M = 2048 tokens: G = dY^T X on tcgen05 plus dg, dh
+    try:
+        Mt = 2048
+        Xt = torch.from_numpy(synth.activations(Mt, K_IN, seed=21).view(np.int16)).to(dev)
+        dYt = torch.from_numpy(synth.activations(Mt, N_OUT, seed=22).view(np.int16)).to(dev)
+        dWt = torch.empty(N_OUT, K_IN, dtype=torch.float32, device=dev)
+        dgt = torch.empty(K_PLANES, N_OUT, dtype=torch.float32, device=dev)
+        dht = torch.empty(K_PLANES, K_IN, dtype=torch.float32, device=dev)
+        wsg = rbw.workspace(int(rbw.lib().rb_qat_backward_workspace_bytes(N_OUT, K_IN, K_PLANES)), dev)
+        t = time_events(torch, lambda: rbw.qat_backward(Lp, g, h, Xt, dYt, dW=dWt, dg=dgt, dh=dht, ws=wsg,
+                                                        stream=stream), 10, stream)
+        fl = 2.0 * Mt * N_OUT * K_IN
+        out["qat_backward_M2048"] = {"us": t * 1e6, "G_TFLOPs": fl / t / 1e12, "flops": fl,
+                                     "frac_of_bf16_peak": fl / t / 1e12 / bf16_peak}
+        del Xt, dYt, dWt, wsg
+    except rbw.RbError as e:
+        out["qat_backward_M2048"] = {"unavailable": str(e)}
     # rb_gemm at M = 2048 on the prefill shape
     try:
         X = torch.from_numpy(synth.activations(2048, K_IN, seed=7).view(np.int16)).to(dev)

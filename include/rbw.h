@@ -123,6 +123,23 @@ RB_API rb_status rb_planes_to_rowmajor(const uint32_t *planes, int n_out, int k_
                                        uint32_t *rowmajor, cudaStream_t stream);
 
 /*
+ * rb_shard_rows -- rows [row0, row0 + rows) of a packed layer as a packed layer
+ * of their own, for a row-parallel split over P GPUs: rank r applies its shard
+ * to the full X and the [M][rows] outputs are concatenated along N (an
+ * all-gather).  The pages give no multi-GPU scheme; since every output row of
+ * Y = sum_i g_i .* (B_i (h_i .* X)) depends only on its own sign rows and g
+ * values, the split needs no other exchange.
+ *   row0         a multiple of 32 (RB_ERR_SHAPE otherwise), rows >= 1,
+ *                row0 + rows <= N.
+ *   planes_out   rb_packed_words(rows, K, k) words (every word written; rows
+ *                past `rows` in the last tile are zero).
+ *   g16_out      [k][rows] fp16, copied from layer->g16.
+ * The shard's h16 is layer->h16 itself.  Must not overlap layer->planes.
+ */
+RB_API rb_status rb_shard_rows(const rb_layer_t *layer, int row0, int rows, uint32_t *planes_out,
+                               uint16_t *g16_out, cudaStream_t stream);
+
+/*
  * rb_pack -- derive and bit-pack the residual sign planes (RaBiT, Algorithm 2
  * forward pass; deployment freezes these planes and drops W).
  *   W        [N][K] fp32 latent weight.

@@ -107,3 +107,54 @@ extern "C" rb_status rb_planes_to_rowmajor(const uint32_t* planes, int n_out, in
     return launch(to_rowmajor_kernel, dim3(layout_grid((int64_t)nr)), dim3(kLayoutThreads), 0, stream, false,
                   planes, n_out, k_in, k_planes, rowmajor);
 }
+
+// ---------------------------------------------------------------- row shards
+// Rows [row0, row0 + rows) of a layer as a layer of their own (row0 a multiple
+// of 32): every (plane, slice, row tile) block of the shard is the source
+// block of tile row0/32 + t, with the rows past `rows` of a ragged last tile
+// cleared; g16 rows are copied, h16 is the same array for every shard.  This
+// is the per-GPU part of a row-parallel split (each GPU applies its shard to
+// the full X and the outputs are concatenated along N).
+namespace rbw {
+namespace {
+
+__global__ void __launch_bounds__(kLayoutThreads)
+shard_rows_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ g16, int N, int K, int kp,
+                  int row0, int rows, uint32_t* __restrict__ out, uint16_t* __restrict__ g_out)
+{
+    const int64_t S = num_slices(K), Nt = num_row_tiles(N), Ntd = num_row_tiles(rows);
+    const int64_t t0 = row0 / 32;
+    const int64_t total = (int64_t)kp * S * Ntd * 256, ng = (int64_t)kp * rows;
+    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < total + ng;
+         x += (int64_t)gridDim.x * blockDim.x) {
+        if (x < total) {
+            const int64_t blk = x >> 8, t = blk % Ntd, s = (blk / Ntd) % S, i = blk / (Ntd * S);
+            const int rho = (int)(x & 31);
+            out[x] = t * 32 + rho < rows ? __ldg(planes + block_index((int)i, s, t0 + t, S, Nt) * 256 + (x & 255))
+                                         : 0u;
+        } else {
+            const int64_t y = x - total, i = y / rows, r = y % rows;
+            g_out[y] = g16[i * N + row0 + r];
+        }
+    }
+}
+
+}  // namespace
+}  // namespace rbw
+
+extern "C" rb_status rb_shard_rows(const rb_layer_t* layer, int row0, int rows, uint32_t* planes_out,
+                                   uint16_t* g16_out, cudaStream_t stream)
+{
+    if (!layer || !layer->planes || !layer->g16 || !planes_out || !g16_out || layer->reserved != 0) return RB_ERR_ARG;
+    if (layer->k_planes < 1 || layer->k_planes > 8) return RB_ERR_ARG;
+    if (layer->n_out < 1 || layer->k_in < 32 || layer->k_in % 32 != 0) return RB_ERR_SHAPE;
+    if (row0 < 0 || row0 % 32 != 0 || rows < 1 || (int64_t)row0 + rows > layer->n_out) return RB_ERR_SHAPE;
+    if (!aligned16(layer->planes) || !aligned16(planes_out) || !aligned16(g16_out)) return RB_ERR_ALIGN;
+    const size_t nw = rb_packed_words(rows, layer->k_in, layer->k_planes);
+    const size_t nsrc = rb_packed_words(layer->n_out, layer->k_in, layer->k_planes);
+    if (overlaps(layer->planes, nsrc * 4, planes_out, nw * 4)) return RB_ERR_ARG;
+    if (!device_is_sm100()) return RB_ERR_UNSUPPORTED;
+    return launch(shard_rows_kernel, dim3(layout_grid((int64_t)nw + (int64_t)layer->k_planes * rows)),
+                  dim3(kLayoutThreads), 0, stream, false, layer->planes, layer->g16, layer->n_out, layer->k_in,
+                  layer->k_planes, row0, rows, planes_out, g16_out);
+}

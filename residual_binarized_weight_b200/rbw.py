@@ -36,6 +36,7 @@ SIGNATURES = {
     "rb_gemm_noalloc": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _u32, _vp]),
     "rb_transpose_planes": (_i32, [_vp, _vp, _vp]),
     "rb_rowmajor_words": (_sz, [_i32, _i32, _i32]),
+    "rb_shard_rows": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp]),
     "rb_planes_from_rowmajor": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "rb_planes_to_rowmajor": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "rb_qat_backward_workspace_bytes": (_sz, [_i32, _i32, _i32]),
@@ -307,3 +308,20 @@ def svid_pack(W, k_planes, sweeps=0, iters=20, out: PackedLayer | None = None, w
                             _ptr(out.g16), _ptr(out.h16), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream))
     _check("rb_svid_pack", st)
     return out, g, h
+
+
+def shard_bounds(n_out, world, rank):
+    """Rows [row0, row1) of rank `rank` in a row-parallel split of n_out rows over
+    `world` ranks: contiguous ranges starting on 32-row tiles, as even as that allows."""
+    tiles = (n_out + 31) // 32
+    t0, t1 = tiles * rank // world, tiles * (rank + 1) // world
+    return min(32 * t0, n_out), min(32 * t1, n_out)
+
+
+def shard_rows(layer: PackedLayer, row0, rows, stream=None):
+    """rb_shard_rows: rows [row0, row0 + rows) of `layer` as a PackedLayer sharing its h16."""
+    out = PackedLayer(rows, layer.k_in, layer.k_planes, layer.planes.device, h16=layer.h16)
+    L = layer.struct()
+    st = lib().rb_shard_rows(ctypes.byref(L), row0, rows, _ptr(out.planes), _ptr(out.g16), _stream(stream))
+    _check("rb_shard_rows", st)
+    return out

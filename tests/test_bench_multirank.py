@@ -139,3 +139,55 @@ def test_clock_sampler_keeps_samples_inside_the_timed_region(tmp_path, monkeypat
     assert c["sm_mhz"] == 1950.0 and c["sm_max_mhz"] == 1965.0
     assert c["reasons"] == ["sw_power_cap"]
     assert not bench.clocks_rejected(c)
+
+
+def _shard_bounds(n_out, world, rank):
+    from residual_binarized_weight_b200.rbw import shard_bounds
+    return shard_bounds(n_out, world, rank)
+
+
+def _rowsplit_main(rank, world, port, out_path):
+    """Each rank applies its row shard (oracle planes of its rows; the
+    recurrence is row-local) and the shards are all-gathered along N."""
+    os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    import numpy as np
+    import torch
+    import oracle
+    from residual_binarized_weight_b200 import synth
+    d = bench.Dist()
+    d.init("gloo")
+    N, K, k, M = 300, 256, 2, 3                       # ragged: 10 row tiles over the ranks
+    rng = np.random.default_rng(4)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=4)
+    X = synth.activations(M, K, seed=2)
+    r0, r1 = _shard_bounds(N, world, rank)
+    planes, g16, h16, _, _ = oracle.pack(W[r0:r1], g[:, r0:r1], h, k)
+    y_local = torch.from_numpy(oracle.apply(planes, g16, h16, r1 - r0, K, k, X))
+    y = bench.rowsplit_gather(d, y_local, N, _shard_bounds)
+    if rank == 0:
+        planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+        ref = oracle.apply(planes, g16, h16, N, K, k, X)
+        np.save(out_path, np.stack([y.numpy(), ref]))
+    d.close()
+
+
+def test_row_split_all_gather_reassembles_the_full_output(tmp_path):
+    out = str(tmp_path / "rs.npy")
+    mp.start_processes(_rowsplit_main, args=(2, _free_port(), out), nprocs=2, join=True, start_method="spawn")
+    import numpy as np
+    y, ref = np.load(out)
+    assert y.shape == ref.shape == (3, 300)
+    assert np.array_equal(y, ref)                     # the same float64 oracle on every row
+
+
+def test_shard_bounds_tile_aligned_and_complete():
+    from residual_binarized_weight_b200.rbw import shard_bounds
+    for n in (1, 31, 32, 300, 4096, 11008):
+        for world in (1, 2, 3, 4, 8):
+            b = [shard_bounds(n, world, r) for r in range(world)]
+            assert b[0][0] == 0 and b[-1][1] == n
+            for (a0, a1), (c0, c1) in zip(b, b[1:]):
+                assert a1 == c0
+            assert all(r0 % 32 == 0 and r0 <= r1 for r0, r1 in b)

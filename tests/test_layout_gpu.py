@@ -74,3 +74,45 @@ def test_rowmajor_argument_errors():
     with pytest.raises(rbw.RbError) as e:
         rbw.planes_to_rowmajor(L, out=buf[1:])           # 4-byte offset
     assert e.value.status == rbw.RB_ERR_ALIGN
+
+
+@pytest.mark.parametrize("N,K,k,world", [(4096, 4096, 2, 4), (300, 544, 3, 2), (11008, 4096, 2, 8), (100, 256, 1, 3)])
+def test_row_shards_are_the_planes_of_the_row_ranges(N, K, k, world):
+    """rb_shard_rows over a row-parallel split: each shard is bit for bit the
+    oracle's packing of its rows (the recurrence is row-local), and the shards'
+    outputs, concatenated along N, match the oracle's output of the whole layer."""
+    rng = np.random.default_rng(N + K + k)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=4)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    X = synth.activations(2, K, seed=9)
+    Xd = cases.to_dev(X)
+    parts = []
+    for r in range(world):
+        r0, r1 = rbw.shard_bounds(N, world, r)
+        if r1 == r0:
+            continue
+        Sh = rbw.shard_rows(L, r0, r1 - r0)
+        torch.cuda.synchronize()
+        sp, sg, _, _, _ = oracle.pack(W[r0:r1], g[:, r0:r1], h, k)
+        assert np.array_equal(cases.to_host(Sh.planes, np.uint32), sp)
+        assert np.array_equal(cases.to_host(Sh.g16, np.uint16).reshape(k, r1 - r0), sg)
+        parts.append(rbw.gemv(Sh, Xd))
+    Y = torch.cat(parts, dim=1)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([np.arange(min(N, 64)), np.arange(max(0, N - 64), N),
+                                     rng.choice(N, min(N, 200), replace=False)]))
+    Yr = oracle.apply(planes, g16, h16, N, K, k, X, rows=rows)
+    cases.check_y(Y.cpu().numpy().astype(np.float64)[:, rows], Yr, cases.abs_bound(g16, h16, X, rows), bf16=False,
+                  per_elem=1e-4)
+
+
+def test_shard_rows_argument_errors():
+    L = rbw.PackedLayer(128, 256, 2)
+    with pytest.raises(rbw.RbError) as e:
+        rbw.shard_rows(L, 16, 32)                        # not on a 32-row tile
+    assert e.value.status == rbw.RB_ERR_SHAPE
+    with pytest.raises(rbw.RbError) as e:
+        rbw.shard_rows(L, 96, 64)                        # past the last row
+    assert e.value.status == rbw.RB_ERR_SHAPE
