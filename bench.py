@@ -789,7 +789,8 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="skip the extra per-row timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--mode", choices=["full", "gemv-kernel", "gemv-batch-kernel", "pack-kernel", "gemm-kernel"],
+    ap.add_argument("--mode", choices=["full", "gemv-kernel", "gemv-batch-kernel", "pack-kernel", "gemm-kernel",
+                                       "grad-kernel", "svid-kernel", "transpose-kernel", "rowmajor-kernel"],
                     default="full",
                     help="kernel-only modes run one kernel a few times (used for ncu captures)")
     ap.add_argument("--launches", type=int, default=20)
@@ -817,6 +818,24 @@ def run_kernel_mode(args):
     if args.mode == "pack-kernel":
         for _ in range(args.launches):
             rbw.pack(W, g, h, K_PLANES, out=base)
+    elif args.mode == "grad-kernel":                 # rb_qat_backward at M tokens (default 2048)
+        M = args.M if args.M > 1 else 2048
+        X = torch.from_numpy(synth.activations(M, K_IN, seed=21).view(np.int16)).to(dev)
+        dY = torch.from_numpy(synth.activations(M, N_OUT, seed=22).view(np.int16)).to(dev)
+        for _ in range(args.launches):
+            rbw.qat_backward(base, g, h, X, dY)
+    elif args.mode == "svid-kernel":                 # greedy SVID, 2 power iterations per plane
+        for _ in range(args.launches):
+            rbw.svid_greedy(W, K_PLANES, iters=2)
+    elif args.mode == "transpose-kernel":
+        t = rbw.transpose(base)
+        for _ in range(args.launches):
+            rbw.transpose(base, out=t)
+    elif args.mode == "rowmajor-kernel":
+        rm = rbw.planes_to_rowmajor(base)
+        L2 = rbw.PackedLayer(N_OUT, K_IN, K_PLANES, dev)
+        for _ in range(args.launches):
+            rbw.planes_from_rowmajor(rm, N_OUT, K_IN, K_PLANES, out=L2)
     else:
         nl = LAYERS                         # distinct layers: 96 x 4.2 MB of planes, larger than L2
         layers = []
