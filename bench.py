@@ -699,7 +699,15 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
         fl = 2.0 * Mt * N_OUT * K_IN
         out["qat_backward_M2048"] = {"us": t * 1e6, "G_TFLOPs": fl / t / 1e12, "flops": fl,
                                      "frac_of_bf16_peak": fl / t / 1e12 / bf16_peak}
-        del Xt, dYt, dWt, wsg
+        # the matching forward: planes derived from fp32 W (pack kernel), then the tcgen05 GEMM with fp32 g
+        Yt = torch.empty(Mt, N_OUT, dtype=torch.float32, device=dev)
+        wsf = rbw.workspace(rbw.qat_forward_workspace_bytes(N_OUT, K_IN, K_PLANES, Mt), dev)
+        t = time_events(torch, lambda: rbw.qat_forward(W, g, h, K_PLANES, Xt, Y=Yt, ws=wsf, stream=stream),
+                        10, stream)
+        fl = 2.0 * K_PLANES * Mt * N_OUT * K_IN
+        out["qat_forward_M2048"] = {"us": t * 1e6, "TFLOPs": fl / t / 1e12, "flops": fl,
+                                    "frac_of_bf16_peak": fl / t / 1e12 / bf16_peak}
+        del Xt, dYt, dWt, wsg, Yt, wsf
     except rbw.RbError as e:
         out["qat_backward_M2048"] = {"unavailable": str(e)}
     # rb_gemm at M = 2048 on the prefill shape
@@ -790,7 +798,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--mode", choices=["full", "gemv-kernel", "gemv-batch-kernel", "pack-kernel", "gemm-kernel",
-                                       "grad-kernel", "svid-kernel", "transpose-kernel", "rowmajor-kernel"],
+                                       "grad-kernel", "qat-forward-kernel", "svid-kernel", "transpose-kernel",
+                                       "rowmajor-kernel"],
                     default="full",
                     help="kernel-only modes run one kernel a few times (used for ncu captures)")
     ap.add_argument("--launches", type=int, default=20)
@@ -824,6 +833,11 @@ def run_kernel_mode(args):
         dY = torch.from_numpy(synth.activations(M, N_OUT, seed=22).view(np.int16)).to(dev)
         for _ in range(args.launches):
             rbw.qat_backward(base, g, h, X, dY)
+    elif args.mode == "qat-forward-kernel":          # rb_qat_forward at M tokens (default 2048)
+        M = args.M if args.M > 1 else 2048
+        X = torch.from_numpy(synth.activations(M, K_IN, seed=21).view(np.int16)).to(dev)
+        for _ in range(args.launches):
+            rbw.qat_forward(W, g, h, K_PLANES, X)
     elif args.mode == "svid-kernel":                 # greedy SVID, 2 power iterations per plane
         for _ in range(args.launches):
             rbw.svid_greedy(W, K_PLANES, iters=2)

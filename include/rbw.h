@@ -285,6 +285,33 @@ RB_API rb_status rb_gemm_noalloc(const rb_layer_t *layer, const uint16_t *X, int
 RB_API rb_status rb_transpose_planes(const rb_layer_t *layer, uint32_t *planes_t, cudaStream_t stream);
 
 /*
+ * rb_qat_forward -- forward pass of one coupled-training layer (RaBiT,
+ * Algorithm 2 forward: the binary cores are derived from the latent weight
+ * at every step): Y = X What^T with What = sum_i diag(g_i) B_i diag(h_i), the
+ * B_i taken from W by the same fp32 recurrence as rb_pack and the trainable
+ * fp32 scales used as they are.  The planes are derived once into the
+ * workspace (one read of W), then the prefill GEMM runs on them with fp32 g
+ * in its epilogue: no fp16 copy of g is made.
+ *   W        [N][K] fp32 latent weight.   g, h  [k][N], [k][K] fp32.
+ *   X        [M][K] bfloat16 bits.        Y     [M][N] fp32 or bf16.
+ *   workspace  rb_qat_forward_workspace_bytes(N, K, k, M) bytes, 16-byte
+ *              aligned: the derived planes (rb_packed_words(N, K, k) words in
+ *              the storage layout, left there for the caller) followed by
+ *              rb_gemm's workspace.
+ * k = 1..8 with rb_gemm's limits on K (RB_ERR_UNSUPPORTED before any launch).
+ * Precision: the MMA operands are +-fp16(h_i) (round to nearest even) and
+ * fp16(x) with fp32 accumulation, g is applied in fp32, so |Y - exact| <=
+ * 2^-11 sum |g h x| plus the accumulation error.  dev_status gets
+ * RB_DEV_RANGE when an x or h overflows fp16, RB_DEV_NONFINITE for a NaN h or
+ * a NaN / infinite W, RB_DEV_TIMEOUT as rb_gemm.
+ */
+RB_API size_t rb_qat_forward_workspace_bytes(int n_out, int k_in, int k_planes, int M);
+RB_API rb_status rb_qat_forward(const float *W, const float *g, const float *h, int n_out, int k_in,
+                                int k_planes, const uint16_t *X, int M, void *Y, rb_dtype y_dtype,
+                                void *workspace, size_t workspace_bytes, int32_t *dev_status, unsigned flags,
+                                cudaStream_t stream);
+
+/*
  * rb_qat_backward -- gradients of one coupled-training layer (RaBiT,
  * Algorithm 2 backward pass: the signs derived on the fly from the latent
  * weight W are held constant, W takes the gradient of the effective weight,

@@ -51,6 +51,8 @@ def _load():
         lib.oracle_apply.restype = None
         lib.oracle_qat_backward.argtypes = [vp, vp, vp, i64, i64, i32, vp, vp, i64, vp, vp, vp, vp]
         lib.oracle_qat_backward.restype = i32
+        lib.oracle_qat_forward.argtypes = [vp, vp, vp, i64, i64, i32, vp, i64, vp, i64, vp, i64, vp]
+        lib.oracle_qat_forward.restype = i32
         lib.oracle_set_threads.argtypes = [i32]
         lib.oracle_set_threads.restype = None
         lib.oracle_threads.argtypes = []
@@ -205,6 +207,24 @@ def qat_backward(W, g, h, k: int, X_bf16, dY_bf16):
     st = _load().oracle_qat_backward(_p(W), _p(g), _p(h), N, K, k, _p(X), _p(dY), M,
                                      _p(dW), _p(dg), _p(dh), _p(dX))
     return int(st), dW, dg, dh, dX
+
+
+def qat_forward(W, g, h, k: int, X_bf16, rows=None, toks=None):
+    """float64 forward of the coupled-training layer: signs derived from W by the
+    fp32 recurrence, fp32 scales; returns (status, Y [len(toks)][len(rows)])."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    g = _c(g, np.float32).reshape(k, N)
+    h = _c(h, np.float32).reshape(k, K)
+    X = _c(X_bf16, np.uint16)
+    M = X.shape[0]
+    rows_a = None if rows is None else _c(rows, np.int64)
+    toks_a = None if toks is None else _c(toks, np.int64)
+    nr = N if rows_a is None else len(rows_a)
+    nt = M if toks_a is None else len(toks_a)
+    Y = np.zeros((nt, nr), np.float64)
+    st = _load().oracle_qat_forward(_p(W), _p(g), _p(h), N, K, k, _p(X), M, _p(rows_a), nr, _p(toks_a), nt, _p(Y))
+    return int(st), Y
 
 
 def svid_greedy(W, k: int, iters: int = 20):

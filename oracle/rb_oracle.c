@@ -443,6 +443,50 @@ int oracle_qat_backward(const float *W, const float *g, const float *h,
     return st;
 }
 
+/* Forward pass of the coupled-training layer (RaBiT, Algorithm 2 forward:
+ * the signs are derived on the fly from the latent weight W by the fp32
+ * recurrence, with the trainable fp32 scales):
+ *   Y[m][n] = sum_c X[m][c] * sum_i g_i[n] B_i[n][c] h_i[c]    (float64)
+ * X is bfloat16 bits [M][K].  rows / toks (nullable) select output rows n and
+ * tokens m; Y is [nt][nr].  Returns the status codes of oracle_pack's input
+ * scan (-1 bad arguments, 1 non-finite input). */
+int oracle_qat_forward(const float *W, const float *g, const float *h, int64_t N, int64_t K, int k,
+                       const uint16_t *X, int64_t M, const int64_t *rows, int64_t nr,
+                       const int64_t *toks, int64_t nt, double *Y)
+{
+    if (check_args(N, K, k) || M < 1) return -1;
+    int st = scan_inputs(W, g, h, N, K, k, NULL, NULL) == 1 ? 1 : 0;
+    #pragma omp parallel
+    {
+        float *R = (float *)malloc(sizeof(float) * (size_t)K);
+        unsigned char *bits = (unsigned char *)malloc((size_t)k * (size_t)K);
+        double *w = (double *)malloc(sizeof(double) * (size_t)K);
+        #pragma omp for schedule(static)
+        for (int64_t a = 0; a < nr; ++a) {
+            const int64_t r = rows ? rows[a] : a;
+            derive_row(W + r * K, g, h, N, K, k, r, R, bits);
+            for (int64_t c = 0; c < K; ++c) {        /* What[r][c] */
+                double v = 0.0;
+                for (int i = 0; i < k; ++i) {
+                    double s = bits[(int64_t)i * K + c] ? 1.0 : -1.0;
+                    v += (double)g[(int64_t)i * N + r] * s * (double)h[(int64_t)i * K + c];
+                }
+                w[c] = v;
+            }
+            for (int64_t b = 0; b < nt; ++b) {
+                const int64_t m = toks ? toks[b] : b;
+                double acc = 0.0;
+                for (int64_t c = 0; c < K; ++c) acc += decode_bfloat16(X[m * K + c]) * w[c];
+                Y[b * nr + a] = acc;
+            }
+        }
+        free(R);
+        free(bits);
+        free(w);
+    }
+    return st;
+}
+
 /* ------------------------------------------------------------------ */
 /* Greedy SVID scales (rank-1 of |R_{i-1}| per plane, power iteration)   */
 /* ------------------------------------------------------------------ */

@@ -123,6 +123,9 @@ constexpr uint64_t kWaitTimeoutNs = 1000000000ull;    // bound on each device-si
 rb_status gemm_with_timeout(const rb_layer_t* layer, const uint16_t* X, int M, void* Y, rb_dtype y_dtype,
                             void* workspace, size_t workspace_bytes, int32_t* dev_status, unsigned flags,
                             cudaStream_t stream, uint64_t timeout_ns, bool decode);
+// rb_pack's sign-plane kernel alone (no fp16 scale copies); arguments already checked
+rb_status pack_planes(const float* W, const float* g, const float* h, int N, int K, int kp, uint32_t* planes,
+                      int32_t* dev_status, cudaStream_t stream);
 size_t gemm_workspace(int k_in, int k_planes, int M);  // bytes of its workspace (X in fp16, h pairs)
 bool device_is_sm100();        // current device is compute capability 10.x
 

@@ -39,6 +39,8 @@ SIGNATURES = {
     "rb_shard_rows": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp]),
     "rb_planes_from_rowmajor": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "rb_planes_to_rowmajor": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
+    "rb_qat_forward_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
+    "rb_qat_forward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _u32, _vp]),
     "rb_qat_backward_workspace_bytes": (_sz, [_i32, _i32, _i32]),
     "rb_qat_backward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
     "rb_svid_workspace_bytes": (_sz, [_i32, _i32]),
@@ -250,6 +252,25 @@ def planes_to_rowmajor(layer: PackedLayer, out=None, stream=None):
                                      _stream(stream))
     _check("rb_planes_to_rowmajor", st)
     return out
+
+
+def qat_forward_workspace_bytes(n_out, k_in, k_planes, M):
+    return int(lib().rb_qat_forward_workspace_bytes(n_out, k_in, k_planes, M))
+
+
+def qat_forward(W, g, h, k_planes, X, Y=None, ws=None, flags=0, dev_status=None, stream=None,
+                y_dtype=torch.float32):
+    """rb_qat_forward: Y = X What^T, planes derived from fp32 W into the workspace, fp32 scales (CUDA tensors)."""
+    N, K = W.shape
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=y_dtype, device=W.device)
+    ws = ws if ws is not None else workspace(qat_forward_workspace_bytes(N, K, k_planes, M), W.device)
+    ydt = RB_BF16 if Y.dtype == torch.bfloat16 else RB_F32
+    st = lib().rb_qat_forward(_ptr(W), _ptr(g), _ptr(h), N, K, k_planes, _ptr(X), M, _ptr(Y), ydt, _ptr(ws),
+                              ws.numel(), _ptr(dev_status), flags, _stream(stream))
+    _check("rb_qat_forward", st)
+    return Y
 
 
 def qat_backward(layer: PackedLayer, g, h, X, dY, dW=None, dg=None, dh=None, ws=None, dev_status=None,

@@ -126,3 +126,86 @@ def test_qat_backward_is_deterministic_and_checks_args():
     with pytest.raises(rbw.RbError) as e:
         rbw.qat_backward(L2, gd[:, :100].contiguous(), hd, X, cases.to_dev(synth.activations(M, 100, seed=3)))
     assert e.value.status == rbw.RB_ERR_SHAPE
+
+
+@pytest.mark.parametrize("N,K,k,M", [(256, 512, 2, 100), (300, 800, 1, 64), (4096, 1024, 2, 2048), (128, 288, 2, 7),
+                                     (1000, 4096, 1, 1500), (4097, 544, 2, 300), (640, 1024, 3, 1100),
+                                     (256, 512, 4, 129), (160, 256, 8, 40)])
+def test_qat_forward_matches_oracle(N, K, k, M):
+    """rb_qat_forward (planes derived from fp32 W, then the tcgen05 GEMM with
+    the fp32 g) against the oracle's float64 training forward.
+    Gate from the arithmetic: the +-h operands are fp16(h) (relative error <=
+    2^-11) and the MMA accumulates exact products in fp32, so each element is
+    within (2^-11 + 1e-4) sum |g h x| (bf16 output: plus one bf16 step)."""
+    rng = np.random.default_rng(N + K + k + M)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[rng.random((N, K)) < 0.01] = 0.0
+    g, h = oracle.svid_greedy(W, k, iters=6)
+    X = synth.activations(M, K, seed=M + 3)
+    rows = np.unique(np.concatenate([np.arange(min(N, 40)), np.arange(max(0, N - 40), N),
+                                     rng.choice(N, min(N, 160), replace=False)]))
+    toks = np.unique(np.concatenate([np.arange(min(M, 16)), np.arange(max(0, M - 16), M),
+                                     rng.choice(M, min(M, 40), replace=False)]))
+    st, Yr = oracle.qat_forward(W, g, h, k, X, rows=rows, toks=toks)
+    assert st == 0
+    Xf = np.abs(bf16(X[toks]))
+    bound = Xf @ np.abs(h.astype(np.float64)).T @ np.abs(g.astype(np.float64)[:, rows])     # sum |g h x|
+    for ydt in (torch.float32, torch.bfloat16):
+        s = torch.zeros(4, dtype=torch.int32, device="cuda")
+        Y = rbw.qat_forward(cases.to_dev(W), cases.to_dev(g), cases.to_dev(h), k, cases.to_dev(X), dev_status=s,
+                            y_dtype=ydt)
+        torch.cuda.synchronize()
+        assert int(s[0].item()) == 0
+        Yg = Y.float().cpu().numpy().astype(np.float64)[np.ix_(toks, rows)]
+        cases.check_y(Yg, Yr, bound, bf16=ydt == torch.bfloat16, per_elem=2.0 ** -11 + 1e-4)
+
+
+def test_qat_forward_equals_deployment_gemm_on_fp16_exact_scales():
+    """With fp16-exact scales the training forward reaches the packed layer's
+    product bit for bit: rb_qat_forward(W, g, h) equals rb_gemm on rb_pack's
+    planes of the same W (the same MMA operands, the same accumulation), and
+    the planes it leaves in its workspace are rb_pack's."""
+    N, K, k, M = 512, 1024, 2, 256
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=6)
+    g = g.astype(np.float16).astype(np.float32)
+    h = h.astype(np.float16).astype(np.float32)
+    Wd, gd, hd = cases.to_dev(W), cases.to_dev(g), cases.to_dev(h)
+    X = cases.to_dev(synth.activations(M, K, seed=8))
+    wsf = rbw.workspace(rbw.qat_forward_workspace_bytes(N, K, k, M))
+    Yf = rbw.qat_forward(Wd, gd, hd, k, X, ws=wsf)
+    L = rbw.pack(Wd, gd, hd, k)
+    Yp = rbw.gemm(L, X, ws=rbw.workspace(rbw.gemm_workspace_bytes(N, K, k, M)))
+    torch.cuda.synchronize()
+    assert torch.equal(Yf, Yp)
+    nw = int(rbw.lib().rb_packed_words(N, K, k))
+    assert torch.equal(wsf.view(torch.int32)[:nw], L.planes.view(torch.int32)[:nw])
+
+
+def test_qat_forward_flags_and_limits():
+    """A NaN or infinite latent weight and a NaN h raise RB_DEV_NONFINITE (the
+    run still completes); k = 9 and a workspace one byte short are refused."""
+    N, K, k, M = 128, 256, 2, 64
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=4)
+    X = cases.to_dev(synth.activations(M, K, seed=4))
+    for bad in ("W_nan", "W_inf", "h_nan"):
+        Wb, hb = W.copy(), h.copy()
+        if bad == "W_nan":
+            Wb[77, 130] = np.nan
+        elif bad == "W_inf":
+            Wb[3, 255] = -np.inf
+        else:
+            hb[1, 31] = np.nan
+        s = torch.zeros(4, dtype=torch.int32, device="cuda")
+        rbw.qat_forward(cases.to_dev(Wb), cases.to_dev(g), cases.to_dev(hb), k, X, dev_status=s)
+        torch.cuda.synchronize()
+        assert int(s[0].item()) & rbw.RB_DEV_NONFINITE, bad
+    g9, h9 = np.concatenate([g] * 5)[:9], np.concatenate([h] * 5)[:9]
+    with pytest.raises(rbw.RbError):
+        rbw.qat_forward(cases.to_dev(W), cases.to_dev(g9), cases.to_dev(h9), 9, X)
+    short = rbw.workspace(rbw.qat_forward_workspace_bytes(N, K, k, M) - 16)
+    with pytest.raises(rbw.RbError):
+        rbw.qat_forward(cases.to_dev(W), cases.to_dev(g), cases.to_dev(h), k, X, ws=short)

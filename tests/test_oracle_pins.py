@@ -510,3 +510,36 @@ def test_qat_gradients_agree_with_the_deployment_oracle():
         Yi = oracle.apply(planes[i * per_plane:(i + 1) * per_plane], ones, h16[i:i + 1], N, K, 1, X)
         want = np.sum(bf16_to_f64(dY) * Yi, axis=0)
         assert np.allclose(dg[i], want, rtol=1e-12, atol=1e-15)
+
+
+def test_qat_forward_is_the_adjoint_of_the_pinned_backward_and_the_deployment_apply():
+    """The coupled-training forward (RaBiT, Algorithm 2 forward: signs derived
+    from W on the fly, fp32 scales) is pinned three ways:
+      * adjoint: <dY, Y(X)> = <dX, X> with dX from oracle.qat_backward, which is
+        itself pinned by exact central differences;
+      * with scales exactly representable in fp16 it equals oracle.apply of the
+        packed planes (the deployment path);
+      * rows and tokens selected by index give the same numbers as the full run.
+    A dropped sign, a swapped scale index or a transposed X fails one of them."""
+    rng = np.random.default_rng(41)
+    N, K, k, M = 40, 288, 3, 5
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[rng.random((N, K)) < 0.02] = 0.0
+    g, h = oracle.svid_greedy(W, k, iters=8)
+    X = synth.activations(M, K, seed=6)
+    dY = synth.activations(M, N, seed=7)
+    st, Y = oracle.qat_forward(W, g, h, k, X)
+    assert st == 0 and Y.shape == (M, N)
+    st, _, _, _, dX = oracle.qat_backward(W, g, h, k, X, dY)
+    lhs = float(np.sum(bf16_to_f64(dY) * Y))
+    rhs = float(np.sum(dX * bf16_to_f64(X)))
+    assert abs(lhs - rhs) <= 1e-12 * max(1.0, abs(lhs))
+    g16e = g.astype(np.float16).astype(np.float32)
+    h16e = h.astype(np.float16).astype(np.float32)
+    _, Ye = oracle.qat_forward(W, g16e, h16e, k, X)
+    planes, g16, h16, st2, _ = oracle.pack(W, g16e, h16e, k)
+    assert st2 == 0
+    assert np.allclose(Ye, oracle.apply(planes, g16, h16, N, K, k, X), rtol=1e-12, atol=1e-15)
+    rows, toks = np.array([0, 7, 39]), np.array([4, 1])
+    _, Ys = oracle.qat_forward(W, g, h, k, X, rows=rows, toks=toks)
+    assert np.array_equal(Ys, Y[np.ix_(toks, rows)])
