@@ -636,7 +636,7 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
     except Exception as e:                       # an informational row: record why it is missing
         out["gemv_M1_isolated"] = {"unavailable": repr(e)[:200]}
     # rb_gemv_batch at M = 4 and 16 (one tensor-core launch over the 96 layers), and
-    # rb_gemv at M = 64 with its workspace (tcgen05 kernel), 96 distinct layers
+    # rb_gemv at M = 64 (the path its size selects), 96 distinct layers
     for M in (4, 16):
         X = torch.from_numpy(synth.activations(M, K_IN, seed=M).view(np.int16)).to(dev)
         Ys = [torch.empty(M, N_OUT, dtype=torch.float32, device=dev) for _ in range(LAYERS)]
@@ -650,8 +650,9 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
     it64 = iter(range(10 ** 9))
     t = time_graph_calls(torch, lambda: rbw.gemv(layers[next(it64) % LAYERS], X, Y=Y, ws=ws, stream=stream),
                          2 * LAYERS, stream)
-    out["gemv_M64_tcgen05"] = {"us": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
-                               "TFLOPs": 2.0 * 64 * N_OUT * K_IN * K_PLANES / t / 1e12}
+    out["gemv_M64"] = {"us": t * 1e6, "packed_GBps": Lp.packed_bytes() / t / 1e9,
+                       "TFLOPs": 2.0 * 64 * N_OUT * K_IN * K_PLANES / t / 1e12,
+                       "path": "tcgen05" if rbw.gemv_workspace_bytes(N_OUT, K_IN, K_PLANES, 64) else "mma.sync"}
     # backward data path: rb_transpose_planes over the 96 layers (reads and writes the
     # planes once), then the input gradient dX = dY . What of one token per layer
     # through rb_gemv_batch on the transposed layers

@@ -168,9 +168,11 @@ RB_API rb_status rb_pack(const float *W, const float *g, const float *h,
  *   Calls that share a workspace must not overlap on the GPU.
  * M = 1 and k <= 4: byte tables; h_i .* x is formed exactly in fp32 and every
  * sum is accumulated in fp32 (CUDA cores, additions only).
- * M >= 32 and k <= 4 with the workspace: the tcgen05 kernel of rb_gemm with
- * 16/32/64-token tiles and K split over a thread-block cluster.
- * Otherwise (no workspace, or k > 4): mma.sync kernel.  Both tensor-core paths
+ * 32 <= M <= 64, k <= 4, N*K*k*M > 4.5e9, with the workspace: the tcgen05
+ * kernel of rb_gemm with 16/32/64-token tiles and K split over a thread-block
+ * cluster (the measured crossover: below it the mma.sync kernel is faster,
+ * and rb_gemv_workspace_bytes returns 0).
+ * Otherwise (no workspace, smaller layers, or k > 4): mma.sync kernel.  Both tensor-core paths
  * use fp16 operands with fp32 accumulation: the +-h_i operands are exact in
  * fp16 and X is converted to fp16 (exact for bf16 values of magnitude
  * 2^-14 .. 65504; smaller ones lose low bits; |x| >= 65520 overflows and

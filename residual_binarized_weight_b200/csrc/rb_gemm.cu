@@ -17,9 +17,11 @@
 // Epilogue: Y[m][n] = sum_i g_i[n] * D_i[n][m], one output row per TMEM lane,
 // so every store instruction writes 32 consecutive outputs.
 //
-// Warp roles (192 threads): warp 0 = TMA producer + TMEM allocator, warp 1 =
-// MMA issuer (one thread), warps 2..5 = sign expansion, then epilogue (warp w
-// owns TMEM lanes 32*(w%4) .. +31).  Every mbarrier wait is bounded: on expiry
+// Warp roles (64 + 32 EW threads): warp 0 = TMA producer + TMEM allocator,
+// warp 1 = MMA issuer (one thread), warps 2 .. 1 + EW = sign expansion, then
+// epilogue (warp w owns TMEM lanes 32*(w%4) .. +31; with EW = 8 two warps share
+// a lane quarter and take one 32-column word of each k-block, and every other
+// 32-token chunk of the epilogue).  Every mbarrier wait is bounded: on expiry
 // the kernel raises RB_DEV_TIMEOUT in dev_status, drains what it issued,
 // frees its tensor memory and returns.
 #include <atomic>
@@ -36,7 +38,7 @@ namespace {
 constexpr int kBR = 128;          // output rows per CTA (MMA M, TMEM lanes)
 constexpr int kBK = 64;           // K per pipeline stage (one 128-byte swizzle row of fp16)
 constexpr int kSX = 8;            // X stages (at most; fewer when h pairs of a long K need the room)
-constexpr int kThreads = 192;
+__host__ __device__ constexpr int gemm_threads(int ew) { return 64 + 32 * ew; }
 
 // Instruction descriptor, kind::f16: fp32 D, fp16 A and B, both K-major, N = bt, M = 128.
 __host__ __device__ constexpr uint32_t idesc_f16(int bt) {
@@ -126,8 +128,8 @@ __global__ void gemm_prepass_kernel(const uint16_t* __restrict__ X, const uint16
 // rank order.
 // g32 != nullptr (training forward): the epilogue scales row n of plane i by
 // the fp32 g32[i][n] instead of the stored fp16 g16.
-template <int KP, int BT, int SA>
-__global__ void __launch_bounds__(kThreads, (KP <= 2 && BT <= 64) ? 2 : 1)
+template <int KP, int BT, int SA, int EW>
+__global__ void __launch_bounds__(gemm_threads(EW), (KP <= 2 && BT <= 64) ? 2 : 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ planes,
                const uint16_t* __restrict__ g16, const uint32_t* __restrict__ hperm,
                int N, int K, int M, void* __restrict__ Y, int ydt, int32_t* dev_status, uint64_t timeout_ns,
@@ -168,7 +170,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSX; ++s) { mbar_init(full_x(s), 1); mbar_init(empty_x(s), 1); }
-        for (int s = 0; s < SA; ++s) { mbar_init(full_a(s), 128); mbar_init(empty_a(s), 1); }
+        for (int s = 0; s < SA; ++s) { mbar_init(full_a(s), 32 * EW); mbar_init(empty_a(s), 1); }
         mbar_init(acc_full, 1);
         mbar_init(hp_full, 1);
         *abort_flag = 0;
@@ -243,42 +245,47 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
         const int64_t tile = n >> 5;
         const bool tile_ok = tile < Nt;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        static_assert(EW == 4 || EW == 8, "four or eight expansion warps");
+        constexpr int NWW = EW == 8 ? 1 : 2;     // 32-column words of a k-block per thread
+        const int hh = EW == 8 ? (warp - 2) >> 2 : 0;   // with EW = 8: this warp's word of the k-block
         bool ok = true;
         if constexpr (!gemm_hp_in_smem(KP)) {
             // Sign words and +-h pairs of one k-block, fetched one k-block ahead from
             // global memory (L1/L2 hits: every row of the CTA reads the same h pairs).
-            auto load_kb = [&](int kb, uint32_t (&wv)[KP][2], uint32_t (&hp)[KP][32]) {
+            auto load_kb = [&](int kb, uint32_t (&wv)[KP][NWW], uint32_t (&hp)[KP][16 * NWW]) {
                 const int64_t sl = kb / 4;
                 const int w0 = (kb & 3) * 2;
 #pragma unroll
                 for (int i = 0; i < KP; ++i) {
 #pragma unroll
-                    for (int ww = 0; ww < 2; ++ww) {
+                    for (int w2 = 0; w2 < NWW; ++w2) {
+                        const int ww = NWW == 1 ? hh : w2;
                         const int64_t col0 = (int64_t)kb * kBK + ww * 32;
-                        wv[i][ww] = (tile_ok && col0 < K)
+                        wv[i][w2] = (tile_ok && col0 < K)
                             ? planes[block_index(i, sl, tile, S, Nt) * 256 + (((w0 + ww) ^ (lane >> 2)) * 32) + lane]
                             : 0u;
-                    }
-                    const int64_t hbase = (int64_t)i * (K / 2) + (int64_t)kb * 32;
+                        const int64_t hbase = (int64_t)i * (K / 2) + (int64_t)kb * 32 + ww * 16;
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        uint4 u = make_uint4(0, 0, 0, 0);
-                        if ((int64_t)kb * 32 + 4 * v < K / 2) u = *reinterpret_cast<const uint4*>(hperm + hbase + 4 * v);
-                        hp[i][4 * v] = u.x; hp[i][4 * v + 1] = u.y; hp[i][4 * v + 2] = u.z; hp[i][4 * v + 3] = u.w;
+                        for (int v = 0; v < 4; ++v) {
+                            uint4 u = make_uint4(0, 0, 0, 0);
+                            if (col0 < K) u = *reinterpret_cast<const uint4*>(hperm + hbase + 4 * v);
+                            hp[i][16 * w2 + 4 * v] = u.x; hp[i][16 * w2 + 4 * v + 1] = u.y;
+                            hp[i][16 * w2 + 4 * v + 2] = u.z; hp[i][16 * w2 + 4 * v + 3] = u.w;
+                        }
                     }
                 }
             };
-            uint32_t wv[KP][2], hp[KP][32];
+            uint32_t wv[KP][NWW], hp[KP][16 * NWW];
             load_kb(kb0, wv, hp);
             for (int kb = kb0; kb < kb1 && ok; ++kb) {
                 const int it = kb - kb0, sa = it % SA;
-                uint32_t cw[KP][2], ch[KP][32];
+                uint32_t cw[KP][NWW], ch[KP][16 * NWW];
 #pragma unroll
                 for (int i = 0; i < KP; ++i) {
-                    cw[i][0] = wv[i][0];
-                    cw[i][1] = wv[i][1];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) ch[i][j] = hp[i][j];
+                    for (int w2 = 0; w2 < NWW; ++w2) cw[i][w2] = wv[i][w2];
+#pragma unroll
+                    for (int j = 0; j < 16 * NWW; ++j) ch[i][j] = hp[i][j];
                 }
                 if (kb + 1 < kb1) load_kb(kb + 1, wv, hp);
                 if (it >= SA) {
@@ -290,13 +297,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
                 }
 #pragma unroll
                 for (int i = 0; i < KP; ++i) {
-                    uint32_t a[32];
+                    uint32_t a[16 * NWW];
 #pragma unroll
-                    for (int ww = 0; ww < 2; ++ww)
+                    for (int w2 = 0; w2 < NWW; ++w2)
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            a[ww * 16 + j] = lop3_sign(cw[i][ww] << (15 - j), ch[i][ww * 16 + j]);
-                    tc_st_32x32b_x32(tmem + lane_base + (uint32_t)(KP * BT + (sa * KP + i) * 32), a);
+                            a[w2 * 16 + j] = lop3_sign(cw[i][w2] << (15 - j), ch[i][w2 * 16 + j]);
+                    const uint32_t col = (uint32_t)(KP * BT + (sa * KP + i) * 32);
+                    if constexpr (NWW == 2) tc_st_32x32b_x32(tmem + lane_base + col, a);
+                    else tc_st_32x32b_x16(tmem + lane_base + col + (uint32_t)(hh * 16), a);
                 }
                 tc_wait_st();
                 tc_fence_before();
@@ -333,21 +342,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
                     }
     #pragma unroll
                     for (int i = 0; i < KP; ++i) {
-                        uint32_t hp[32];
-                        const uint32_t* hrow = hsm + (size_t)i * (K / 2) + (size_t)kb * 32;
+                        uint32_t hp[16 * NWW];
+                        uint32_t a[16 * NWW];
     #pragma unroll
-                        for (int v = 0; v < 8; ++v) {
-                            uint4 u = make_uint4(0, 0, 0, 0);
-                            if (kb * 32 + 4 * v < K / 2) u = *reinterpret_cast<const uint4*>(hrow + 4 * v);
-                            hp[4 * v] = u.x; hp[4 * v + 1] = u.y; hp[4 * v + 2] = u.z; hp[4 * v + 3] = u.w;
-                        }
-                        uint32_t a[32];
+                        for (int w2 = 0; w2 < NWW; ++w2) {
+                            const int ww = NWW == 1 ? hh : w2;
+                            const uint32_t* hrow = hsm + (size_t)i * (K / 2) + (size_t)kb * 32 + ww * 16;
     #pragma unroll
-                        for (int ww = 0; ww < 2; ++ww)
+                            for (int v = 0; v < 4; ++v) {
+                                uint4 u = make_uint4(0, 0, 0, 0);
+                                if (kb * 64 + ww * 32 < K) u = *reinterpret_cast<const uint4*>(hrow + 4 * v);
+                                hp[16 * w2 + 4 * v] = u.x; hp[16 * w2 + 4 * v + 1] = u.y;
+                                hp[16 * w2 + 4 * v + 2] = u.z; hp[16 * w2 + 4 * v + 3] = u.w;
+                            }
     #pragma unroll
                             for (int j = 0; j < 16; ++j)
-                                a[ww * 16 + j] = lop3_sign(cur[i][2 * qk + ww] << (15 - j), hp[ww * 16 + j]);
-                        tc_st_32x32b_x32(tmem + lane_base + (uint32_t)(KP * BT + (sa * KP + i) * 32), a);
+                                a[w2 * 16 + j] = lop3_sign(cur[i][2 * qk + ww] << (15 - j), hp[w2 * 16 + j]);
+                        }
+                        const uint32_t col = (uint32_t)(KP * BT + (sa * KP + i) * 32);
+                        if constexpr (NWW == 2) tc_st_32x32b_x32(tmem + lane_base + col, a);
+                        else tc_st_32x32b_x16(tmem + lane_base + col + (uint32_t)(hh * 16), a);
                     }
                     tc_wait_st();
                     tc_fence_before();
@@ -370,7 +384,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
             constexpr int CW = BT < 32 ? BT : 32;            // tokens per TMEM load
             constexpr int PB = KP <= 4 ? KP : 2;             // planes per batch of TMEM loads (registers)
 #pragma unroll 1
-            for (int c = 0; c < BT / CW; ++c) {
+            for (int c = NWW == 1 ? hh : 0; c < BT / CW; c += 3 - NWW) {
                 float y[CW];
 #pragma unroll
                 for (int j = 0; j < CW; ++j) y[j] = 0.0f;
@@ -417,7 +431,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __res
         cluster_sync_all();
         const int rpo = (kBR + ks - 1) / ks;
         const int row0 = (kBR * rank + ks - 1) / ks, nrow = (kBR * (rank + 1) + ks - 1) / ks - row0;
-        for (int idx = threadIdx.x; idx < nrow * BT; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < nrow * BT; idx += (int)blockDim.x) {
             const int tok = idx / nrow, lr = idx - tok * nrow;
             float v = 0.0f;
             for (int j = 0; j < ks; ++j) v += recv[(j * rpo + lr) * BT + tok];
@@ -477,7 +491,7 @@ GemmWs gemm_ws_layout(int K, int kp, int M, void* base)
 
 // ks > 1: K split over clusters of (1, 1, ks); every rank gets a whole number
 // of 256-column slices and at least one k-block.
-template <int KP, int BT, int SA>
+template <int KP, int BT, int SA, int EW = 4>
 rb_status launch_gemm(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs& ws,
                       int32_t* dev_status, bool pdl, cudaStream_t stream, uint64_t timeout_ns, int ks,
                       const float* g32 = nullptr, bool dry = false)
@@ -512,16 +526,16 @@ rb_status launch_gemm(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs
     const int smem = gemm_smem_bytes(KP, BT, L->k_in, nsx, ks);
     if (smem > kMaxSmem) return RB_ERR_UNSUPPORTED;          // K too long for the h pairs in shared memory
     if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(gemm_tc_kernel<KP, BT, SA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemm_tc_kernel<KP, BT, SA, EW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxSmem) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_tc_kernel<KP, BT, SA>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaFuncSetAttribute(gemm_tc_kernel<KP, BT, SA, EW>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                 cudaSuccess)
             return RB_ERR_CUDA;
         attr_set[dev].store(true, std::memory_order_release);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((L->n_out + kBR - 1) / kBR), (unsigned)((M + BT - 1) / BT), (unsigned)ks);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(gemm_threads(EW));
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -540,7 +554,7 @@ rb_status launch_gemm(const rb_layer_t* L, int M, void* Y, int ydt, const GemmWs
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<KP, BT, SA>, map, L->planes, L->g16, (const uint32_t*)ws.hperm,
+    if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<KP, BT, SA, EW>, map, L->planes, L->g16, (const uint32_t*)ws.hperm,
                            (int)L->n_out, (int)L->k_in, M, Y, ydt, dev_status, timeout_ns, nsx, kb_per, g32) !=
         cudaSuccess)
         return RB_ERR_CUDA;
@@ -563,6 +577,11 @@ rb_status launch_gemm_decode(const rb_layer_t* L, int M, void* Y, int ydt, const
     return launch_gemm<KP, 64, 2>(L, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, ks);
 }
 
+// Expansion warps of the prefill tiles: eight for k = 4 (its expansion is the
+// longest; 614 against 549 TFLOP/s at M = 2048 on 4096 x 4096), four below
+// (eight measured within +-3 % for k <= 2 and 5 % slower for k = 3).
+template <int KP> constexpr int kPrefillEW = KP == 4 ? 8 : 4;
+
 // Tile shape per k and M for the prefill kernel (the prepass has run).
 rb_status gemm_dispatch(const rb_layer_t* layer, int M, void* Y, int ydt, const GemmWs& ws, int32_t* dev_status,
                         cudaStream_t stream, uint64_t timeout_ns, const float* g32, bool dry = false)
@@ -573,15 +592,15 @@ rb_status gemm_dispatch(const rb_layer_t* layer, int M, void* Y, int ydt, const 
     // M fills them; narrower below that, where a wide last tile pads more.
     switch (layer->k_planes) {
         case 1:
-            if (M >= 1024) return launch_gemm<1, 256, 4>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
-            return launch_gemm<1, gemm_bt(1), gemm_sa(1)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
+            if (M >= 1024) return launch_gemm<1, 256, 4, kPrefillEW<1>>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
+            return launch_gemm<1, gemm_bt(1), gemm_sa(1), kPrefillEW<1>>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
         case 2:
-            if (M >= 1536) return launch_gemm<2, 192, 2>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
-            return launch_gemm<2, gemm_bt(2), gemm_sa(2)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
+            if (M >= 1536) return launch_gemm<2, 192, 2, kPrefillEW<2>>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
+            return launch_gemm<2, gemm_bt(2), gemm_sa(2), kPrefillEW<2>>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
         case 3:
-            if (M >= 1024) return launch_gemm<3, 96, 2>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
-            return launch_gemm<3, gemm_bt(3), gemm_sa(3)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
-        case 4: return launch_gemm<4, gemm_bt(4), gemm_sa(4)>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
+            if (M >= 1024) return launch_gemm<3, 96, 2, kPrefillEW<3>>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
+            return launch_gemm<3, gemm_bt(3), gemm_sa(3), kPrefillEW<3>>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
+        case 4: return launch_gemm<4, gemm_bt(4), gemm_sa(4), kPrefillEW<4>>(layer, M, Y, ydt, ws, dev_status, true, stream, timeout_ns, 1, g32, dry);
         // k = 5..8: the accumulators (k x BT columns) and the A stages (SA x k x 32)
         // share the 512 tensor-memory columns, so the tiles narrow and the
         // pipeline shortens as k grows.

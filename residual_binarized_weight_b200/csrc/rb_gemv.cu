@@ -39,7 +39,6 @@ template <int KP> struct LutCfg {
     static constexpr int min_blocks = KP >= 3 ? 1 : 2;
 };
 constexpr int kLutPF = 2;              // row tiles per warp held in registers ahead of use
-constexpr int kLutPD = 6;              // row tiles per warp prefetched into L2 ahead of use
 
 __host__ __device__ constexpr int lut_table_bytes(int kp) { return ((kp + 1) / 2) * 65536; }
 
@@ -52,19 +51,6 @@ __device__ __forceinline__ void lut_load_tile(uint32_t (&wd)[KP][8], const uint3
         const uint32_t* blk = planes + block_index(i, s, t, S, Nt) * 256 + lane;
 #pragma unroll
         for (int sl = 0; sl < 8; ++sl) wd[i][sl] = __ldcs(blk + sl * 32);
-    }
-}
-
-// L2 prefetch of one row tile's sign words (KP blocks of 1 KB = 8 lines each):
-// lane l < 8*KP touches line l%8 of plane l/8.  Keeps DRAM busy further ahead
-// than the register-held tiles can.
-template <int KP>
-__device__ __forceinline__ void lut_prefetch_tile(const uint32_t* __restrict__ planes, int64_t s, int64_t t,
-                                                  int64_t S, int64_t Nt, int lane)
-{
-    if (lane < 8 * KP) {
-        const uint32_t* p = planes + block_index(lane >> 3, s, t, S, Nt) * 256 + (lane & 7) * 32;
-        asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
     }
 }
 
@@ -204,9 +190,9 @@ __device__ __forceinline__ void lut_lookups(float (&acc)[kLutPF][KP][2], const u
 // with the tile kLutPF further on, clamped to the warp's last tile when that
 // runs past the end (the slot is then not used), and after the last group with
 // tile j = slot of the CTA's next slice, so a slice starts on loaded registers.
-// L2 prefetches run kLutPD tiles ahead in the same sequence, on into the next
-// slice.  Tile validity only gates the red[] update, so no load is guarded by
-// a branch.
+// Tile validity only gates the red[] update, so no load is guarded by a branch.
+// (Software L2 prefetches further ahead, per line or as bulk copies of whole
+// tiles, measured 1-10 % slower: the loads two tiles ahead already keep up.)
 template <int KP>
 __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_t (&gv)[kLutPF][KP],
                                           const uint32_t (&G)[8], const uint32_t (&SEL)[4], uint32_t tbase,
@@ -224,11 +210,6 @@ __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_
         cur[i] = planes + block_index(i, s, 0, S, Nt) * 256 + lane;
         nxt[i] = has_next ? planes + block_index(i, s_next, 0, S, Nt) * 256 + lane : cur[i];
     }
-    // this lane's L2-prefetch line: plane lane/8, line lane%8 of a tile block
-    const bool pf_lane = lane < 8 * KP;
-    const uint32_t* pf_cur = planes + block_index(pf_lane ? lane >> 3 : 0, s, 0, S, Nt) * 256 + (lane & 7) * 32;
-    const uint32_t* pf_nxt = has_next
-        ? planes + block_index(pf_lane ? lane >> 3 : 0, s_next, 0, S, Nt) * 256 + (lane & 7) * 32 : pf_cur;
     const int t_w = tb + warp;                    // the warp's first tile
     for (int it = 0; it < iters; ++it) {
         float acc[kLutPF][KP][2];
@@ -246,13 +227,6 @@ __device__ __forceinline__ void lut_tiles(uint32_t (&wd)[kLutPF][KP][8], uint16_
             for (int i = 0; i < KP; ++i)
                 pr += __half2float(__ushort_as_half(gv[p][i])) * (acc[p][i][0] + acc[p][i][1]);
             if (j < nw) red[(j * LutCfg<KP>::warps + warp) * 32 + lane] += pr;
-            const int jp = j + kLutPD;
-            const bool pf_here = jp < nw;
-            if (pf_lane && (pf_here || (has_next && jp - nw < nw))) {
-                const uint32_t* q = pf_here ? pf_cur + (size_t)(t_w + jp * LutCfg<KP>::warps) * 256
-                                            : pf_nxt + (size_t)(t_w + (jp - nw) * LutCfg<KP>::warps) * 256;
-                asm volatile("prefetch.global.L2 [%0];" :: "l"(q));
-            }
             if (!last || (has_next && p < nw)) {
                 const int jn = last ? p : min(j + kLutPF, nw - 1);
                 const size_t tn = (size_t)(t_w + jn * LutCfg<KP>::warps);
@@ -326,14 +300,7 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
             }
         }
     }
-    if (s_first < S) {
-        lut_load_h<KP>(hr, h16, s_first, K);
-#pragma unroll
-        for (int p = kLutPF; p < kLutPD; ++p) {
-            const int64_t t = t_begin + warp + (int64_t)p * LutCfg<KP>::warps;
-            if (t < t_end) lut_prefetch_tile<KP>(planes, s_first, t, S, Nt, lane);
-        }
-    }
+    if (s_first < S) lut_load_h<KP>(hr, h16, s_first, K);
     for (int64_t x = threadIdx.x; x < chunk_rows; x += LutCfg<KP>::threads) red[x] = 0.0f;
 
     // Per-lane lookup constants: G[sl] byte b' = group offset ((4 sl + b') ^ lane) * 4;
@@ -751,8 +718,8 @@ int lut_resident(int CS, int smem)
 constexpr int kLutBuildTiles = 8;
 
 // Single layer (count == 1): lowest latency.  Slices per CTA = ceil(S/16),
-// CS = ceil(S / that) CTAs per cluster, as many row chunks (R) as the GPU keeps
-// clusters resident, one wave.
+// CS = ceil(S / that) CTAs per cluster, one row chunk (R) fewer than the GPU
+// keeps clusters resident, one wave.
 // Batch: CS (a power of two) and R minimise the modelled time waves * (time of
 // one CTA), where a CTA builds ceil(S/CS) tables and runs ceil(rows/R) row
 // tiles through each, and the count * R clusters run in ceil(count * R /
@@ -777,7 +744,12 @@ rb_status lut_plan_uncached(int N, int K, int count, LutPlan* plan)
         while (R < Nt && lut_table_bytes(KP) + lut_row_bytes(Nt, R, CS) > cap) ++R;
         LutPlan p{CS, R, lut_table_bytes(KP) + lut_row_bytes(Nt, R, CS)};
         if (CS > 1) {
-            const int active = lut_resident<KP>(CS, p.smem);
+            // one cluster fewer than the GPU keeps resident, which leaves SMs free for
+            // the first CTAs of the next layer's launch (PDL): 8 clusters of 16
+            // against 9 measured 4.37 against 4.60 us per layer in a dependent
+            // chain of 4096 x 4096 layers (7 and 6: 4.57 and 5.8 us)
+            int active = lut_resident<KP>(CS, p.smem);
+            if (active > 1) --active;
             if (active > 0 && active < R) {
                 p.R = active;
                 p.smem = lut_table_bytes(KP) + lut_row_bytes(Nt, p.R, CS);
@@ -972,13 +944,26 @@ bool use_lut(const rb_layer_t* L, int M) { return M == 1 && L->k_planes <= 4; }
 
 using namespace rbw;
 
-// From this many tokens (and k <= 4) rb_gemv runs on the tcgen05 kernel when
-// the caller passes the workspace it needs (X in fp16 and the h pairs).
+// rb_gemv runs on the tcgen05 kernel (K split over a cluster) when the caller
+// passes its workspace and the layer is large enough for it: 32 <= M <= 64,
+// k <= 4 and N*K*k*M above 4.5e9 multiply-adds.  Measured single-layer times
+// (back-to-back launches over layers that do not fit in L2), tcgen05 against
+// mma.sync: 4096 x 4096 k = 2, M = 64: 43.4 against 38.4 us; 14336 x 4096
+// k = 2, M = 64: 64.9 against 86.9 us; 28672 x 8192 k = 2, M = 32: 139
+// against 153 us; 11008 x 4096 k = 2, M = 48 (4.3e9): 61.3 against 51.9 us.
 constexpr int kTcMinM = 32;
+constexpr double kTcMinWork = 4.5e9;
+
+static bool use_tc_decode(int n_out, int k_in, int k_planes, int M)
+{
+    return M >= kTcMinM && M <= 64 && k_planes <= 4 &&
+           (double)n_out * (double)k_in * (double)k_planes * (double)M > kTcMinWork;
+}
 
 extern "C" size_t rb_gemv_workspace_bytes(int n_out, int k_in, int k_planes, int M)
 {
-    if (n_out < 1 || k_in < 32 || k_in % 32 != 0 || M < kTcMinM || M > 64 || k_planes < 1 || k_planes > 4) return 0;
+    if (n_out < 1 || k_in < 32 || k_in % 32 != 0 || k_planes < 1 || k_planes > 4) return 0;
+    if (!use_tc_decode(n_out, k_in, k_planes, M)) return 0;
     return gemm_workspace(k_in, k_planes, M);
 }
 
@@ -1023,7 +1008,7 @@ extern "C" rb_status rb_gemv(const rb_layer_t* layer, const uint16_t* X, int M, 
                              int32_t* dev_status, unsigned flags, cudaStream_t stream)
 {
     if (!layer) return RB_ERR_ARG;
-    if (M >= kTcMinM && M <= 64 && layer->k_planes <= 4 && workspace != nullptr &&
+    if (use_tc_decode(layer->n_out, layer->k_in, layer->k_planes, M) && workspace != nullptr &&
         workspace_bytes >= rb_gemv_workspace_bytes(layer->n_out, layer->k_in, layer->k_planes, M))
         return gemm_with_timeout(layer, X, M, Y, y_dtype, workspace, workspace_bytes, dev_status, flags, stream,
                                  kWaitTimeoutNs, true);

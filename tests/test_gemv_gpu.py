@@ -213,20 +213,22 @@ def test_gemv_batch_multi_token(N, K, k, M, count):
                       per_elem=per_elem(M, k))
 
 
-@pytest.mark.parametrize("N,K,k,M", [(4096, 4096, 2, 32), (1000, 2048, 1, 48), (300, 4096, 4, 33), (4096, 11008, 2, 64),
-                                     (70, 1056, 2, 40)])
+@pytest.mark.parametrize("N,K,k,M", [(4096, 11008, 2, 64), (14336, 4096, 2, 48), (8192, 4096, 4, 40),
+                                     (20000, 5152, 2, 40), (28672, 8192, 1, 32)])
 def test_gemv_both_tensor_core_paths(N, K, k, M):
-    """For M >= 32 rb_gemv runs the tcgen05 kernel when given its workspace
-    (K split over clusters of any size up to 16) and the mma.sync kernel
-    without one; both match the oracle."""
+    """Above the measured crossover (N*K*k*M > 4.5e9, 32 <= M <= 64, k <= 4)
+    rb_gemv runs the tcgen05 kernel when given its workspace (K split over a
+    cluster; ragged N and K included) and the mma.sync kernel without one;
+    both match the oracle on sampled rows."""
     rng = np.random.default_rng(N + K + M)
     W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
-    g, h = oracle.svid_greedy(W, k, iters=6)
+    g, h = oracle.svid_greedy(W, k, iters=4)
     planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
     L = cases.upload_layer(planes, g16, h16, N, K, k)
     X = synth.activations(M, K, seed=M + 5)
-    Yr = oracle.apply(planes, g16, h16, N, K, k, X)
-    bound = cases.abs_bound(g16, h16, X)
+    rows = np.unique(np.concatenate([np.arange(40), np.arange(N - 40, N), rng.choice(N, 200, replace=False)]))
+    Yr = oracle.apply(planes, g16, h16, N, K, k, X, rows=rows)
+    bound = cases.abs_bound(g16, h16, X, rows=rows)
     assert rbw.gemv_workspace_bytes(N, K, k, M) > 0
     Xd = cases.to_dev(X)
     for ws in (rbw.workspace(rbw.gemv_workspace_bytes(N, K, k, M)), None):
@@ -234,7 +236,24 @@ def test_gemv_both_tensor_core_paths(N, K, k, M):
         Y = rbw.gemv(L, Xd, ws=ws, dev_status=st)
         torch.cuda.synchronize()
         assert int(st[0].item()) == 0
-        cases.check_y(Y.cpu().numpy().astype(np.float64), Yr, bound, bf16=False, per_elem=per_elem(M, k))
+        cases.check_y(Y.cpu().numpy().astype(np.float64)[:, rows], Yr, bound, bf16=False, per_elem=per_elem(M, k))
+
+
+@pytest.mark.parametrize("N,K,k,M", [(4096, 4096, 2, 64), (300, 4096, 4, 33), (70, 1056, 2, 40), (4096, 4096, 1, 48)])
+def test_gemv_small_layers_need_no_workspace(N, K, k, M):
+    """Below the crossover the mma.sync kernel is the faster one: no workspace
+    is asked for, and one passed anyway changes nothing."""
+    assert rbw.gemv_workspace_bytes(N, K, k, M) == 0
+    rng = np.random.default_rng(N + K + M)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    g, h = oracle.svid_greedy(W, k, iters=4)
+    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    Xd = cases.to_dev(synth.activations(M, K, seed=M + 5))
+    Ya = rbw.gemv(L, Xd)
+    Yb = rbw.gemv(L, Xd, ws=rbw.workspace(1 << 20))
+    torch.cuda.synchronize()
+    assert torch.equal(Ya, Yb)
 
 
 def test_gemv_batch_rejects_mixed_shapes():
@@ -252,14 +271,14 @@ def test_activation_overflow_is_reported_on_tensor_core_paths():
     RB_DEV_RANGE on the mma.sync path (rb_gemv and rb_gemv_batch at M >= 2) and
     on the tcgen05 path; the byte-table path (M = 1) forms h*x in fp32 and
     raises nothing."""
-    N, K, k = 256, 512, 2
-    rng = np.random.default_rng(3)
-    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
-    g, h = oracle.svid_greedy(W, k, iters=6)
-    planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
-    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    k = 2
     big = np.uint16(0x4789)                        # bf16 70144: finite, above fp16's range
-    for M, ws in ((1, None), (4, None), (40, None), (40, "ws")):
+    for M, ws, N, K in ((1, None, 256, 512), (4, None, 256, 512), (40, None, 256, 512), (48, "ws", 14336, 4096)):
+        rng = np.random.default_rng(3)
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+        g, h = oracle.svid_greedy(W, k, iters=2)
+        planes, g16, h16, _, _ = oracle.pack(W, g, h, k)
+        L = cases.upload_layer(planes, g16, h16, N, K, k)
         X = synth.activations(M, K, seed=M)
         X[M - 1, 100] = big
         Xd = cases.to_dev(X)
