@@ -67,6 +67,18 @@ def _load():
         lib.oracle_svid_iterative.restype = i32
         lib.oracle_plane_words.argtypes = [i64, i64, i32]
         lib.oracle_plane_words.restype = i64
+        lib.oracle_btc_index_bits.argtypes = [i32]
+        lib.oracle_btc_index_bits.restype = i32
+        lib.oracle_btc_row_words.argtypes = [i64, i32]
+        lib.oracle_btc_row_words.restype = i64
+        lib.oracle_btc_patterns.argtypes = [vp, i64, i64, i32, i32, vp]
+        lib.oracle_btc_patterns.restype = None
+        lib.oracle_btc_encode.argtypes = [vp, i64, i64, i32, i32, i32, i32, vp, vp, vp, vp]
+        lib.oracle_btc_encode.restype = i32
+        lib.oracle_btc_pack_indices.argtypes = [vp, i64, i64, i32, vp]
+        lib.oracle_btc_pack_indices.restype = None
+        lib.oracle_btc_apply.argtypes = [vp, i32, vp, vp, vp, i64, i64, i32, vp, i64, vp, i64, vp]
+        lib.oracle_btc_apply.restype = None
         lib.oracle_f64_to_f16.argtypes = [dbl]
         lib.oracle_f64_to_f16.restype = ctypes.c_uint16
         lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
@@ -273,3 +285,54 @@ def f64_array_to_bf16_bits(a) -> np.ndarray:
     lib = _load()
     out = np.fromiter((lib.oracle_f64_to_bf16(float(x)) for x in a.ravel()), np.uint16, a.size)
     return out.reshape(a.shape)
+
+
+# ---------------------------------------------------------------- binary codebook (BTC-LLM)
+def btc_index_bits(c_max: int) -> int:
+    """Bits per stored index: ceil(log2 c_max), at least 1."""
+    return int(_load().oracle_btc_index_bits(c_max))
+
+
+def btc_row_words(K: int, w: int) -> int:
+    return int(_load().oracle_btc_row_words(K, w))
+
+
+def btc_patterns(planes, N: int, K: int, k: int, i: int):
+    """uint16 [N][K/16]: the 16-column sign patterns of plane i (bit q = column 16j+q is +1)."""
+    pat = np.zeros((N, K // 16), np.uint16)
+    _load().oracle_btc_patterns(_p(_c(planes, np.uint32)), N, K, k, i, _p(pat))
+    return pat
+
+
+def btc_encode(planes, N: int, K: int, k: int, i: int, c_max: int, iters: int):
+    """Binary k-means codebook of plane i: (codebook uint16 [c_max], c, idx uint16 [N][K/16],
+    objective float64 [iters + 1])."""
+    cb = np.zeros(c_max, np.uint16)
+    idx = np.zeros((N, K // 16), np.uint16)
+    obj = np.zeros(iters + 1, np.float64)
+    c = ctypes.c_int(0)
+    st = _load().oracle_btc_encode(_p(_c(planes, np.uint32)), N, K, k, i, c_max, iters, _p(cb),
+                                   ctypes.byref(c), _p(idx), _p(obj))
+    if st != 0:
+        raise ValueError("oracle_btc_encode: bad arguments")
+    return cb, int(c.value), idx, obj
+
+
+def btc_pack_indices(idx, N: int, K: int, w: int):
+    """uint32 [N][row_words]: index j of row r at bits [j w, j w + w) of the row's stream."""
+    words = np.zeros((N, btc_row_words(K, w)), np.uint32)
+    _load().oracle_btc_pack_indices(_p(_c(idx, np.uint16)), N, K, w, _p(words))
+    return words
+
+
+def btc_apply(codebooks, c_max: int, idx, g16, h16, N: int, K: int, k: int, X_bf16, rows=None):
+    """float64 Y [M][len(rows)] of the codebook-reconstructed layer; codebooks [k][c_max],
+    idx [k][N][K/16] plain indices."""
+    X = _c(X_bf16, np.uint16)
+    M = X.shape[0]
+    rows_a = None if rows is None else _c(rows, np.int64)
+    nr = N if rows_a is None else len(rows_a)
+    Y = np.zeros((M, nr), np.float64)
+    _load().oracle_btc_apply(_p(_c(codebooks, np.uint16)), c_max, _p(_c(idx, np.uint16)), _p(_c(g16, np.uint16)),
+                             _p(_c(h16, np.uint16)), N, K, k, _p(X), M, _p(rows_a), nr, _p(Y))
+    return Y

@@ -646,3 +646,181 @@ int oracle_svid_iterative(const float *W, int64_t N, int64_t K, int k, int sweep
     free(v);
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Binary codebook and its LUT application (BTC-LLM: "Binary codebook",  */
+/* 2.1.1 binary k-means and dynamic codebook size; 2.1.2 LUT-GEMM;       */
+/* 3.2.1 index of ceil(log2 c) bits; 5.1 v = 16, c = 7132 for 7B)          */
+/* ------------------------------------------------------------------ */
+
+/* Readings (listed in the design notes):
+ *   - the vectors clustered are the v = 16 column groups of one sign plane
+ *     B_i; pattern bit q = 1 <=> B_i[r][16 j + q] = +1 (the planes' own bit
+ *     order);
+ *   - the codebook size is c = min(c_max, number of distinct patterns)
+ *     (dynamic size); the c initial centroids are the c most frequent
+ *     patterns, ties to the smaller pattern value, in that order;
+ *   - one round = assignment of every vector to the centroid at the least
+ *     Hamming distance popcount(u ^ C[p]) (ties to the smaller p), then each
+ *     centroid that has members becomes the per-bit majority of its members,
+ *     sign(0) = +1 (a member-less centroid is kept); `iters` rounds, then a
+ *     final assignment gives the indices;
+ *   - index j of row r (the j-th 16-column group) is stored in w = ceil(log2
+ *     c_max) bits (at least 1), LSB-first in a per-row bit stream of
+ *     ceil(K/16 * w / 32) words: bits [j w, j w + w) of the row's stream.   */
+
+static int popcount16(uint32_t x)
+{
+    int n = 0;
+    for (int b = 0; b < 16; ++b) n += (x >> b) & 1u;
+    return n;
+}
+
+int oracle_btc_index_bits(int c_max)
+{
+    int w = 1;
+    while ((1 << w) < c_max) ++w;
+    return w;
+}
+
+int64_t oracle_btc_row_words(int64_t K, int w) { return (K / 16 * w + 31) / 32; }
+
+/* 16-bit patterns [N][K/16] of plane i from the storage layout. */
+void oracle_btc_patterns(const uint32_t *planes, int64_t N, int64_t K, int k, int i, uint16_t *pat)
+{
+    int64_t J = K / 16;
+    for (int64_t r = 0; r < N; ++r)
+        for (int64_t j = 0; j < J; ++j) {
+            uint32_t word = planes[word_index(N, K, i, r, 16 * j)];
+            pat[r * J + j] = (uint16_t)((word >> ((16 * j) % 32)) & 0xFFFFu);
+        }
+    (void)k;
+}
+
+/* Binary k-means over the patterns of plane i.  codebook gets c_max entries
+ * (those past *c_out are 0), idx [N][K/16] the final assignment; objective
+ * (nullable) iters + 1 values: sum over all vectors of the Hamming distance
+ * to the assigned centroid after each assignment step.  Returns 0, or -1 for
+ * bad arguments. */
+int oracle_btc_encode(const uint32_t *planes, int64_t N, int64_t K, int k, int i, int c_max, int iters,
+                      uint16_t *codebook, int *c_out, uint16_t *idx, double *objective)
+{
+    if (N < 1 || K < 32 || K % 32 != 0 || k < 1 || k > 8 || i < 0 || i >= k || c_max < 1 || c_max > 65536 ||
+        iters < 0)
+        return -1;
+    int64_t J = K / 16, nv = N * J;
+    uint16_t *pat = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)nv);
+    uint64_t *hist = (uint64_t *)calloc(65536, sizeof(uint64_t));
+    int32_t *assign = (int32_t *)malloc(sizeof(int32_t) * 65536);
+    oracle_btc_patterns(planes, N, K, k, i, pat);
+    for (int64_t x = 0; x < nv; ++x) hist[pat[x]]++;
+    int U = 0;
+    for (int u = 0; u < 65536; ++u) U += hist[u] > 0;
+    int c = U < c_max ? U : c_max;
+    /* initial centroids: the c most frequent patterns (count descending, then
+     * pattern ascending), by repeated selection of the best remaining one */
+    unsigned char *taken = (unsigned char *)calloc(65536, 1);
+    for (int p = 0; p < c_max; ++p) codebook[p] = 0;
+    for (int p = 0; p < c; ++p) {
+        int best = -1;
+        for (int u = 0; u < 65536; ++u) {
+            if (taken[u] || hist[u] == 0) continue;
+            if (best < 0 || hist[u] > hist[best]) best = u;
+        }
+        taken[best] = 1;
+        codebook[p] = (uint16_t)best;
+    }
+    free(taken);
+    for (int round = 0; round <= iters; ++round) {
+        double obj = 0.0;
+        #pragma omp parallel for schedule(dynamic, 256) reduction(+ : obj)
+        for (int u = 0; u < 65536; ++u) {
+            if (hist[u] == 0) { assign[u] = -1; continue; }
+            int bp = 0, bd = 17;
+            for (int p = 0; p < c; ++p) {
+                int d = popcount16((uint32_t)u ^ codebook[p]);
+                if (d < bd) { bd = d; bp = p; }
+            }
+            assign[u] = bp;
+            obj += (double)hist[u] * bd;
+        }
+        if (objective) objective[round] = obj;
+        if (round == iters) break;
+        /* majority of the members, bit by bit: +1 when the +1 count is at least the -1 count */
+        int64_t *sum = (int64_t *)calloc((size_t)c * 16, sizeof(int64_t));
+        uint64_t *members = (uint64_t *)calloc((size_t)c, sizeof(uint64_t));
+        for (int u = 0; u < 65536; ++u) {
+            if (hist[u] == 0) continue;
+            int p = assign[u];
+            members[p] += hist[u];
+            for (int q = 0; q < 16; ++q) sum[(int64_t)p * 16 + q] += ((u >> q) & 1) ? (int64_t)hist[u] : -(int64_t)hist[u];
+        }
+        for (int p = 0; p < c; ++p) {
+            if (members[p] == 0) continue;
+            uint32_t cw = 0;
+            for (int q = 0; q < 16; ++q) cw |= (sum[(int64_t)p * 16 + q] >= 0 ? 1u : 0u) << q;
+            codebook[p] = (uint16_t)cw;
+        }
+        free(sum);
+        free(members);
+    }
+    for (int64_t x = 0; x < nv; ++x) idx[x] = (uint16_t)assign[pat[x]];
+    *c_out = c;
+    free(pat);
+    free(hist);
+    free(assign);
+    return 0;
+}
+
+/* Index bit stream of one plane: [N][row_words], index j of row r at bits
+ * [j w, j w + w) of the row's words, LSB-first; unused bits zero. */
+void oracle_btc_pack_indices(const uint16_t *idx, int64_t N, int64_t K, int w, uint32_t *words)
+{
+    int64_t J = K / 16, rw = oracle_btc_row_words(K, w);
+    for (int64_t x = 0; x < N * rw; ++x) words[x] = 0u;
+    for (int64_t r = 0; r < N; ++r)
+        for (int64_t j = 0; j < J; ++j)
+            for (int b = 0; b < w; ++b)
+                if ((idx[r * J + j] >> b) & 1u) {
+                    int64_t bit = j * w + b;
+                    words[r * rw + bit / 32] |= 1u << (bit % 32);
+                }
+}
+
+/* Y[t][j] = sum_i g_i[n] sum_c Bhat_i[n][c] h_i[c] x_m[c] in float64, with
+ * Bhat_i[n][16 jj + q] = +1 if bit q of codebook_i[idx_i[n][jj]] is set, else
+ * -1: the dense product of the codebook-reconstructed layer.  codebooks
+ * [k][c_max], idx [k][N][K/16] (plain indices). */
+void oracle_btc_apply(const uint16_t *codebooks, int c_max, const uint16_t *idx, const uint16_t *g16,
+                      const uint16_t *h16, int64_t N, int64_t K, int k, const uint16_t *X, int64_t M,
+                      const int64_t *rows, int64_t nrows, double *Y)
+{
+    if (!rows) nrows = N;
+    int64_t J = K / 16;
+    #pragma omp parallel
+    {
+        double *What = (double *)malloc(sizeof(double) * (size_t)K);
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t jr = 0; jr < nrows; ++jr) {
+            int64_t n = rows ? rows[jr] : jr;
+            for (int64_t c = 0; c < K; ++c) What[c] = 0.0;
+            for (int i = 0; i < k; ++i) {
+                double gi = decode_binary16(g16[(int64_t)i * N + n]);
+                for (int64_t jj = 0; jj < J; ++jj) {
+                    uint32_t p = codebooks[(int64_t)i * c_max + idx[((int64_t)i * N + n) * J + jj]];
+                    for (int q = 0; q < 16; ++q) {
+                        int64_t c = 16 * jj + q;
+                        double s = ((p >> q) & 1u) ? 1.0 : -1.0;
+                        What[c] += gi * s * decode_binary16(h16[(int64_t)i * K + c]);
+                    }
+                }
+            }
+            for (int64_t m = 0; m < M; ++m) {
+                double acc = 0.0;
+                for (int64_t c = 0; c < K; ++c) acc += decode_bfloat16(X[m * K + c]) * What[c];
+                Y[m * nrows + jr] = acc;
+            }
+        }
+        free(What);
+    }
+}
