@@ -686,6 +686,30 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
     t = time_graph_calls(torch, lambda: rbw.planes_from_rowmajor(rm, N_OUT, K_IN, K_PLANES, out=Ls, stream=stream),
                          20, stream)
     out["planes_from_rowmajor"] = {"us": t * 1e6, "GBps": 2 * Lp.packed_bytes() / t / 1e9}
+    # binary-codebook layer of the same planes (c = 7132, the 7B configuration: 13-bit
+    # indices): the encoder once, then the LUT application over 32 copies (> L2)
+    try:
+        t0 = time.perf_counter()
+        Bc = rbw.btc_encode(Lp, 7132, iters=10, stream=stream)
+        torch.cuda.synchronize()
+        t_enc = time.perf_counter() - t0
+        bcs = [Bc] + [rbw.BtcLayer(N_OUT, K_IN, K_PLANES, 7132, Lp.g16, Lp.h16, dev) for _ in range(31)]
+        for C in bcs[1:]:
+            C.codebooks.copy_(Bc.codebooks)
+            C.indices.copy_(Bc.indices)
+        Xb = torch.from_numpy(synth.activations(1, K_IN, seed=5).view(np.int16)).to(dev)
+        Yb = torch.empty(1, N_OUT, dtype=torch.float32, device=dev)
+        wsb = rbw.workspace(int(rbw.lib().rb_btc_gemv_workspace_bytes(N_OUT, K_IN)), dev)
+        itb = iter(range(10 ** 9))
+        t = time_graph_calls(torch, lambda: rbw.btc_gemv(bcs[next(itb) % len(bcs)], Xb, Y=Yb, ws=wsb,
+                                                         flags=rbw.RB_LAUNCH_PDL, stream=stream), 64, stream)
+        out["btc_gemv_M1_c7132"] = {"us": t * 1e6, "index_GBps": Bc.index_bytes() / t / 1e9,
+                                    "bits_per_weight": Bc.index_bits / 16, "index_bytes": Bc.index_bytes(),
+                                    "codebook_sizes": [int(Bc.sizes[i, 0].item()) for i in range(K_PLANES)],
+                                    "encode_ms_10_rounds": t_enc * 1e3}
+        del bcs, Bc
+    except rbw.RbError as e:
+        out["btc_gemv_M1_c7132"] = {"unavailable": str(e)}
     # coupled-training gradients of one layer at M = 2048 tokens: G = dY^T X on tcgen05 plus dg, dh
     try:
         Mt = 2048
@@ -799,7 +823,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--mode", choices=["full", "gemv-kernel", "gemv-batch-kernel", "pack-kernel", "gemm-kernel",
-                                       "grad-kernel", "qat-forward-kernel", "svid-kernel", "transpose-kernel",
+                                       "grad-kernel", "qat-forward-kernel", "btc-kernel", "svid-kernel", "transpose-kernel",
                                        "rowmajor-kernel"],
                     default="full",
                     help="kernel-only modes run one kernel a few times (used for ncu captures)")
@@ -839,6 +863,11 @@ def run_kernel_mode(args):
         X = torch.from_numpy(synth.activations(M, K_IN, seed=21).view(np.int16)).to(dev)
         for _ in range(args.launches):
             rbw.qat_forward(W, g, h, K_PLANES, X)
+    elif args.mode == "btc-kernel":                  # rb_btc_gemv at M = 1 on the c = 7132 codebook layer
+        Bc = rbw.btc_encode(base, 7132, iters=2)
+        Xb = torch.from_numpy(synth.activations(1, K_IN, seed=5).view(np.int16)).to(dev)
+        for _ in range(args.launches):
+            rbw.btc_gemv(Bc, Xb)
     elif args.mode == "svid-kernel":                 # greedy SVID, 2 power iterations per plane
         for _ in range(args.launches):
             rbw.svid_greedy(W, K_PLANES, iters=2)

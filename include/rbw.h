@@ -287,6 +287,72 @@ RB_API rb_status rb_gemm_noalloc(const rb_layer_t *layer, const uint16_t *X, int
 RB_API rb_status rb_transpose_planes(const rb_layer_t *layer, uint32_t *planes_t, cudaStream_t stream);
 
 /*
+ * Binary-codebook layer (BTC-LLM, "Binary codebook" and "LUT-GEMM"): every
+ * 16-column group (v = 16) of sign plane i is replaced by the index of a
+ * 16-bit codebook pattern (bit q = column 16 j + q is +1), stored in
+ * w = rb_btc_index_bits(c_max) = ceil(log2 c_max) bits: w / 16 bits per weight
+ * (13 / 16 = 0.8125 at the page's c = 7132).
+ *   codebooks  [k][c_max] uint16 patterns (entries past a plane's size unused).
+ *   indices    [k][N][rb_btc_row_words(K, w)] uint32 streams: index j of row r
+ *              at bits [j w, j w + w) of the row's words, LSB-first.
+ *   g16, h16   as rb_layer_t.
+ */
+typedef struct {
+    int32_t n_out;              /* N */
+    int32_t k_in;               /* K (multiple of 32) */
+    int32_t k_planes;           /* k, 1 or 2 for rb_btc_gemv */
+    int32_t c_max;              /* codebook entries per plane, 1..65536 */
+    int32_t index_bits;         /* rb_btc_index_bits(c_max) */
+    int32_t reserved;           /* must be 0 */
+    const uint16_t *codebooks;
+    const uint32_t *indices;
+    const uint16_t *g16;
+    const uint16_t *h16;
+} rb_btc_layer_t;
+
+RB_API int rb_btc_index_bits(int c_max);                 /* 0 for c_max outside 1..65536 */
+RB_API size_t rb_btc_row_words(int k_in, int index_bits);
+RB_API size_t rb_btc_encode_workspace_bytes(int c_max);
+
+/*
+ * rb_btc_encode -- codebook and index stream of sign plane `plane` of a packed
+ * layer by binary k-means (BTC-LLM, "Binary codebook": Hamming assignment by
+ * XOR + popcount, majority-vote centroids with sign(0) = +1, codebook size
+ * c = min(c_max, number of distinct patterns)).  The initial centroids are
+ * the c most frequent patterns (count descending, then pattern ascending);
+ * `iters` rounds of assignment (ties to the smaller index) and majority update
+ * (a centroid without members is kept) precede the final assignment.
+ *   codebook   [c_max] out (2-byte aligned); entries past c are 0.
+ *   c_out      device int32 (4-byte aligned), nullable: c.
+ *   indices    [N][rb_btc_row_words(K, w)] out (4-byte aligned),
+ *              w = rb_btc_index_bits(c_max).
+ *   workspace  rb_btc_encode_workspace_bytes(c_max) bytes, 16-byte aligned.
+ * Integer arithmetic throughout: bit-exact and deterministic.  iters <= 1000;
+ * N * K / 16 < 2^31.
+ */
+RB_API rb_status rb_btc_encode(const rb_layer_t *layer, int plane, int c_max, int iters, uint16_t *codebook,
+                               int32_t *c_out, uint32_t *indices, void *workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/*
+ * rb_btc_gemv -- Y = sum_i g_i .* (Bhat_i (h_i .* x)) for one token (M = 1),
+ * Bhat_i the codebook reconstruction of plane i (BTC-LLM, "LUT-GEMM": dot
+ * products of the input blocks with the weight patterns are precomputed and
+ * the weights only select them).  The tables are this library's byte tables
+ * (sum of +-h x over 8 columns for all 256 sign bytes, fp32, exact products);
+ * a codebook pattern's product is the sum of the entries of its two bytes.
+ * One CTA per (256-row block, 256-column slice) writes row partials to the
+ * workspace; a second launch adds them in slice order (deterministic).
+ *   X [K] bfloat16 bits.  Y [N] fp32 or bf16.  k = 1 or 2 (else UNSUPPORTED).
+ *   workspace  rb_btc_gemv_workspace_bytes(N, K) bytes.  dev_status: unused
+ *   (nullable); flags: RB_LAUNCH_PDL.
+ */
+RB_API size_t rb_btc_gemv_workspace_bytes(int n_out, int k_in);
+RB_API rb_status rb_btc_gemv(const rb_btc_layer_t *layer, const uint16_t *X, void *Y, rb_dtype y_dtype,
+                             void *workspace, size_t workspace_bytes, int32_t *dev_status, unsigned flags,
+                             cudaStream_t stream);
+
+/*
  * rb_qat_forward -- forward pass of one coupled-training layer (RaBiT,
  * Algorithm 2 forward: the binary cores are derived from the latent weight
  * at every step): Y = X What^T with What = sum_i diag(g_i) B_i diag(h_i), the

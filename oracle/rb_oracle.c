@@ -669,12 +669,7 @@ int oracle_svid_iterative(const float *W, int64_t N, int64_t K, int k, int sweep
  *     c_max) bits (at least 1), LSB-first in a per-row bit stream of
  *     ceil(K/16 * w / 32) words: bits [j w, j w + w) of the row's stream.   */
 
-static int popcount16(uint32_t x)
-{
-    int n = 0;
-    for (int b = 0; b < 16; ++b) n += (x >> b) & 1u;
-    return n;
-}
+static int popcount16(uint32_t x) { return __builtin_popcount(x & 0xFFFFu); }
 
 int oracle_btc_index_bits(int c_max)
 {

@@ -97,11 +97,10 @@ __device__ __forceinline__ void lut_load_h(uint4 (&hr)[KP], const uint16_t* __re
         hr[i] = c0 < K ? *reinterpret_cast<const uint4*>(h16 + (int64_t)i * K + c0) : make_uint4(0, 0, 0, 0);
 }
 
-template <int KP>
-__device__ __forceinline__ void lut_build(float* lut, const uint4 (&hrr)[KP], const uint16_t* __restrict__ X,
-                                          int64_t s, int K)
+template <int KP, int PARTS>
+__device__ __forceinline__ void lut_build_part(float* lut, const uint4 (&hrr)[KP], const uint16_t* __restrict__ X,
+                                               int64_t s, int K, int gg, int part)
 {
-    const int gg = threadIdx.x & 31, part = threadIdx.x >> 5;
     const int64_t c0 = s * 256 + gg * 8;
     const bool col_ok = c0 < K;                   // K % 32 == 0: a group is all in or all out
     float xv[8];
@@ -129,7 +128,7 @@ __device__ __forceinline__ void lut_build(float* lut, const uint4 (&hrr)[KP], co
             const int q = low == 1 ? 0 : low == 2 ? 1 : low == 4 ? 2 : 3;
             L[n] = L[n & (n - 1)] + 2.0f * v[q];
         }
-        constexpr int kBPP = 256 / LutCfg<KP>::warps;          // table bytes per part (thread of a group)
+        constexpr int kBPP = 256 / PARTS;                       // table bytes per part (thread of a group)
         constexpr int kHN = kBPP >= 16 ? kBPP / 16 : 1;         // high nibbles per part
         float Hh[kHN];                            // signed sums of columns 4..7 for this part's high nibbles
 #pragma unroll
@@ -147,6 +146,13 @@ __device__ __forceinline__ void lut_build(float* lut, const uint4 (&hrr)[KP], co
             *reinterpret_cast<float*>(base + b * 256) = L[b & 15] + Hh[(b >> 4) - kHN * part];
         }
     }
+}
+
+template <int KP>
+__device__ __forceinline__ void lut_build(float* lut, const uint4 (&hrr)[KP], const uint16_t* __restrict__ X,
+                                          int64_t s, int K)
+{
+    lut_build_part<KP, LutCfg<KP>::warps>(lut, hrr, X, s, K, threadIdx.x & 31, threadIdx.x >> 5);
 }
 
 // All lookups of the kLutPF register-held tiles: for each word slot, the PRMT
@@ -368,6 +374,108 @@ gemv_lut_kernel(const __grid_constant__ LutBatch batch, int N, int K, int CS, in
         for (int j = 0; j < CS; ++j) y += recv[j * my_span + xo];
         const int64_t r = t_begin * 32 + x0 + xo;
         if (r < N) store_y(Y, ydt, r, y);
+    }
+}
+
+// ---------------------------------------------------------------- binary-codebook LUT kernel
+// rb_btc_gemv (BTC-LLM, "LUT-GEMM").  CTA = (block of 8 row tiles, slice s):
+// it builds the byte tables of slice s, then warp w takes tile 8 b + w with
+// lane l on byte group l of the slice (16-column group l / 2, its low or high
+// byte), so the 32 lanes read 32 different groups of the table (conflict-free)
+// and every lane walks the tile's 32 rows: index from the row's stream
+// (funnel shift of two words), pattern from the codebook (read-only cache),
+// one table entry.  Each lane then holds 32 partial row sums; a transposing
+// warp reduction (16 + 8 + 4 + 2 + 1 shuffles) leaves row r's sum in lane r,
+// which applies g and writes the slice's partial.
+constexpr int kBtcWarps = 8;
+
+// a[32] per lane -> the sum over the warp's lanes of a[lane], in lane `lane`
+__device__ __forceinline__ float warp_transpose_sum(const float (&a)[32], int lane)
+{
+    float b16[16], b8[8], b4[4], b2[2];
+#pragma unroll
+    for (int v = 0; v < 16; ++v) {
+        const bool up = lane & 16;
+        b16[v] = (up ? a[v + 16] : a[v]) + __shfl_xor_sync(0xffffffffu, up ? a[v] : a[v + 16], 16);
+    }
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+        const bool up = lane & 8;
+        b8[v] = (up ? b16[v + 8] : b16[v]) + __shfl_xor_sync(0xffffffffu, up ? b16[v] : b16[v + 8], 8);
+    }
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        const bool up = lane & 4;
+        b4[v] = (up ? b8[v + 4] : b8[v]) + __shfl_xor_sync(0xffffffffu, up ? b8[v] : b8[v + 4], 4);
+    }
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+        const bool up = lane & 2;
+        b2[v] = (up ? b4[v + 2] : b4[v]) + __shfl_xor_sync(0xffffffffu, up ? b4[v] : b4[v + 2], 2);
+    }
+    const bool up = lane & 1;
+    return (up ? b2[1] : b2[0]) + __shfl_xor_sync(0xffffffffu, up ? b2[0] : b2[1], 1);
+}
+
+template <int KP>
+__global__ void __launch_bounds__(kBtcWarps * 32)
+btc_gemv_kernel(const rb_btc_layer_t L, const uint16_t* __restrict__ X, float* __restrict__ part)
+{
+    static_assert(KP <= 2, "one 64 KB table region holds k <= 2");
+    extern __shared__ __align__(1024) float lut[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int N = L.n_out, K = L.k_in, w = L.index_bits;
+    const int64_t S = num_slices(K), Nt = num_row_tiles(N);
+    const int64_t s = blockIdx.x % S, t = (blockIdx.x / S) * kBtcWarps + warp;
+    const int64_t rw = ((int64_t)(K / 16) * w + 31) / 32;
+    uint4 hr[KP];
+    lut_load_h<KP>(hr, L.h16, s, K);
+    pdl_launch_dependents();
+    pdl_wait();
+    lut_build_part<KP, kBtcWarps>(lut, hr, X, s, K, lane, warp);
+    __syncthreads();
+    if (t >= Nt) return;
+
+    const int64_t J = s * 16 + (lane >> 1);                 // this lane's 16-column group
+    const bool col_ok = s * 256 + lane * 8 < K;
+    const int64_t bit = J * w;
+    const int64_t wi = bit >> 5;
+    const uint32_t sh = (uint32_t)(bit & 31), mask = (1u << w) - 1u, bsh = 8u * (lane & 1);
+    const uint32_t tb = smem_u32(lut) + (uint32_t)lane * 4u;
+    float acc[KP][32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+        const int64_t row = min(t * 32 + r, (int64_t)N - 1);   // rows past N: any valid row, not stored
+#pragma unroll
+        for (int i = 0; i < KP; ++i) {
+            const uint32_t* st = L.indices + ((int64_t)i * N + row) * rw;
+            const uint32_t lo = col_ok ? __ldg(st + wi) : 0u;
+            const uint32_t hi = (col_ok && wi + 1 < rw) ? __ldg(st + wi + 1) : 0u;
+            const uint32_t idx = min(__funnelshift_r(lo, hi, sh) & mask, (uint32_t)L.c_max - 1u);
+            const uint32_t pat = __ldg(L.codebooks + (int64_t)i * L.c_max + idx);
+            const uint32_t byte = (pat >> bsh) & 0xFFu;
+            acc[i][r] = col_ok ? lds_f32(tb + (uint32_t)(i & 1) * 128u + byte * 256u) : 0.0f;
+        }
+    }
+    const int64_t row = t * 32 + lane;
+    float y = 0.0f;
+#pragma unroll
+    for (int i = 0; i < KP; ++i) {
+        const float sum = warp_transpose_sum(acc[i], lane);
+        y += row < N ? __half2float(__ushort_as_half(L.g16[(int64_t)i * N + row])) * sum : 0.0f;
+    }
+    if (row < N) part[s * N + row] = y;
+}
+
+// Y[n] = sum over slices of the partials, in slice order
+__global__ void btc_reduce_kernel(const float* __restrict__ part, int N, int S, void* __restrict__ Y, int ydt)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    for (int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; n < N; n += (int64_t)gridDim.x * blockDim.x) {
+        float y = 0.0f;
+        for (int s = 0; s < S; ++s) y += part[(int64_t)s * N + n];
+        store_y(Y, ydt, n, y);
     }
 }
 
@@ -1023,4 +1131,58 @@ extern "C" rb_status rb_gemv_batch(const rb_layer_t* const* layers, const uint16
     for (int j = 0; j < count; ++j)
         if (!layers[j]) return RB_ERR_ARG;
     return gemv_dispatch(layers, X, Y, count, M, y_dtype, dev_status, flags, stream);
+}
+
+extern "C" size_t rb_btc_gemv_workspace_bytes(int n_out, int k_in)
+{
+    if (n_out < 1 || k_in < 32 || k_in % 32 != 0) return 0;
+    return (size_t)num_slices(k_in) * (size_t)n_out * 4;
+}
+
+extern "C" rb_status rb_btc_gemv(const rb_btc_layer_t* layer, const uint16_t* X, void* Y, rb_dtype y_dtype,
+                                 void* workspace, size_t workspace_bytes, int32_t* dev_status, unsigned flags,
+                                 cudaStream_t stream)
+{
+    (void)dev_status;
+    if (!layer || !X || !Y || !layer->codebooks || !layer->indices || !layer->g16 || !layer->h16 ||
+        layer->reserved != 0)
+        return RB_ERR_ARG;
+    if ((y_dtype != RB_F32 && y_dtype != RB_BF16) || (flags & ~RB_LAUNCH_PDL)) return RB_ERR_ARG;
+    if (layer->c_max < 1 || layer->c_max > 65536 || layer->index_bits != rb_btc_index_bits(layer->c_max))
+        return RB_ERR_ARG;
+    if (layer->k_planes < 1 || layer->k_planes > 8) return RB_ERR_ARG;
+    if (layer->k_planes > 2) return RB_ERR_UNSUPPORTED;
+    const int N = layer->n_out, K = layer->k_in;
+    if (N < 1 || K < 32 || K % 32 != 0) return RB_ERR_SHAPE;
+    const void* ptrs[] = {layer->codebooks, layer->indices, layer->g16, layer->h16, X, Y};
+    for (const void* q : ptrs)
+        if (!aligned16(q)) return RB_ERR_ALIGN;
+    if (!workspace || workspace_bytes < rb_btc_gemv_workspace_bytes(N, K)) return RB_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return RB_ERR_ALIGN;
+    if (!device_is_sm100()) return RB_ERR_UNSUPPORTED;
+    const bool pdl = (flags & RB_LAUNCH_PDL) != 0;
+    const int64_t S = num_slices(K), Nt = num_row_tiles(N);
+    const int64_t ctas = (Nt + kBtcWarps - 1) / kBtcWarps * S;
+    if (ctas > INT32_MAX) return RB_ERR_UNSUPPORTED;
+    const int smem = lut_table_bytes(2);
+    float* part = static_cast<float*>(workspace);
+    static std::atomic<bool> attr_set[64][2];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RB_ERR_CUDA;
+    const int kk = layer->k_planes - 1;
+    if (!attr_set[dev][kk].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kk ? btc_gemv_kernel<2> : btc_gemv_kernel<1>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return RB_ERR_CUDA;
+        attr_set[dev][kk].store(true, std::memory_order_release);
+    }
+    rb_status st = kk ? launch(btc_gemv_kernel<2>, dim3((unsigned)ctas), dim3(kBtcWarps * 32), (size_t)smem, stream,
+                               pdl, *layer, X, part)
+                      : launch(btc_gemv_kernel<1>, dim3((unsigned)ctas), dim3(kBtcWarps * 32), (size_t)smem, stream,
+                               pdl, *layer, X, part);
+    if (st != RB_OK) return st;
+    int64_t rb = (N + 255) / 256;
+    if (rb > 4 * num_sms()) rb = 4 * num_sms();
+    return launch(btc_reduce_kernel, dim3((unsigned)rb), dim3(256), 0, stream, true, (const float*)part, N, (int)S, Y,
+                  (int)y_dtype);
 }

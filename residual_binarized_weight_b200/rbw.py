@@ -43,6 +43,12 @@ SIGNATURES = {
     "rb_qat_forward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _u32, _vp]),
     "rb_qat_backward_workspace_bytes": (_sz, [_i32, _i32, _i32]),
     "rb_qat_backward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "rb_btc_index_bits": (_i32, [_i32]),
+    "rb_btc_row_words": (_sz, [_i32, _i32]),
+    "rb_btc_encode_workspace_bytes": (_sz, [_i32]),
+    "rb_btc_encode": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "rb_btc_gemv_workspace_bytes": (_sz, [_i32, _i32]),
+    "rb_btc_gemv": (_i32, [_vp, _vp, _vp, _i32, _vp, _sz, _vp, _u32, _vp]),
     "rb_svid_workspace_bytes": (_sz, [_i32, _i32]),
     "rb_svid_greedy": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "rb_svid_iterative_workspace_bytes": (_sz, [_i32, _i32, _i32]),
@@ -55,6 +61,12 @@ SIGNATURES = {
 class RbLayer(ctypes.Structure):
     _fields_ = [("n_out", ctypes.c_int32), ("k_in", ctypes.c_int32), ("k_planes", ctypes.c_int32),
                 ("reserved", ctypes.c_int32), ("planes", _vp), ("g16", _vp), ("h16", _vp)]
+
+
+class RbBtcLayer(ctypes.Structure):
+    _fields_ = [("n_out", ctypes.c_int32), ("k_in", ctypes.c_int32), ("k_planes", ctypes.c_int32),
+                ("c_max", ctypes.c_int32), ("index_bits", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("codebooks", _vp), ("indices", _vp), ("g16", _vp), ("h16", _vp)]
 
 
 _lib = None
@@ -346,3 +358,53 @@ def shard_rows(layer: PackedLayer, row0, rows, stream=None):
     st = lib().rb_shard_rows(ctypes.byref(L), row0, rows, _ptr(out.planes), _ptr(out.g16), _stream(stream))
     _check("rb_shard_rows", st)
     return out
+
+
+# ---------------------------------------------------------------- binary codebook
+class BtcLayer:
+    """Device tensors of a binary-codebook layer (owns the codebooks and index streams; shares g16, h16)."""
+
+    def __init__(self, n_out, k_in, k_planes, c_max, g16, h16, device="cuda"):
+        self.n_out, self.k_in, self.k_planes, self.c_max = n_out, k_in, k_planes, c_max
+        self.index_bits = int(lib().rb_btc_index_bits(c_max))
+        self.row_words = int(lib().rb_btc_row_words(k_in, self.index_bits))
+        if self.index_bits == 0 or self.row_words == 0:
+            raise ValueError("invalid codebook layer shape")
+        self.codebooks = torch.zeros(k_planes, c_max, dtype=torch.int16, device=device)
+        self.indices = torch.zeros(k_planes, n_out, self.row_words, dtype=torch.int32, device=device)
+        self.sizes = torch.zeros(k_planes, 4, dtype=torch.int32, device=device)   # c of each plane in column 0
+        self.g16, self.h16 = g16, h16
+
+    def struct(self):
+        return RbBtcLayer(self.n_out, self.k_in, self.k_planes, self.c_max, self.index_bits, 0,
+                          self.codebooks.data_ptr(), self.indices.data_ptr(), self.g16.data_ptr(),
+                          self.h16.data_ptr())
+
+    def index_bytes(self):
+        return self.indices.numel() * 4
+
+
+def btc_encode(layer: PackedLayer, c_max, iters=10, stream=None):
+    """rb_btc_encode for every plane of a packed layer -> BtcLayer."""
+    out = BtcLayer(layer.n_out, layer.k_in, layer.k_planes, c_max, layer.g16, layer.h16, layer.planes.device)
+    ws = workspace(int(lib().rb_btc_encode_workspace_bytes(c_max)), layer.planes.device)
+    L = layer.struct()
+    for i in range(layer.k_planes):
+        st = lib().rb_btc_encode(ctypes.byref(L), i, c_max, iters, _ptr(out.codebooks[i]), _ptr(out.sizes[i]),
+                                 _ptr(out.indices[i]), _ptr(ws), ws.numel(), _stream(stream))
+        _check("rb_btc_encode", st)
+    return out
+
+
+def btc_gemv(layer: BtcLayer, X, Y=None, ws=None, flags=0, stream=None, y_dtype=torch.float32):
+    """rb_btc_gemv: X bf16 [1][K] (or [K]) -> Y [1][N]."""
+    if Y is None:
+        Y = torch.empty(1, layer.n_out, dtype=y_dtype, device=X.device)
+    ws = ws if ws is not None else workspace(int(lib().rb_btc_gemv_workspace_bytes(layer.n_out, layer.k_in)),
+                                             X.device)
+    L = layer.struct()
+    ydt = RB_BF16 if Y.dtype == torch.bfloat16 else RB_F32
+    st = lib().rb_btc_gemv(ctypes.byref(L), _ptr(X), _ptr(Y), ydt, _ptr(ws), ws.numel(), None, flags,
+                           _stream(stream))
+    _check("rb_btc_gemv", st)
+    return Y
