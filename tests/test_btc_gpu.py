@@ -50,8 +50,11 @@ def test_encode_is_bit_exact(N, K, k, c_max, iters, skew):
 
 
 @pytest.mark.parametrize("N,K,k,c_max,skew", [(96, 256, 1, 5, True), (300, 800, 2, 40, True), (4097, 544, 2, 300, False),
-                                              (4096, 4096, 2, 256, False), (1000, 4096, 1, 1024, False)])
+                                              (4096, 4096, 2, 256, False), (1000, 4096, 1, 1024, False),
+                                              (260, 8192, 2, 100, False)])
 def test_gemv_matches_oracle(N, K, k, c_max, skew):
+    """Ragged N and K, k = 1 and 2, up to 32 slices (K = 8192), fp32 and bf16
+    output, with and without PDL (bit-identical)."""
     planes, g16, h16 = make(N, K, k, seed=N * 3 + K + k, skew=skew)
     L = cases.upload_layer(planes, g16, h16, N, K, k)
     B = rbw.btc_encode(L, c_max, iters=3)
