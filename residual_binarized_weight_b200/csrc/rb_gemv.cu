@@ -826,8 +826,8 @@ int lut_resident(int CS, int smem)
 constexpr int kLutBuildTiles = 8;
 
 // Single layer (count == 1): lowest latency.  Slices per CTA = ceil(S/16),
-// CS = ceil(S / that) CTAs per cluster, one row chunk (R) fewer than the GPU
-// keeps clusters resident, one wave.
+// CS = ceil(S / that) CTAs per cluster, row chunks (R): one cluster fewer than
+// the SMs hold at one CTA each (and no more than stay resident), one wave.
 // Batch: CS (a power of two) and R minimise the modelled time waves * (time of
 // one CTA), where a CTA builds ceil(S/CS) tables and runs ceil(rows/R) row
 // tiles through each, and the count * R clusters run in ceil(count * R /
@@ -846,18 +846,17 @@ rb_status lut_plan_uncached(int N, int K, int count, LutPlan* plan)
         const int spc = (int)((S + 15) / 16);
         const int CS = (int)((S + spc - 1) / spc);
         const int sms = num_sms();
-        int R = CS > 1 ? sms / CS : sms;
+        // clusters: one fewer than the SMs hold at one CTA each, which leaves SMs
+        // free for the first CTAs of the next layer's launch (PDL): 8 clusters of
+        // 16 on 148 SMs measured 4.37 against 4.60 us per layer with 9 in a
+        // dependent chain of 4096 x 4096 layers (7 and 6: 4.57 and 5.8 us)
+        int R = CS > 1 ? sms / CS - 1 : sms;
         if (R < 1) R = 1;
         if (R > Nt) R = (int)Nt;
         while (R < Nt && lut_table_bytes(KP) + lut_row_bytes(Nt, R, CS) > cap) ++R;
         LutPlan p{CS, R, lut_table_bytes(KP) + lut_row_bytes(Nt, R, CS)};
         if (CS > 1) {
-            // one cluster fewer than the GPU keeps resident, which leaves SMs free for
-            // the first CTAs of the next layer's launch (PDL): 8 clusters of 16
-            // against 9 measured 4.37 against 4.60 us per layer in a dependent
-            // chain of 4096 x 4096 layers (7 and 6: 4.57 and 5.8 us)
-            int active = lut_resident<KP>(CS, p.smem);
-            if (active > 1) --active;
+            const int active = lut_resident<KP>(CS, p.smem);
             if (active > 0 && active < R) {
                 p.R = active;
                 p.smem = lut_table_bytes(KP) + lut_row_bytes(Nt, p.R, CS);
