@@ -707,6 +707,13 @@ def other_rows(args, torch, rbw, synth, dev, W, g, h, bf16_peak):
                                     "bits_per_weight": Bc.index_bits / 16, "index_bytes": Bc.index_bytes(),
                                     "codebook_sizes": [int(Bc.sizes[i, 0].item()) for i in range(K_PLANES)],
                                     "encode_ms_10_rounds": t_enc * 1e3}
+        # the same 32 layers in one rb_btc_gemv_batch call (one launch pair)
+        Ybs = [torch.empty(1, N_OUT, dtype=torch.float32, device=dev) for _ in bcs]
+        wsbb = rbw.workspace(int(rbw.lib().rb_btc_gemv_batch_workspace_bytes(N_OUT, K_IN, len(bcs))), dev)
+        t = time_graph_calls(torch, lambda: rbw.btc_gemv_batch(bcs, [Xb] * len(bcs), Ybs, ws=wsbb,
+                                                               flags=rbw.RB_LAUNCH_PDL, stream=stream), 8,
+                             stream) / len(bcs)
+        out["btc_gemv_batch32_M1_c7132"] = {"us_per_layer": t * 1e6, "index_GBps": Bc.index_bytes() / t / 1e9}
         del bcs, Bc
     except rbw.RbError as e:
         out["btc_gemv_M1_c7132"] = {"unavailable": str(e)}

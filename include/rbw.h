@@ -353,6 +353,20 @@ RB_API rb_status rb_btc_gemv(const rb_btc_layer_t *layer, const uint16_t *X, voi
                              cudaStream_t stream);
 
 /*
+ * rb_btc_gemv_batch -- rb_btc_gemv for `count` independent codebook layers of
+ * one shape (same N, K, k, c_max), up to 64 per launch pair (more are cut into
+ * groups of 64 that reuse the workspace in stream order).  layers[j], X[j],
+ * Y[j] are host arrays of device pointers; each Y[j] equals rb_btc_gemv's
+ * result for that layer bit for bit (the same per-slice partials, added in
+ * the same order).
+ *   workspace  rb_btc_gemv_batch_workspace_bytes(N, K, count) bytes.
+ */
+RB_API size_t rb_btc_gemv_batch_workspace_bytes(int n_out, int k_in, int count);
+RB_API rb_status rb_btc_gemv_batch(const rb_btc_layer_t *const *layers, const uint16_t *const *X, void *const *Y,
+                                   int count, rb_dtype y_dtype, void *workspace, size_t workspace_bytes,
+                                   int32_t *dev_status, unsigned flags, cudaStream_t stream);
+
+/*
  * rb_qat_forward -- forward pass of one coupled-training layer (RaBiT,
  * Algorithm 2 forward: the binary cores are derived from the latent weight
  * at every step): Y = X What^T with What = sum_i diag(g_i) B_i diag(h_i), the

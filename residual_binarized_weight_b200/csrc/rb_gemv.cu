@@ -417,19 +417,38 @@ __device__ __forceinline__ float warp_transpose_sum(const float (&a)[32], int la
     return (up ? b2[1] : b2[0]) + __shfl_xor_sync(0xffffffffu, up ? b2[0] : b2[1], 1);
 }
 
+// Independent codebook layers of one shape handled by one launch (pointers per layer).
+constexpr int kBtcMaxBatch = 64;
+struct BtcBatch {
+    const uint32_t* indices[kBtcMaxBatch];
+    const uint16_t* codebooks[kBtcMaxBatch];
+    const uint16_t* g16[kBtcMaxBatch];
+    const uint16_t* h16[kBtcMaxBatch];
+    const uint16_t* X[kBtcMaxBatch];
+    void* Y[kBtcMaxBatch];
+};
+
+// grid: layers x row blocks x slices; part [layer][S][N]
 template <int KP>
 __global__ void __launch_bounds__(kBtcWarps * 32)
-btc_gemv_kernel(const rb_btc_layer_t L, const uint16_t* __restrict__ X, float* __restrict__ part)
+btc_gemv_kernel(const __grid_constant__ BtcBatch B, int N, int K, int c_max, int w, float* __restrict__ part)
 {
     static_assert(KP <= 2, "one 64 KB table region holds k <= 2");
     extern __shared__ __align__(1024) float lut[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int N = L.n_out, K = L.k_in, w = L.index_bits;
     const int64_t S = num_slices(K), Nt = num_row_tiles(N);
-    const int64_t s = blockIdx.x % S, t = (blockIdx.x / S) * kBtcWarps + warp;
+    const int64_t per_layer = (Nt + kBtcWarps - 1) / kBtcWarps * S;
+    const int layer = (int)(blockIdx.x / per_layer);
+    const int64_t bx = blockIdx.x % per_layer;
+    const int64_t s = bx % S, t = (bx / S) * kBtcWarps + warp;
     const int64_t rw = ((int64_t)(K / 16) * w + 31) / 32;
+    const uint32_t* __restrict__ indices = B.indices[layer];
+    const uint16_t* __restrict__ codebooks = B.codebooks[layer];
+    const uint16_t* __restrict__ g16 = B.g16[layer];
+    const uint16_t* __restrict__ X = B.X[layer];
+    part += (int64_t)layer * S * N;
     uint4 hr[KP];
-    lut_load_h<KP>(hr, L.h16, s, K);
+    lut_load_h<KP>(hr, B.h16[layer], s, K);
     pdl_launch_dependents();
     pdl_wait();
     lut_build_part<KP, kBtcWarps>(lut, hr, X, s, K, lane, warp);
@@ -448,11 +467,11 @@ btc_gemv_kernel(const rb_btc_layer_t L, const uint16_t* __restrict__ X, float* _
         const int64_t row = min(t * 32 + r, (int64_t)N - 1);   // rows past N: any valid row, not stored
 #pragma unroll
         for (int i = 0; i < KP; ++i) {
-            const uint32_t* st = L.indices + ((int64_t)i * N + row) * rw;
+            const uint32_t* st = indices + ((int64_t)i * N + row) * rw;
             const uint32_t lo = col_ok ? __ldg(st + wi) : 0u;
             const uint32_t hi = (col_ok && wi + 1 < rw) ? __ldg(st + wi + 1) : 0u;
-            const uint32_t idx = min(__funnelshift_r(lo, hi, sh) & mask, (uint32_t)L.c_max - 1u);
-            const uint32_t pat = __ldg(L.codebooks + (int64_t)i * L.c_max + idx);
+            const uint32_t idx = min(__funnelshift_r(lo, hi, sh) & mask, (uint32_t)c_max - 1u);
+            const uint32_t pat = __ldg(codebooks + (int64_t)i * c_max + idx);
             const uint32_t byte = (pat >> bsh) & 0xFFu;
             acc[i][r] = col_ok ? lds_f32(tb + (uint32_t)(i & 1) * 128u + byte * 256u) : 0.0f;
         }
@@ -462,20 +481,25 @@ btc_gemv_kernel(const rb_btc_layer_t L, const uint16_t* __restrict__ X, float* _
 #pragma unroll
     for (int i = 0; i < KP; ++i) {
         const float sum = warp_transpose_sum(acc[i], lane);
-        y += row < N ? __half2float(__ushort_as_half(L.g16[(int64_t)i * N + row])) * sum : 0.0f;
+        y += row < N ? __half2float(__ushort_as_half(g16[(int64_t)i * N + row])) * sum : 0.0f;
     }
     if (row < N) part[s * N + row] = y;
 }
 
-// Y[n] = sum over slices of the partials, in slice order
-__global__ void btc_reduce_kernel(const float* __restrict__ part, int N, int S, void* __restrict__ Y, int ydt)
+// Y[layer][n] = sum over slices of the partials, in slice order
+__global__ void btc_reduce_kernel(const __grid_constant__ BtcBatch B, int count, const float* __restrict__ part,
+                                  int N, int S, int ydt)
 {
     pdl_launch_dependents();
     pdl_wait();
-    for (int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; n < N; n += (int64_t)gridDim.x * blockDim.x) {
+    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < (int64_t)count * N;
+         x += (int64_t)gridDim.x * blockDim.x) {
+        const int layer = (int)(x / N);
+        const int64_t n = x - (int64_t)layer * N;
+        const float* p = part + (int64_t)layer * S * N + n;
         float y = 0.0f;
-        for (int s = 0; s < S; ++s) y += part[(int64_t)s * N + n];
-        store_y(Y, ydt, n, y);
+        for (int s = 0; s < S; ++s) y += p[(int64_t)s * N];
+        store_y(B.Y[layer], ydt, n, y);
     }
 }
 
@@ -1138,50 +1162,86 @@ extern "C" size_t rb_btc_gemv_workspace_bytes(int n_out, int k_in)
     return (size_t)num_slices(k_in) * (size_t)n_out * 4;
 }
 
-extern "C" rb_status rb_btc_gemv(const rb_btc_layer_t* layer, const uint16_t* X, void* Y, rb_dtype y_dtype,
-                                 void* workspace, size_t workspace_bytes, int32_t* dev_status, unsigned flags,
-                                 cudaStream_t stream)
+extern "C" size_t rb_btc_gemv_batch_workspace_bytes(int n_out, int k_in, int count)
+{
+    if (count < 1) return 0;
+    return rb_btc_gemv_workspace_bytes(n_out, k_in) * (size_t)(count < kBtcMaxBatch ? count : kBtcMaxBatch);
+}
+
+extern "C" rb_status rb_btc_gemv_batch(const rb_btc_layer_t* const* layers, const uint16_t* const* X,
+                                       void* const* Y, int count, rb_dtype y_dtype, void* workspace,
+                                       size_t workspace_bytes, int32_t* dev_status, unsigned flags,
+                                       cudaStream_t stream)
 {
     (void)dev_status;
-    if (!layer || !X || !Y || !layer->codebooks || !layer->indices || !layer->g16 || !layer->h16 ||
-        layer->reserved != 0)
-        return RB_ERR_ARG;
+    if (!layers || !X || !Y || count < 1) return RB_ERR_ARG;
     if ((y_dtype != RB_F32 && y_dtype != RB_BF16) || (flags & ~RB_LAUNCH_PDL)) return RB_ERR_ARG;
-    if (layer->c_max < 1 || layer->c_max > 65536 || layer->index_bits != rb_btc_index_bits(layer->c_max))
-        return RB_ERR_ARG;
-    if (layer->k_planes < 1 || layer->k_planes > 8) return RB_ERR_ARG;
-    if (layer->k_planes > 2) return RB_ERR_UNSUPPORTED;
-    const int N = layer->n_out, K = layer->k_in;
+    const rb_btc_layer_t* L0 = layers[0];
+    if (!L0) return RB_ERR_ARG;
+    for (int j = 0; j < count; ++j) {
+        const rb_btc_layer_t* L = layers[j];
+        if (!L || !X[j] || !Y[j] || !L->codebooks || !L->indices || !L->g16 || !L->h16 || L->reserved != 0)
+            return RB_ERR_ARG;
+        if (L->c_max < 1 || L->c_max > 65536 || L->index_bits != rb_btc_index_bits(L->c_max)) return RB_ERR_ARG;
+        if (L->k_planes < 1 || L->k_planes > 8) return RB_ERR_ARG;
+        if (L->n_out != L0->n_out || L->k_in != L0->k_in || L->k_planes != L0->k_planes || L->c_max != L0->c_max)
+            return RB_ERR_SHAPE;
+        const void* ptrs[] = {L->codebooks, L->indices, L->g16, L->h16, X[j], Y[j]};
+        for (const void* q : ptrs)
+            if (!aligned16(q)) return RB_ERR_ALIGN;
+    }
+    if (L0->k_planes > 2) return RB_ERR_UNSUPPORTED;
+    const int N = L0->n_out, K = L0->k_in;
     if (N < 1 || K < 32 || K % 32 != 0) return RB_ERR_SHAPE;
-    const void* ptrs[] = {layer->codebooks, layer->indices, layer->g16, layer->h16, X, Y};
-    for (const void* q : ptrs)
-        if (!aligned16(q)) return RB_ERR_ALIGN;
-    if (!workspace || workspace_bytes < rb_btc_gemv_workspace_bytes(N, K)) return RB_ERR_WORKSPACE;
+    if (!workspace || workspace_bytes < rb_btc_gemv_batch_workspace_bytes(N, K, count)) return RB_ERR_WORKSPACE;
     if (!aligned16(workspace)) return RB_ERR_ALIGN;
     if (!device_is_sm100()) return RB_ERR_UNSUPPORTED;
     const bool pdl = (flags & RB_LAUNCH_PDL) != 0;
     const int64_t S = num_slices(K), Nt = num_row_tiles(N);
-    const int64_t ctas = (Nt + kBtcWarps - 1) / kBtcWarps * S;
-    if (ctas > INT32_MAX) return RB_ERR_UNSUPPORTED;
+    const int64_t per_layer = (Nt + kBtcWarps - 1) / kBtcWarps * S;
+    if (per_layer * kBtcMaxBatch > INT32_MAX) return RB_ERR_UNSUPPORTED;
     const int smem = lut_table_bytes(2);
     float* part = static_cast<float*>(workspace);
     static std::atomic<bool> attr_set[64][2];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RB_ERR_CUDA;
-    const int kk = layer->k_planes - 1;
+    const int kk = L0->k_planes - 1;
     if (!attr_set[dev][kk].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(kk ? btc_gemv_kernel<2> : btc_gemv_kernel<1>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return RB_ERR_CUDA;
         attr_set[dev][kk].store(true, std::memory_order_release);
     }
-    rb_status st = kk ? launch(btc_gemv_kernel<2>, dim3((unsigned)ctas), dim3(kBtcWarps * 32), (size_t)smem, stream,
-                               pdl, *layer, X, part)
-                      : launch(btc_gemv_kernel<1>, dim3((unsigned)ctas), dim3(kBtcWarps * 32), (size_t)smem, stream,
-                               pdl, *layer, X, part);
-    if (st != RB_OK) return st;
-    int64_t rb = (N + 255) / 256;
-    if (rb > 4 * num_sms()) rb = 4 * num_sms();
-    return launch(btc_reduce_kernel, dim3((unsigned)rb), dim3(256), 0, stream, true, (const float*)part, N, (int)S, Y,
-                  (int)y_dtype);
+    for (int base = 0; base < count; base += kBtcMaxBatch) {
+        const int n = count - base < kBtcMaxBatch ? count - base : kBtcMaxBatch;
+        BtcBatch b = {};
+        for (int j = 0; j < n; ++j) {
+            const rb_btc_layer_t* L = layers[base + j];
+            b.indices[j] = L->indices;
+            b.codebooks[j] = L->codebooks;
+            b.g16[j] = L->g16;
+            b.h16[j] = L->h16;
+            b.X[j] = X[base + j];
+            b.Y[j] = Y[base + j];
+        }
+        const dim3 grid((unsigned)(per_layer * n));
+        rb_status st = kk ? launch(btc_gemv_kernel<2>, grid, dim3(kBtcWarps * 32), (size_t)smem, stream, pdl, b, N, K,
+                                   L0->c_max, L0->index_bits, part)
+                          : launch(btc_gemv_kernel<1>, grid, dim3(kBtcWarps * 32), (size_t)smem, stream, pdl, b, N, K,
+                                   L0->c_max, L0->index_bits, part);
+        if (st != RB_OK) return st;
+        int64_t rb = ((int64_t)n * N + 255) / 256;
+        if (rb > 4 * num_sms()) rb = 4 * num_sms();
+        st = launch(btc_reduce_kernel, dim3((unsigned)rb), dim3(256), 0, stream, true, b, n, (const float*)part, N,
+                    (int)S, (int)y_dtype);
+        if (st != RB_OK) return st;
+    }
+    return RB_OK;
+}
+
+extern "C" rb_status rb_btc_gemv(const rb_btc_layer_t* layer, const uint16_t* X, void* Y, rb_dtype y_dtype,
+                                 void* workspace, size_t workspace_bytes, int32_t* dev_status, unsigned flags,
+                                 cudaStream_t stream)
+{
+    return rb_btc_gemv_batch(&layer, &X, &Y, 1, y_dtype, workspace, workspace_bytes, dev_status, flags, stream);
 }

@@ -49,6 +49,8 @@ SIGNATURES = {
     "rb_btc_encode": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "rb_btc_gemv_workspace_bytes": (_sz, [_i32, _i32]),
     "rb_btc_gemv": (_i32, [_vp, _vp, _vp, _i32, _vp, _sz, _vp, _u32, _vp]),
+    "rb_btc_gemv_batch_workspace_bytes": (_sz, [_i32, _i32, _i32]),
+    "rb_btc_gemv_batch": (_i32, [_vp, _vp, _vp, _i32, _i32, _vp, _sz, _vp, _u32, _vp]),
     "rb_svid_workspace_bytes": (_sz, [_i32, _i32]),
     "rb_svid_greedy": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "rb_svid_iterative_workspace_bytes": (_sz, [_i32, _i32, _i32]),
@@ -408,3 +410,19 @@ def btc_gemv(layer: BtcLayer, X, Y=None, ws=None, flags=0, stream=None, y_dtype=
                            _stream(stream))
     _check("rb_btc_gemv", st)
     return Y
+
+
+def btc_gemv_batch(layers, Xs, Ys, ws=None, flags=0, stream=None):
+    """rb_btc_gemv_batch: codebook layers of one shape; Xs[j] bf16 [1][K], Ys[j] [1][N] (CUDA tensors)."""
+    n = len(layers)
+    structs = (RbBtcLayer * n)(*[L.struct() for L in layers])
+    lp = (ctypes.POINTER(RbBtcLayer) * n)(*[ctypes.pointer(structs[j]) for j in range(n)])
+    xp = (ctypes.c_void_p * n)(*[X.data_ptr() for X in Xs])
+    yp = (ctypes.c_void_p * n)(*[Y.data_ptr() for Y in Ys])
+    L0 = layers[0]
+    ws = ws if ws is not None else workspace(
+        int(lib().rb_btc_gemv_batch_workspace_bytes(L0.n_out, L0.k_in, n)), Xs[0].device)
+    ydt = RB_BF16 if Ys[0].dtype == torch.bfloat16 else RB_F32
+    st = lib().rb_btc_gemv_batch(lp, xp, yp, n, ydt, _ptr(ws), ws.numel(), None, flags, _stream(stream))
+    _check("rb_btc_gemv_batch", st)
+    return Ys

@@ -110,3 +110,23 @@ def test_errors():
     with pytest.raises(rbw.RbError) as e:
         rbw.btc_gemv(B, Xd)
     assert e.value.status == rbw.RB_ERR_UNSUPPORTED
+
+
+def test_gemv_batch_equals_single_calls():
+    """A batch of distinct codebook layers and tokens (70 layers: a group of 64
+    and one of 6) reproduces each single-layer call bit for bit."""
+    N, K, k = 200, 512, 2
+    layers, Xs, singles = [], [], []
+    for j in range(70):
+        planes, g16, h16 = make(N, K, k, seed=100 + j % 5)
+        L = cases.upload_layer(planes, g16, h16, N, K, k)
+        layers.append(rbw.btc_encode(L, 32, iters=2))
+        layers[-1].keep = L                           # the scales live in the packed layer
+        Xs.append(cases.to_dev(synth.activations(1, K, seed=200 + j)))
+    for B, X in zip(layers, Xs):
+        singles.append(rbw.btc_gemv(B, X))
+    Ys = [torch.empty(1, N, device="cuda") for _ in layers]
+    rbw.btc_gemv_batch(layers, Xs, Ys, flags=rbw.RB_LAUNCH_PDL)
+    torch.cuda.synchronize()
+    for a, b in zip(Ys, singles):
+        assert torch.equal(a, b)
