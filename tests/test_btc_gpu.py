@@ -130,3 +130,20 @@ def test_gemv_batch_equals_single_calls():
     torch.cuda.synchronize()
     for a, b in zip(Ys, singles):
         assert torch.equal(a, b)
+
+
+def test_gemv_batch_of_full_size_layers_equals_single_calls():
+    """48 layers of 4096 x 1024 in one batch (3072 CTAs): every output equals
+    the single-layer call bit for bit."""
+    N, K, k = 4096, 1024, 2
+    planes, g16, h16 = make(N, K, k, seed=77)
+    L = cases.upload_layer(planes, g16, h16, N, K, k)
+    B = rbw.btc_encode(L, 512, iters=2)
+    B.keep = L
+    Xs = [cases.to_dev(synth.activations(1, K, seed=300 + j)) for j in range(48)]
+    singles = [rbw.btc_gemv(B, X) for X in Xs]
+    Ys = [torch.empty(1, N, device="cuda") for _ in Xs]
+    rbw.btc_gemv_batch([B] * 48, Xs, Ys)
+    torch.cuda.synchronize()
+    for a, b in zip(Ys, singles):
+        assert torch.equal(a, b)
