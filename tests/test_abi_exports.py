@@ -65,6 +65,28 @@ def test_size_helpers_reject_bad_shapes(L):
     assert L.rb_qat_backward_workspace_bytes(4096, 4096, 2) > 0
     assert L.rb_rowmajor_words(4096, 4096, 2) == 2 * 4096 * 128
     assert L.rb_svid_workspace_bytes(4096, 4096) > 0
+    # rb_gemv takes the tcgen05 path (and asks for a workspace) only above the crossover
+    assert L.rb_gemv_workspace_bytes(4096, 4096, 2, 64) == 0
+    assert L.rb_gemv_workspace_bytes(14336, 4096, 2, 64) > 0
+    assert L.rb_gemv_workspace_bytes(14336, 4096, 2, 16) == 0
+    assert L.rb_gemv_workspace_bytes(14336, 4096, 5, 64) == 0
+    # training forward: the planes (256-byte aligned) in front of rb_gemm's workspace
+    pb = (L.rb_packed_words(4096, 4096, 2) * 4 + 255) // 256 * 256
+    assert L.rb_qat_forward_workspace_bytes(4096, 4096, 2, 2048) == pb + L.rb_gemm_workspace_bytes(4096, 4096, 2, 2048)
+    assert L.rb_qat_forward_workspace_bytes(4096, 4096, 9, 2048) == 0
+
+
+def test_codebook_size_helpers_match_the_oracle(L):
+    for c in (1, 2, 3, 255, 256, 257, 7132, 65535, 65536):
+        assert L.rb_btc_index_bits(c) == oracle.btc_index_bits(c)
+    assert L.rb_btc_index_bits(0) == 0 and L.rb_btc_index_bits(65537) == 0
+    for K, w in ((4096, 13), (544, 7), (32, 1), (8192, 16)):
+        assert L.rb_btc_row_words(K, w) == oracle.btc_row_words(K, w)
+    assert L.rb_btc_row_words(48, 13) == 0
+    assert L.rb_btc_gemv_workspace_bytes(4096, 4096) == 16 * 4096 * 4            # one partial per slice and row
+    assert L.rb_btc_gemv_batch_workspace_bytes(4096, 4096, 100) == 64 * 16 * 4096 * 4  # groups of 64 layers
+    assert L.rb_btc_encode_workspace_bytes(7132) > 65536 * 16
+    assert L.rb_btc_encode_workspace_bytes(0) == 0
 
 
 def _fake(addr):
@@ -125,6 +147,38 @@ def test_svid_argument_errors_on_host(L):
     assert L.rb_svid_greedy(a, 4, 64, 1, 20, a, a, a, 16, None) == rbw.RB_ERR_WORKSPACE
 
 
+def test_training_forward_argument_errors_on_host(L):
+    a = _fake(0x10000)
+    ws = L.rb_qat_forward_workspace_bytes(64, 256, 2, 8)
+    assert L.rb_qat_forward(None, a, a, 64, 256, 2, a, 8, a, 0, a, ws, None, 0, None) == rbw.RB_ERR_ARG
+    assert L.rb_qat_forward(a, a, a, 64, 256, 9, a, 8, a, 0, a, ws, None, 0, None) == rbw.RB_ERR_ARG
+    assert L.rb_qat_forward(a, a, a, 64, 248, 2, a, 8, a, 0, a, ws, None, 0, None) == rbw.RB_ERR_SHAPE
+    assert L.rb_qat_forward(_fake(0x10004), a, a, 64, 256, 2, a, 8, a, 0, a, ws, None, 0, None) == rbw.RB_ERR_ALIGN
+    assert L.rb_qat_forward(a, a, a, 64, 256, 2, a, 8, a, 0, a, ws - 16, None, 0, None) == rbw.RB_ERR_WORKSPACE
+
+
+def test_codebook_argument_errors_on_host(L):
+    a = _fake(0x10000)
+    lay = rbw.RbLayer(64, 256, 2, 0, 0x10000, 0x10000, 0x10000)
+    ws = L.rb_btc_encode_workspace_bytes(16)
+    enc = L.rb_btc_encode
+    assert enc(None, 0, 16, 2, a, None, a, a, ws, None) == rbw.RB_ERR_ARG
+    assert enc(ctypes.byref(lay), 2, 16, 2, a, None, a, a, ws, None) == rbw.RB_ERR_ARG        # plane >= k
+    assert enc(ctypes.byref(lay), 0, 0, 2, a, None, a, a, ws, None) == rbw.RB_ERR_ARG         # c_max
+    bad = rbw.RbLayer(64, 248, 2, 0, 0x10000, 0x10000, 0x10000)
+    assert enc(ctypes.byref(bad), 0, 16, 2, a, None, a, a, ws, None) == rbw.RB_ERR_SHAPE
+    assert enc(ctypes.byref(lay), 0, 16, 2, _fake(0x10001), None, a, a, ws, None) == rbw.RB_ERR_ALIGN
+    assert enc(ctypes.byref(lay), 0, 16, 2, a, None, a, a, ws - 16, None) == rbw.RB_ERR_WORKSPACE
+    blay = rbw.RbBtcLayer(64, 256, 2, 16, 4, 0, 0x10000, 0x10000, 0x10000, 0x10000)
+    wsg = L.rb_btc_gemv_workspace_bytes(64, 256)
+    assert L.rb_btc_gemv(None, a, a, 0, a, wsg, None, 0, None) == rbw.RB_ERR_ARG
+    wrong_w = rbw.RbBtcLayer(64, 256, 2, 16, 5, 0, 0x10000, 0x10000, 0x10000, 0x10000)
+    assert L.rb_btc_gemv(ctypes.byref(wrong_w), a, a, 0, a, wsg, None, 0, None) == rbw.RB_ERR_ARG
+    k3 = rbw.RbBtcLayer(64, 256, 3, 16, 4, 0, 0x10000, 0x10000, 0x10000, 0x10000)
+    assert L.rb_btc_gemv(ctypes.byref(k3), a, a, 0, a, wsg, None, 0, None) == rbw.RB_ERR_UNSUPPORTED
+    assert L.rb_btc_gemv(ctypes.byref(blay), a, a, 0, a, wsg - 16, None, 0, None) == rbw.RB_ERR_WORKSPACE
+
+
 @no_device
 def test_well_formed_calls_fail_loudly_without_a_device(L):
     """Calls that pass every argument check return RB_ERR_UNSUPPORTED when no
@@ -136,6 +190,10 @@ def test_well_formed_calls_fail_loudly_without_a_device(L):
         assert fn(ctypes.byref(lay), a, 1, a, 0, a, 1 << 30, None, 0, None) == rbw.RB_ERR_UNSUPPORTED
     assert L.rb_transpose_planes(ctypes.byref(lay), _fake(0x100000), None) == rbw.RB_ERR_UNSUPPORTED
     assert L.rb_svid_greedy(a, 4, 64, 1, 20, a, a, a, 1 << 20, None) == rbw.RB_ERR_UNSUPPORTED
+    assert L.rb_qat_forward(a, a, a, 64, 256, 2, a, 8, a, 0, a, 1 << 30, None, 0, None) == rbw.RB_ERR_UNSUPPORTED
+    assert L.rb_btc_encode(ctypes.byref(lay), 0, 16, 2, a, None, a, a, 1 << 30, None) == rbw.RB_ERR_UNSUPPORTED
+    blay = rbw.RbBtcLayer(64, 256, 2, 16, 4, 0, 0x10000, 0x10000, 0x10000, 0x10000)
+    assert L.rb_btc_gemv(ctypes.byref(blay), a, a, 0, a, 1 << 30, None, 0, None) == rbw.RB_ERR_UNSUPPORTED
 
 
 def test_product_does_not_import_oracle():
