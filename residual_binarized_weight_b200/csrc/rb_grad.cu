@@ -212,33 +212,50 @@ scale_grad_partial_kernel(const float* __restrict__ G, const uint32_t* __restric
 #pragma unroll
         for (int e = 0; e < 8; ++e) dh_acc[i][e] = 0.0f;
 
-    for (int j = 0; j < 32; ++j) {
-        const int64_t r = (int64_t)rb * kSgRows + warp * 32 + j;
-        if (r >= N) break;                                // warp-uniform
-        float gv[8];
-        if (col_ok) {
-            const float4 a = *reinterpret_cast<const float4*>(G + r * K + c);
-            const float4 b = *reinterpret_cast<const float4*>(G + r * K + c + 4);
-            gv[0] = a.x; gv[1] = a.y; gv[2] = a.z; gv[3] = a.w; gv[4] = b.x; gv[5] = b.y; gv[6] = b.z; gv[7] = b.w;
-        } else {
+    // U rows per step: their G, sign words and g are all in flight before any is used
+    // (four for k <= 2, fewer as the per-plane registers grow)
+    constexpr int U = KP <= 2 ? 4 : KP <= 4 ? 2 : 1;
+    for (int j0 = 0; j0 < 32; j0 += U) {
+        const int64_t r0 = (int64_t)rb * kSgRows + warp * 32 + j0;
+        if (r0 >= N) break;                               // warp-uniform
+        float gv[U][8];
+        uint32_t wd[U][KP];
+        float gi[U][KP];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) gv[e] = 0.0f;
+        for (int u = 0; u < U; ++u) {
+            const int64_t r = r0 + u;
+            const bool rok = r < N;
+            float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f), b = a;
+            if (rok && col_ok) {
+                a = *reinterpret_cast<const float4*>(G + r * K + c);
+                b = *reinterpret_cast<const float4*>(G + r * K + c + 4);
+            }
+            gv[u][0] = a.x; gv[u][1] = a.y; gv[u][2] = a.z; gv[u][3] = a.w;
+            gv[u][4] = b.x; gv[u][5] = b.y; gv[u][6] = b.z; gv[u][7] = b.w;
+#pragma unroll
+            for (int i = 0; i < KP; ++i) {
+                wd[u][i] = rok ? planes[word_offset(i, s, r, lane >> 2, S, Nt)] : 0u;
+                gi[u][i] = rok ? g[(int64_t)i * N + r] : 0.0f;
+            }
         }
 #pragma unroll
-        for (int i = 0; i < KP; ++i) {
-            const uint32_t word = planes[word_offset(i, s, r, lane >> 2, S, Nt)];
-            const uint32_t byte = (word >> ((lane & 3) * 8)) & 0xffu;
-            const float gi = g[(int64_t)i * N + r];
-            float dgp = 0.0f;
+        for (int u = 0; u < U; ++u) {
+            const int64_t r = r0 + u;
+            if (r >= N) break;                            // warp-uniform
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float v = ((byte >> e) & 1u) ? gv[e] : -gv[e];
-                dgp = fmaf(v, hv[i][e], dgp);
-                dh_acc[i][e] = fmaf(v, gi, dh_acc[i][e]);
+            for (int i = 0; i < KP; ++i) {
+                const uint32_t byte = (wd[u][i] >> ((lane & 3) * 8)) & 0xffu;
+                float dgp = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float v = ((byte >> e) & 1u) ? gv[u][e] : -gv[u][e];
+                    dgp = fmaf(v, hv[i][e], dgp);
+                    dh_acc[i][e] = fmaf(v, gi[u][i], dh_acc[i][e]);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) dgp += __shfl_xor_sync(0xffffffffu, dgp, o);
+                if (lane == 0) dg_part[((int64_t)s * KP + i) * N + r] = dgp;
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) dgp += __shfl_xor_sync(0xffffffffu, dgp, o);
-            if (lane == 0) dg_part[((int64_t)s * KP + i) * N + r] = dgp;
         }
     }
 #pragma unroll
